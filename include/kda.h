@@ -1,0 +1,134 @@
+/*
+ * kda.h -- C ABI of libkda.so, the B200 (sm_100a) Kimi Delta Attention forward pass.
+ *
+ * The operation (FlashKDA de código abierto de Moonshot AI, 7minutos.es, sections
+ * "¿Qué es la atención Kimi Delta...?" and "Debajo del capó: CUTLASS en Hopper";
+ * flags from the chunk_kda call on github.zuobiaodaohang.com "FlashKDA：用CUTLASS
+ * fused kernel 给 Kimi Delta Attention 提速 3-5 倍", section "作为 FLA 后端的用法"):
+ *
+ *   for each sequence s and head h, S (K x V, fp32) = initial_state[s,h] or 0;
+ *   for each token t of s:
+ *     qh = q_t / sqrt(|q_t|^2 + 1e-6),  kh = k_t / sqrt(|k_t|^2 + 1e-6)
+ *     b  = sigmoid(beta_t)
+ *     lam[c] = max(lower_bound, -exp(A_log[h]) * softplus(g_t[c] + dt_bias[h,c]))
+ *     S = (I - b kh kh^T) Diag(exp(lam)) S + b kh v_t^T
+ *     out_t = scale * S^T qh
+ *   final_state[s,h] = S
+ *
+ * The pages do not print the gate formula; the one above (natural log,
+ * lower_bound in [-5, 0] as the pages state) is this library's reading.
+ *
+ * Layouts: every tensor is row-major and contiguous (the pages require contiguous
+ * inputs on one GPU):
+ *   q, k, g      [B, T, H, K]  bf16      v, out  [B, T, H, V]  bf16
+ *   beta         [B, T, H]     bf16 (logits; the sigmoid is applied inside)
+ *   A_log        [H]           fp32      dt_bias [H, K]        fp32
+ *   states       [N, H, K, V]  S[k][v] at ((n*H + h)*K + k)*V + v, N = B, or
+ *                               num_seqs with cu_seqlens
+ *   cu_seqlens   [num_seqs+1]  int64, cumulative token offsets; requires B == 1,
+ *                               cu_seqlens[0] == 0 and cu_seqlens[num_seqs] == T.
+ * K = V = 128 is the only head size (the pages' current restriction).
+ *
+ * Ownership: the caller owns every buffer; the library keeps no pointer after a
+ * call returns and allocates no device memory on the kda_fwd path.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* bf16 element (raw IEEE bfloat16 bits). */
+typedef uint16_t kda_bf16;
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *kda_stream_t;
+
+/* initial_state element types */
+#define KDA_STATE_NONE 0
+#define KDA_STATE_F32 1
+#define KDA_STATE_BF16 2
+
+/* Return codes.  Every negative code except KDA_ERR_CUDA is detected on the host
+ * before anything is launched. */
+#define KDA_OK 0
+#define KDA_ERR_HEAD_DIM (-1)     /* K != 128 or V != 128 */
+#define KDA_ERR_NULL (-2)         /* a required pointer is NULL */
+#define KDA_ERR_VARLEN_BATCH (-3) /* cu_seqlens given with B != 1 */
+#define KDA_ERR_NUM_SEQS (-4)     /* cu_seqlens given with num_seqs < 1 */
+#define KDA_ERR_LOWER_BOUND (-5)  /* lower_bound outside [-5, 0] or NaN */
+#define KDA_ERR_STATE_DTYPE (-6)  /* initial_state_dtype not NONE/F32/BF16, or a
+                                     state pointer without a matching dtype */
+#define KDA_ERR_ALIGN (-7)        /* a pointer is not 16-byte aligned (4 for fp32
+                                     vectors, 8 for cu_seqlens, 2 for beta) */
+#define KDA_ERR_SHAPE (-8)        /* B < 1, T < 0, H < 1, or sizes overflow */
+#define KDA_ERR_CUDA (-9)         /* a CUDA call or launch failed */
+#define KDA_ERR_WORKSPACE (-10)   /* workspace missing or too small */
+#define KDA_ERR_DEVICE (-11)      /* no usable sm_100 device for this call */
+#define KDA_ERR_SCALE (-12)       /* scale is not finite */
+
+/*
+ * kda_fwd -- the forward/prefill pass on device buffers.
+ *
+ * q, k, v, g, beta, A_log, dt_bias, out: device pointers (layouts above).
+ * scale, lower_bound: host scalars (lower_bound in [-5, 0]).
+ * initial_state: device pointer or NULL; initial_state_dtype says KDA_STATE_F32
+ *   or KDA_STATE_BF16 (KDA_STATE_NONE when NULL).
+ * final_state: device fp32 [N,H,K,V] or NULL when not wanted.
+ * cu_seqlens: device int64 [num_seqs+1] or NULL (then B sequences of length T).
+ *   It is not read on the host (that would need a synchronisation); a sequence
+ *   of length 0 returns its initial state (or zeros) as final state and writes
+ *   no output; tokens outside [cu_seqlens[0], cu_seqlens[num_seqs]) are not
+ *   written.
+ * stream: the work is enqueued on it; the call does not synchronise.
+ * T == 0 is valid: only final_state is written.
+ * Returns KDA_OK or a negative code (see above).  Never traps the GPU.
+ */
+int kda_fwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
+            const kda_bf16 *beta, float scale, const float *A_log, const float *dt_bias,
+            float lower_bound, const void *initial_state, int initial_state_dtype,
+            float *final_state, const int64_t *cu_seqlens, int64_t num_seqs, kda_bf16 *out,
+            int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, kda_stream_t stream);
+
+/*
+ * kda_fwd_host_workspace_size -- bytes of device memory kda_fwd_host needs for a
+ * call of this shape (all inputs, out, and the states it copies).  Returns 0 for
+ * invalid sizes.
+ */
+size_t kda_fwd_host_workspace_size(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                                   int64_t num_seqs, int initial_state_dtype,
+                                   int want_final_state);
+
+/*
+ * kda_fwd_host -- the same pass on HOST buffers (end-to-end path).
+ *
+ * Every pointer except workspace is a host pointer (pinned memory gives
+ * asynchronous copies; pageable memory works but copies synchronously).  The
+ * call copies the inputs into `workspace` (a device buffer of at least
+ * kda_fwd_host_workspace_size(...) bytes, owned by the caller), runs kda_fwd on
+ * `stream`, copies out (and final_state) back, and synchronises `stream` before
+ * returning, so the host buffers are ready on return.  Same return codes as
+ * kda_fwd, plus KDA_ERR_WORKSPACE.
+ */
+int kda_fwd_host(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
+                 const kda_bf16 *beta, float scale, const float *A_log, const float *dt_bias,
+                 float lower_bound, const void *initial_state, int initial_state_dtype,
+                 float *final_state, const int64_t *cu_seqlens, int64_t num_seqs,
+                 kda_bf16 *out, int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                 void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/* Human-readable text of a return code (static storage; never NULL). */
+const char *kda_strerror(int code);
+
+/* Number of kernel launches the last successful kda_fwd call on this host
+ * thread enqueued (for launch accounting in benchmarks). */
+int kda_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

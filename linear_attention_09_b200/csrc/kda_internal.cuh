@@ -1,0 +1,28 @@
+// Internal declarations shared by the libkda host code and its kernels.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+namespace kda {
+
+constexpr int kHead = 128;  // K = V = 128 (the pages' only supported head size)
+
+// Arguments of one forward call, already validated on the host.
+struct FwdParams {
+    const __nv_bfloat16 *q, *k, *v, *g, *beta;
+    const float *A_log, *dt_bias;
+    const void *init;        // fp32 or bf16 [N,H,K,V] or nullptr
+    int init_dtype;          // KDA_STATE_*
+    float *final_state;      // fp32 [N,H,K,V] or nullptr
+    const int64_t *cu;       // [N+1] or nullptr
+    __nv_bfloat16 *out;
+    float scale, lower_bound;
+    int64_t B, T, H, N;      // N = number of sequences
+};
+
+// Kernel launchers; each returns the number of kernels it enqueued (>= 0) or a
+// negative KDA_ERR_* code.
+int launch_tokenwise(const FwdParams &p, cudaStream_t stream);
+
+}  // namespace kda
