@@ -127,6 +127,11 @@ const char *kda_strerror(int code);
  * thread enqueued (for launch accounting in benchmarks). */
 int kda_last_launch_count(void);
 
+/* Diagnostic: the error word the kernels set when one of their bounded waits
+ * gave up (0 = none; the kernel then skipped the rest of its work and returned
+ * without trapping).  Synchronous (reads device memory); reset != 0 clears it. */
+int kda_device_status(int reset);
+
 #ifdef __cplusplus
 }
 #endif

@@ -6,7 +6,7 @@ PyTorch fallback: if the library cannot be loaded, the calls raise.
 
 The functions mirror the C ABI in ``include/kda.h``:
   kda_fwd, kda_fwd_host, kda_fwd_host_workspace_size, kda_strerror,
-  kda_last_launch_count.
+  kda_last_launch_count, kda_device_status.
 """
 from __future__ import annotations
 
@@ -57,6 +57,8 @@ def lib() -> ctypes.CDLL:
             L.kda_strerror.restype = ctypes.c_char_p
             L.kda_last_launch_count.argtypes = []
             L.kda_last_launch_count.restype = I
+            L.kda_device_status.argtypes = [I]
+            L.kda_device_status.restype = I
             _lib = L
     return _lib
 
@@ -67,6 +69,11 @@ def kda_strerror(code: int) -> str:
 
 def kda_last_launch_count() -> int:
     return int(lib().kda_last_launch_count())
+
+
+def kda_device_status(reset: bool = False) -> int:
+    """Error word of the last kernels (0 = every bounded wait completed)."""
+    return int(lib().kda_device_status(int(bool(reset))))
 
 
 def kda_fwd_host_workspace_size(B, T, H, K=HEAD, V=HEAD, num_seqs=0,

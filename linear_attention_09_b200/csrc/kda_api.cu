@@ -120,6 +120,8 @@ extern "C" const char *kda_strerror(int code)
 
 extern "C" int kda_last_launch_count(void) { return g_last_launches; }
 
+extern "C" int kda_device_status(int reset) { return kda::chunked_device_error(reset != 0); }
+
 extern "C" int kda_fwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
                        const kda_bf16 *beta, float scale, const float *A_log,
                        const float *dt_bias, float lower_bound, const void *initial_state,
@@ -158,7 +160,7 @@ extern "C" int kda_fwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, 
         g_last_launches = 0;
         return KDA_OK;
     }
-    const int n = kda::launch_tokenwise(p, st);
+    const int n = kda::launch_chunked(p, st);
     if (n < 0) return n;
     g_last_launches = n;
     return KDA_OK;

@@ -1,0 +1,903 @@
+// Chunked KDA forward kernel for sm_100a (B200): tcgen05 tensor cores, TMEM, TMA.
+//
+// Operator: Kimi Delta Attention, the gated delta rule with channel-wise decay
+// described on the FlashKDA pages (7minutos.es, "¿Qué es la atención Kimi
+// Delta...?"; chunk_kda flags on github.zuobiaodaohang.com "FlashKDA：用CUTLASS
+// fused kernel 给 Kimi Delta Attention 提速 3-5 倍", section "作为 FLA 后端的用法").
+//
+// One CTA per (sequence, head).  Tokens are processed in chunks of C = 64.  For a
+// chunk starting from state S0 (K x V), with q^, k^ L2-normalised, b = sigmoid(beta),
+// lam = clamped log-decay and G the inclusive in-chunk cumulative sum of lam:
+//   A_ij = sum_c k^_i k^_j e^{G_i - G_j}   (j <  i)      decay-weighted k k^T
+//   P_ij = sum_c q^_i k^_j e^{G_i - G_j}   (j <= i)      masked q k^T
+//   T    = (I + Diag(b) A)^-1 Diag(b)                   unit-triangular solve (WY/UT form)
+//   w    = T (k^ e^G),  u = T v
+//   U    = u - w S0
+//   O    = scale [(q^ e^G) S0 + P U]
+//   S    = Diag(e^{G_last}) S0 + (k^ e^{G_last - G})^T U
+// (derivation: unrolling S_t = Diag(a_t) S_{t-1} + k^_t u_t^T with
+//  u_t = b_t (v_t - S'_t^T k^_t) inside the chunk).
+//
+// Decay factors: with lam >= -5, e^{G_i - G_j} over 64 tokens spans e^{-320}, so
+// A and P are formed in two 32-token blocks, each with a reference token r at its
+// middle: k^_i e^{G_i - G_r} and k^_j e^{G_r - G_j} stay within e^{+-80} (fp32
+// range), and the cross-block part uses the second block's reference for the
+// first block's columns.  These products run in tf32; the rest in fp16 (bounded
+// operands) or bf16 (the raw v tile with T split into a bf16 hi + lo pair).  The
+// state operand S and U are scaled by a power of two per value column before
+// the fp16 cast; the state itself stays fp32 in TMEM.
+//
+// Orientation: the inter-chunk products are computed transposed (M = value
+// column v on the 128 TMEM lanes), so S^T and U^T are tensor-core A operands
+// read straight from TMEM, and thread v owns value column v.
+#include <cuda.h>
+
+#include "kda.h"
+#include "kda_internal.cuh"
+#include "sm100.cuh"
+
+namespace kda {
+
+__device__ int g_chunk_error;  // set to a non-zero code when a bounded wait gives up
+
+namespace {
+
+using namespace sm100;
+
+constexpr int C = 64;       // chunk length
+constexpr int NT = 256;     // threads per CTA: 8 warps, two per TMEM lane quadrant
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// ---- shared memory (byte offsets from a 1024-byte aligned base) ----
+// q, k, g, v tiles arrive by TMA as 2 boxes of [64 tokens][64 channels] bf16 with
+// the 128-byte swizzle (box b holds channels 64b..64b+63).
+constexpr uint32_t SM_Q = 0;                // 16 KB
+constexpr uint32_t SM_K = 16 * 1024;        // 16 KB
+constexpr uint32_t SM_G = 32 * 1024;        // 16 KB
+constexpr uint32_t SM_V = 48 * 1024;        // 16 KB
+// A/P operands for one half of the channels (the product runs in two K rounds):
+constexpr uint32_t SM_APA = 64 * 1024;      // 32 KB  [k^ rho ; q^ rho] tf32, K-major [128][64]
+constexpr uint32_t SM_APB = 96 * 1024;      // 24 KB  [k^ sig ; k^ e^{G_47-G}] tf32, K-major [96][64]
+//   reused once the A/P product has completed (solve), then for the output tile:
+constexpr uint32_t SM_X = SM_APA;                 // fp32 [64][LST] X = (I + Diag(b) A)^-1
+constexpr uint32_t SM_L = SM_APA + 17 * 1024;     // fp32 [64][LST] Diag(b) A (strict lower)
+constexpr uint32_t SM_Y = SM_APA + 34 * 1024;     // fp32 3 x [16][16] block products
+constexpr uint32_t SM_T16 = SM_APA + 17 * 1024;   // 8 KB fp16 T, K-major [64 i][64 j] (over L)
+constexpr uint32_t SM_THI = SM_APA + 25 * 1024;   // 8 KB bf16 high part of T
+constexpr uint32_t SM_TLO = SM_APA + 33 * 1024;   // 8 KB bf16 low part of T
+constexpr uint32_t SM_O = SM_APA;                 // 16 KB bf16 output tile [64 t][128 v]
+constexpr uint32_t SM_KG = 120 * 1024;      // 16 KB  k^ e^G fp16, MN-major (M = channel, K = token)
+constexpr uint32_t SM_WQ = 136 * 1024;      // 32 KB  [w ; q^ e^G] fp16, K-major [128][128]
+constexpr uint32_t SM_KP = 168 * 1024;      // 16 KB  k^ e^{G_last - G} fp16, MN-major (K = token)
+constexpr uint32_t SM_P = 184 * 1024;       // 8 KB   P fp16, K-major [64 i][64 j]
+constexpr uint32_t SM_MISC = 192 * 1024;    // norms, beta, gamma, octant sums, maxima, barriers
+constexpr uint32_t SM_BYTES = 200 * 1024;
+constexpr uint32_t SMEM_ALLOC = SM_BYTES + 1024;  // + alignment slack
+constexpr int LST = 68;                     // row stride (floats) of the solve matrices
+
+// ---- tensor memory columns (512 allocated) ----
+constexpr uint32_t TM_S = 0;     // fp32 state S, lane v, column k            (128)
+constexpr uint32_t TM_D1 = 128;  // [w S~^T | (q^ e^G) S~^T] per lane v        (128)
+                                 //   cols 0..31 then hold U~^T (fp16 pairs)
+constexpr uint32_t TM_AP = 128;  // A/P product, lanes = rows, cols = 96      (aliases D1)
+constexpr uint32_t TM_D2 = 256;  // (k'^T U~)^T = dS^T per lane v              (128)
+constexpr uint32_t TM_SS = 256;  // S~^T fp16 pairs (A operand), 64 cols      (aliases D2)
+constexpr uint32_t TM_W = 320;   // w^T: lanes = channel, cols = token        (64)
+constexpr uint32_t TM_D3 = 384;  // (P U~)^T per lane v                        (64)
+constexpr uint32_t TM_U = 448;   // u^T: lanes = v, cols = token              (64)
+
+__device__ __forceinline__ uint32_t sw(uint32_t row, uint32_t colbyte) { return sw128_offset(row, colbyte); }
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ float2 bf2x2(uint32_t w)
+{
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w));
+}
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float lg2(float x)
+{
+    float y;
+    asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// fp32 -> tf32 with round-half-away-from-zero: the tensor core reads the upper
+// 19 bits of each 32-bit operand, so adding half a tf32 ulp first rounds.
+__device__ __forceinline__ uint32_t tf32b(float x) { return __float_as_uint(x) + 0x1000u; }
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi)
+{
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+__device__ __forceinline__ void st_u32(uint8_t *base, uint32_t off, uint32_t x)
+{
+    *reinterpret_cast<uint32_t *>(base + off) = x;
+}
+
+__device__ __forceinline__ void st_u64(uint8_t *base, uint32_t off, uint32_t lo, uint32_t hi)
+{
+    *reinterpret_cast<uint2 *>(base + off) = make_uint2(lo, hi);
+}
+
+// Power of two s >= max|x| (1 for zero): the fp16 operand x / s lies in [-1, 1].
+__device__ __forceinline__ float pow2_ceil(float m)
+{
+    if (!(m > 0.f)) return 1.f;
+    const uint32_t e = (__float_as_uint(m) >> 23) & 0xFF;  // m in [2^(e-127), 2^(e-126))
+    return __uint_as_float(min(e + 1u, 254u) << 23);
+}
+
+struct Bars {
+    uint64_t mma;  // tcgen05.commit arrivals
+    uint64_t qkg;  // TMA q, k, g tiles
+    uint64_t v;    // TMA v tile
+};
+
+struct TMaps {
+    CUtensorMap q, k, g, v;  // 2-D [tokens][H*128] bf16, box [64][64], 128-byte swizzle
+};
+
+__device__ __forceinline__ bool wait_or_flag(uint64_t *bar, uint32_t parity, int code)
+{
+    if (mbar_wait(bar, parity)) return true;
+    atomicExch(&g_chunk_error, code);
+    return false;
+}
+
+__device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *tm, uint64_t *bar,
+                                          int64_t h, int64_t tok)
+{
+    tma_load_2d(dst, tm, bar, (int32_t)(h * kHead), (int32_t)tok);
+    tma_load_2d(dst + 8192, tm, bar, (int32_t)(h * kHead + 64), (int32_t)tok);
+}
+
+// Byte offset of the bf16 pair (t, c), (t, c+1) (c even) in a TMA-loaded tile.
+__device__ __forceinline__ uint32_t tile_off(int t, int c)
+{
+    return (uint32_t)(c >> 6) * 8192u + sw(t, (c & 63) * 2);
+}
+
+__global__ void __launch_bounds__(NT, 1)
+chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+    float *rq_s = reinterpret_cast<float *>(sm + SM_MISC);
+    float *rk_s = rq_s + 64;
+    float *b_s = rk_s + 64;
+    float *gam_s = b_s + 64;      // [128]
+    float *osum = gam_s + 128;    // [8][128] octant sums of the log-decay
+    float *xmax = osum + 1024;    // [2][128] partial maxima of the two column halves
+    Bars *bars = reinterpret_cast<Bars *>(xmax + 256);
+    uint32_t *tbase_s = reinterpret_cast<uint32_t *>(bars + 1);
+    float *Lm = reinterpret_cast<float *>(sm + SM_L);
+    float *Xm = reinterpret_cast<float *>(sm + SM_X);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ln = tid & 127, hf = tid >> 7;  // TMEM lane of this thread, column half
+    const int64_t H = p.H;
+    const int64_t s = blockIdx.x / H, h = blockIdx.x % H;
+    int64_t tok0, len;
+    if (p.cu) {
+        tok0 = p.cu[s];
+        len = p.cu[s + 1] - tok0;
+        if (len < 0) len = 0;
+    } else {
+        tok0 = s * p.T;
+        len = p.T;
+    }
+    const int64_t rstride = H * kHead;  // elements between consecutive tokens of one head
+    const int nchunks = (int)((len + C - 1) / C);
+
+    if (tid == 0) {
+        mbar_init(&bars->mma, 1);
+        mbar_init(&bars->qkg, 1);
+        mbar_init(&bars->v, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tbase_s, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0 && nchunks > 0) {  // first chunk's tiles
+        mbar_arrive_expect_tx(&bars->qkg, 3 * 16384);
+        load_tile(sm + SM_Q, &tm.q, &bars->qkg, h, tok0);
+        load_tile(sm + SM_K, &tm.k, &bars->qkg, h, tok0);
+        load_tile(sm + SM_G, &tm.g, &bars->qkg, h, tok0);
+        mbar_arrive_expect_tx(&bars->v, 16384);
+        load_tile(sm + SM_V, &tm.v, &bars->v, h, tok0);
+    }
+    const uint32_t tb = *tbase_s;
+    const uint32_t lq = (uint32_t)((warp & 3) * 32) << 16;  // this warp's TMEM lane quadrant
+    uint32_t mma_phase = 0, qkg_phase = 0, v_phase = 0;
+    bool ok = true;
+
+    // ---- initial state: thread (v, half) loads S0[64 half .. 64 half + 63][v] into TMEM,
+    //      then S~^T = S / sigma (sigma: power of two >= max_k |S[k][v]|) as fp16 pairs ----
+    const size_t soff = (size_t)(s * H + h) * kHead * kHead;
+    const int vcol = ln;
+    float sigma;  // S~ = S / sigma for the current chunk
+    {
+        float mx = 0.f;
+        for (int k0 = 64 * hf; k0 < 64 * hf + 64; k0 += 16) {
+            uint32_t r[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                float x = 0.f;
+                if (p.init && p.init_dtype == KDA_STATE_F32)
+                    x = reinterpret_cast<const float *>(p.init)[soff + (size_t)(k0 + j) * kHead + vcol];
+                else if (p.init)
+                    x = bf2f(reinterpret_cast<const __nv_bfloat16 *>(p.init)[soff + (size_t)(k0 + j) * kHead + vcol]);
+                mx = fmaxf(mx, fabsf(x));
+                r[j] = __float_as_uint(x);
+            }
+            tmem_st16(tb + lq + TM_S + k0, r);
+        }
+        xmax[hf * 128 + vcol] = mx;
+        tmem_wait_st();
+        __syncthreads();
+        sigma = pow2_ceil(fmaxf(xmax[vcol], xmax[128 + vcol]));
+        const float inv = 1.f / sigma;
+        for (int k0 = 64 * hf; k0 < 64 * hf + 64; k0 += 32) {
+            uint32_t a[16], b[16], r[16];
+            tmem_ld16(tb + lq + TM_S + k0, a);
+            tmem_ld16(tb + lq + TM_S + k0 + 16, b);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                r[j] = pack_f16(__uint_as_float(a[2 * j]) * inv, __uint_as_float(a[2 * j + 1]) * inv);
+                r[8 + j] = pack_f16(__uint_as_float(b[2 * j]) * inv, __uint_as_float(b[2 * j + 1]) * inv);
+            }
+            tmem_st16(tb + lq + TM_SS + k0 / 2, r);
+        }
+        tmem_wait_st();
+    }
+
+    const float aexp = (len > 0) ? ex2(p.A_log[h] * kLog2e) : 0.f;
+
+    for (int n = 0; n < nchunks && ok; ++n) {
+        const int64_t ctok = tok0 + (int64_t)n * C;
+        const int64_t rem = len - (int64_t)n * C;
+        const int L = (int)(rem < C ? rem : C);
+        const bool has_next = n + 1 < nchunks;
+
+        ok = __syncthreads_and(wait_or_flag(&bars->qkg, qkg_phase, 6));
+        qkg_phase ^= 1;
+        if (!ok) break;
+
+        // ---- phase 1: per-token L2 norms (thread: token tid/4, channels 32 (tid%4) ..+31)
+        //      and beta ----
+        {
+            const int t = tid >> 2, qq = tid & 3;
+            float sq = 0.f, sk = 0.f;
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {  // 4 x 16 bytes = 32 channels
+                const uint32_t off = (uint32_t)(qq >> 1) * 8192u + sw(t, (qq & 1) * 64 + ch * 16);
+                const uint4 qr = *reinterpret_cast<const uint4 *>(sm + SM_Q + off);
+                const uint4 kr = *reinterpret_cast<const uint4 *>(sm + SM_K + off);
+                const uint32_t qw[4] = {qr.x, qr.y, qr.z, qr.w}, kw[4] = {kr.x, kr.y, kr.z, kr.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 qf = bf2x2(qw[e]), kf = bf2x2(kw[e]);
+                    sq += qf.x * qf.x + qf.y * qf.y;
+                    sk += kf.x * kf.x + kf.y * kf.y;
+                }
+            }
+            sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+            sk += __shfl_xor_sync(0xffffffffu, sk, 1);
+            sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+            sk += __shfl_xor_sync(0xffffffffu, sk, 2);
+            if (qq == 0) {
+                rq_s[t] = (t < L) ? rsqrtf(sq + 1e-6f) : 0.f;
+                rk_s[t] = (t < L) ? rsqrtf(sk + 1e-6f) : 0.f;
+            }
+            if (tid < C) {
+                float bb = 0.f;
+                if (tid < L) {
+                    const float x = bf2f(p.beta[(ctok + tid) * H + h]);
+                    bb = 1.f / (1.f + ex2(-x * kLog2e));
+                }
+                b_s[tid] = bb;
+            }
+        }
+        __syncthreads();
+
+        // ---- phase 2: channel pass in two rounds of 64 channels.  Thread = (channel pair
+        //      2cp, 2cp+1 of the round, token octant oc = warp: tokens 8oc..8oc+7).
+        //      Block 0 = tokens 0..31 (reference token 15), block 1 = 32..63 (reference 47).
+        {
+            const int cp = lane, oc = warp, t0 = oc * 8, blk = oc >> 2;
+            const float lb = p.lower_bound;
+            for (int round = 0; round < 2; ++round) {
+                const int c0 = 64 * round + 2 * cp;  // first channel of the pair
+                const float2 dtb = *reinterpret_cast<const float2 *>(p.dt_bias + h * kHead + c0);
+                float G0[8], G1[8];
+                float run0 = 0.f, run1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int t = t0 + j;
+                    float l0 = 0.f, l1 = 0.f;
+                    if (t < L) {
+                        const float2 g2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_G + tile_off(t, c0)));
+                        const float x0 = g2.x + dtb.x, x1 = g2.y + dtb.y;
+                        const float sp0 = fmaxf(x0, 0.f) + kLn2 * lg2(1.f + ex2(-fabsf(x0) * kLog2e));
+                        const float sp1 = fmaxf(x1, 0.f) + kLn2 * lg2(1.f + ex2(-fabsf(x1) * kLog2e));
+                        l0 = fmaxf(lb, -aexp * sp0);
+                        l1 = fmaxf(lb, -aexp * sp1);
+                    }
+                    run0 += l0;
+                    run1 += l1;
+                    G0[j] = run0;
+                    G1[j] = run1;
+                }
+                // octant sums -> chunk prefix sums and the reference values G15, G31, G47, G63
+                *reinterpret_cast<float2 *>(osum + oc * 128 + c0) = make_float2(run0, run1);
+                __syncthreads();
+                float2 os[8];
+#pragma unroll
+                for (int o = 0; o < 8; ++o) os[o] = *reinterpret_cast<const float2 *>(osum + o * 128 + c0);
+                float pre0 = 0.f, pre1 = 0.f;
+#pragma unroll
+                for (int o = 0; o < 8; ++o)
+                    if (o < oc) { pre0 += os[o].x; pre1 += os[o].y; }
+                float ref0[4], ref1[4];  // G15, G31, G47, G63 of the two channels
+                ref0[0] = os[0].x + os[1].x;
+                ref1[0] = os[0].y + os[1].y;
+#pragma unroll
+                for (int r2 = 1; r2 < 4; ++r2) {
+                    ref0[r2] = ref0[r2 - 1] + os[2 * r2].x + os[2 * r2 + 1].x;
+                    ref1[r2] = ref1[r2 - 1] + os[2 * r2].y + os[2 * r2 + 1].y;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) { G0[j] += pre0; G1[j] += pre1; }
+                if (oc == 7) {
+                    gam_s[c0] = ex2(ref0[3] * kLog2e);
+                    gam_s[c0 + 1] = ex2(ref1[3] * kLog2e);
+                }
+                // per-channel factors (each a decay over at most 32 tokens, so >= e^-160):
+                //   block 0: e^{G_t} = rho e^{G15};  e^{G31-G_t} = sig e^{G31-G15} (=: s1 <= 1)
+                //            e^{G63-G_t} = s1 e^{G63-G31};  e^{G47-G_t} = s1 e^{G47-G31}
+                //   block 1: e^{G_t} = (rho e^{G47-G31}) e^{G31};  e^{G63-G_t} = sig e^{G63-G47}
+                float Gr[2], fa[2], fb[2], fc[2], fo[2];
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const float G15 = e ? ref1[0] : ref0[0], G31 = e ? ref1[1] : ref0[1];
+                    const float G47 = e ? ref1[2] : ref0[2], G63 = e ? ref1[3] : ref0[3];
+                    Gr[e] = blk ? G47 : G15;
+                    fo[e] = ex2((G47 - G31) * kLog2e);
+                    if (blk == 0) {
+                        fa[e] = ex2(G15 * kLog2e);
+                        fb[e] = ex2((G31 - G15) * kLog2e);
+                        fc[e] = ex2((G63 - G31) * kLog2e);
+                    } else {
+                        fa[e] = fo[e];
+                        fb[e] = ex2(G31 * kLog2e);
+                        fc[e] = ex2((G63 - G47) * kLog2e);
+                    }
+                }
+                if (round == 1) {  // A/P operands of round 0 must be consumed first
+                    ok = __syncthreads_and(wait_or_flag(&bars->mma, mma_phase, 1));
+                    mma_phase ^= 1;
+                    if (!ok) break;
+                }
+                const int cl = 2 * cp;  // channel within this round's operand half
+                const uint32_t a32 = (uint32_t)(cl >> 5) * 16384u, cb32 = (uint32_t)(cl & 31) * 4u;
+                const uint32_t b32 = (uint32_t)(cl >> 5) * 12288u;
+                const uint32_t a64 = (uint32_t)(c0 >> 6) * 8192u, cb64 = (uint32_t)(c0 & 63) * 2u;
+                const uint32_t w64 = (uint32_t)(c0 >> 6) * 16384u;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int t = t0 + j;
+                    float k0 = 0.f, k1 = 0.f, q0 = 0.f, q1 = 0.f;
+                    if (t < L) {
+                        const float2 k2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_K + tile_off(t, c0)));
+                        const float2 q2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_Q + tile_off(t, c0)));
+                        const float rk = rk_s[t], rq = rq_s[t];
+                        k0 = k2.x * rk; k1 = k2.y * rk;
+                        q0 = q2.x * rq; q1 = q2.y * rq;
+                    }
+                    const float rho0 = ex2((G0[j] - Gr[0]) * kLog2e), rho1 = ex2((G1[j] - Gr[1]) * kLog2e);
+                    const float sig0 = ex2((Gr[0] - G0[j]) * kLog2e), sig1 = ex2((Gr[1] - G1[j]) * kLog2e);
+                    st_u64(sm, SM_APA + a32 + sw(t, cb32), tf32b(k0 * rho0), tf32b(k1 * rho1));
+                    st_u64(sm, SM_APA + a32 + sw(64 + t, cb32), tf32b(q0 * rho0), tf32b(q1 * rho1));
+                    st_u64(sm, SM_APB + b32 + sw(t, cb32), tf32b(k0 * sig0), tf32b(k1 * sig1));
+                    float gam0, gam1, kp0, kp1;
+                    if (blk == 0) {
+                        gam0 = rho0 * fa[0];
+                        gam1 = rho1 * fa[1];
+                        const float s10 = sig0 * fb[0], s11 = sig1 * fb[1];  // e^{G31 - G_t} <= 1
+                        kp0 = s10 * fc[0];
+                        kp1 = s11 * fc[1];
+                        st_u64(sm, SM_APB + b32 + sw(64 + t, cb32), tf32b(k0 * (s10 * fo[0])),
+                               tf32b(k1 * (s11 * fo[1])));
+                    } else {
+                        gam0 = (rho0 * fa[0]) * fb[0];
+                        gam1 = (rho1 * fa[1]) * fb[1];
+                        kp0 = sig0 * fc[0];
+                        kp1 = sig1 * fc[1];
+                    }
+                    st_u32(sm, SM_KG + a64 + sw(t, cb64), pack_f16(k0 * gam0, k1 * gam1));
+                    st_u32(sm, SM_WQ + w64 + sw(64 + t, cb64), pack_f16(q0 * gam0, q1 * gam1));
+                    st_u32(sm, SM_KP + a64 + sw(t, cb64), pack_f16(k0 * kp0, k1 * kp1));
+                }
+                fence_async_smem();
+                tc_fence_before();
+                __syncthreads();
+                tc_fence_after();
+                // A/P += [k^ rho ; q^ rho] [k^ sig ; k^ e^{G47-G}]^T over this round's 64 channels
+                if (tid == 0) {
+                    const uint32_t id = idesc(128, 96, kTF32, kTF32, false, false);
+                    const uint32_t sa = smem_u32(sm + SM_APA), sb = smem_u32(sm + SM_APB);
+#pragma unroll
+                    for (int st = 0; st < 8; ++st) {
+                        const uint64_t da = desc_sw128(sa + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024);
+                        const uint64_t db = desc_sw128(sb + (st >> 2) * 12288 + (st & 3) * 32, 16, 1024);
+                        mma_tf32_ss(tb + TM_AP, da, db, id, (round > 0 || st > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&bars->mma);
+                }
+            }
+        }
+        if (!ok) break;
+        // q, k, g tiles are consumed: prefetch the next chunk's
+        if (tid == 0 && has_next) {
+            mbar_arrive_expect_tx(&bars->qkg, 3 * 16384);
+            load_tile(sm + SM_Q, &tm.q, &bars->qkg, h, ctok + C);
+            load_tile(sm + SM_K, &tm.k, &bars->qkg, h, ctok + C);
+            load_tile(sm + SM_G, &tm.g, &bars->qkg, h, ctok + C);
+        }
+        ok = __syncthreads_and(wait_or_flag(&bars->mma, mma_phase, 1));
+        mma_phase ^= 1;
+        tc_fence_after();
+        if (!ok) break;
+
+        // ---- phase 4: select the valid blocks of the A/P product.  Thread = (row ln,
+        //      column half hf).  Rows 0..63: Diag(b) A -> fp32 (solve); rows 64..127: P -> fp16.
+        {
+            const int i = ln & 63;
+            const bool ib1 = i >= 32;
+            // columns j in [32 hf, 32 hf + 32): block-0 columns of a block-1 row sit at 64 + j
+            const uint32_t cbase = hf ? 32u : (ib1 ? 64u : 0u);
+            float d[32];
+            {
+                uint32_t u[16], w2[16];
+                tmem_ld16(tb + lq + TM_AP + cbase, u);
+                tmem_ld16(tb + lq + TM_AP + cbase + 16, w2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    d[j] = __uint_as_float(u[j]);
+                    d[16 + j] = __uint_as_float(w2[j]);
+                }
+            }
+            const int jb = 32 * hf;
+            if (ln < 64) {
+                const float bi = b_s[i];
+#pragma unroll
+                for (int j0 = 0; j0 < 32; j0 += 4) {
+                    float e4[4];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj) e4[jj] = (jb + j0 + jj < i) ? bi * d[j0 + jj] : 0.f;
+                    *reinterpret_cast<float4 *>(Lm + i * LST + jb + j0) = make_float4(e4[0], e4[1], e4[2], e4[3]);
+                }
+            } else {
+#pragma unroll
+                for (int j0 = 0; j0 < 32; j0 += 8) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int jj = 0; jj < 8; jj += 2)
+                        pk[jj / 2] = pack_f16((jb + j0 + jj <= i) ? d[j0 + jj] : 0.f,
+                                              (jb + j0 + jj + 1 <= i) ? d[j0 + jj + 1] : 0.f);
+                    *reinterpret_cast<uint4 *>(sm + SM_P + sw(i, (jb + j0) * 2)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- phase 5: X = (I + Diag(b) A)^-1 by blocked forward substitution on 16 x 16
+        //      blocks: diagonal blocks first, then X_IJ = -X_II sum_{K=J}^{I-1} L_IK X_KJ
+        //      by block diagonals; T = X Diag(b) ----
+        if (tid < 64) {
+            const int I = tid >> 4, j = tid & 15, base = 16 * I;
+            float x[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float acc = (i == j) ? 1.f : 0.f;
+                const float *Li = Lm + (base + i) * LST + base;
+#pragma unroll
+                for (int m = 0; m < i; ++m) acc -= Li[m] * x[m];
+                x[i] = acc;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) Xm[(base + i) * LST + base + j] = x[i];
+        } else {
+            // zero the blocks above the block diagonal
+            for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
+                const int blkid = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+                const int I = blkid < 3 ? 0 : (blkid < 5 ? 1 : 2);
+                const int J = blkid < 3 ? blkid + 1 : (blkid < 5 ? blkid - 1 : 3);
+                Xm[(16 * I + r) * LST + 16 * J + cc] = 0.f;
+            }
+        }
+        __syncthreads();
+        {
+            float *Ys = reinterpret_cast<float *>(sm + SM_Y);
+            for (int d = 1; d < 4; ++d) {
+                const int nblk = 4 - d;
+                const bool act = tid < 32 * nblk;
+                const int bi = tid >> 5, J = bi, I = J + d;
+                const int r = (tid & 31) >> 1, c0 = (tid & 1) * 8;
+                if (act) {
+                    float y[8];
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) y[cc] = 0.f;
+                    for (int K = J; K < I; ++K) {
+                        const float *Lr = Lm + (16 * I + r) * LST + 16 * K;
+#pragma unroll
+                        for (int m = 0; m < 16; ++m) {
+                            const float l = Lr[m];
+                            const float4 xa = *reinterpret_cast<const float4 *>(Xm + (16 * K + m) * LST + 16 * J + c0);
+                            const float4 xb = *reinterpret_cast<const float4 *>(Xm + (16 * K + m) * LST + 16 * J + c0 + 4);
+                            y[0] += l * xa.x; y[1] += l * xa.y; y[2] += l * xa.z; y[3] += l * xa.w;
+                            y[4] += l * xb.x; y[5] += l * xb.y; y[6] += l * xb.z; y[7] += l * xb.w;
+                        }
+                    }
+                    float *Yb = Ys + bi * 256 + r * 16 + c0;
+                    *reinterpret_cast<float4 *>(Yb) = make_float4(y[0], y[1], y[2], y[3]);
+                    *reinterpret_cast<float4 *>(Yb + 4) = make_float4(y[4], y[5], y[6], y[7]);
+                }
+                __syncthreads();
+                if (act) {
+                    float xo[8];
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) xo[cc] = 0.f;
+                    const float *Xr = Xm + (16 * I + r) * LST + 16 * I;
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {
+                        const float xi = Xr[m];
+                        const float4 ya = *reinterpret_cast<const float4 *>(Ys + bi * 256 + m * 16 + c0);
+                        const float4 yb = *reinterpret_cast<const float4 *>(Ys + bi * 256 + m * 16 + c0 + 4);
+                        xo[0] -= xi * ya.x; xo[1] -= xi * ya.y; xo[2] -= xi * ya.z; xo[3] -= xi * ya.w;
+                        xo[4] -= xi * yb.x; xo[5] -= xi * yb.y; xo[6] -= xi * yb.z; xo[7] -= xi * yb.w;
+                    }
+                    float *Xo = Xm + (16 * I + r) * LST + 16 * J + c0;
+                    *reinterpret_cast<float4 *>(Xo) = make_float4(xo[0], xo[1], xo[2], xo[3]);
+                    *reinterpret_cast<float4 *>(Xo + 4) = make_float4(xo[4], xo[5], xo[6], xo[7]);
+                }
+                __syncthreads();
+            }
+        }
+        // T = X Diag(b): fp16 copy (for w) and bf16 hi + lo pair (for u = T v).
+        // Thread = (row i = tid / 4, 16 columns 16 (tid % 4) ..)
+        {
+            const int i = tid >> 2, jq = (tid & 3) * 16;
+#pragma unroll
+            for (int j0 = 0; j0 < 16; j0 += 8) {
+                uint32_t p16[4], phi[4], plo[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    float tv[2];
+                    __nv_bfloat16 hv[2], lv[2];
+#pragma unroll
+                    for (int q2 = 0; q2 < 2; ++q2) {
+                        const int j = jq + j0 + e + q2;
+                        tv[q2] = Xm[i * LST + j] * b_s[j];
+                        hv[q2] = __float2bfloat16_rn(tv[q2]);
+                        lv[q2] = __float2bfloat16_rn(tv[q2] - __bfloat162float(hv[q2]));
+                    }
+                    p16[e / 2] = pack_f16(tv[0], tv[1]);
+                    __nv_bfloat162 hh2 = __halves2bfloat162(hv[0], hv[1]);
+                    __nv_bfloat162 ll2 = __halves2bfloat162(lv[0], lv[1]);
+                    phi[e / 2] = *reinterpret_cast<uint32_t *>(&hh2);
+                    plo[e / 2] = *reinterpret_cast<uint32_t *>(&ll2);
+                }
+                const uint32_t off = sw(i, (jq + j0) * 2);
+                *reinterpret_cast<uint4 *>(sm + SM_T16 + off) = make_uint4(p16[0], p16[1], p16[2], p16[3]);
+                *reinterpret_cast<uint4 *>(sm + SM_THI + off) = make_uint4(phi[0], phi[1], phi[2], phi[3]);
+                *reinterpret_cast<uint4 *>(sm + SM_TLO + off) = make_uint4(plo[0], plo[1], plo[2], plo[3]);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- phase 6: w^T = (k^ e^G)^T T^T (fp16), u^T = v^T (T_hi + T_lo)^T (bf16) ----
+        if (tid == 0) {
+            ok = wait_or_flag(&bars->v, v_phase, 2);
+            if (ok) {
+                tc_fence_after();
+                const uint32_t skg = smem_u32(sm + SM_KG), st16 = smem_u32(sm + SM_T16);
+                const uint32_t sv = smem_u32(sm + SM_V), shi = smem_u32(sm + SM_THI),
+                               slo = smem_u32(sm + SM_TLO);
+                const uint32_t idw = idesc(128, 64, kF16, kF16, true, false);
+                const uint32_t idu = idesc(128, 64, kBF16, kBF16, true, false);
+#pragma unroll
+                for (int st = 0; st < 4; ++st)
+                    mma_f16_ss(tb + TM_W, desc_sw128(skg + st * 2048, 8192, 1024),
+                               desc_sw128(st16 + st * 32, 16, 1024), idw, st > 0);
+#pragma unroll
+                for (int st = 0; st < 4; ++st)
+                    mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
+                               desc_sw128(shi + st * 32, 16, 1024), idu, st > 0);
+#pragma unroll
+                for (int st = 0; st < 4; ++st)
+                    mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
+                               desc_sw128(slo + st * 32, 16, 1024), idu, 1);
+                mma_commit(&bars->mma);
+            }
+        }
+        v_phase ^= 1;
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        ok = __syncthreads_and(wait_or_flag(&bars->mma, mma_phase, 3));
+        mma_phase ^= 1;
+        tc_fence_after();
+        if (!ok) break;
+        if (tid == 0 && has_next) {  // the v tile is consumed: prefetch the next chunk's
+            mbar_arrive_expect_tx(&bars->v, 16384);
+            load_tile(sm + SM_V, &tm.v, &bars->v, h, ctok + C);
+        }
+
+        // ---- phase 7: w (lanes = channel) -> fp16 rows of [w ; q^ e^G]; thread = (channel
+        //      ln, tokens 32 hf .. 32 hf + 31) ----
+        {
+            const int c = ln;
+            const uint32_t w64 = (uint32_t)(c >> 6) * 16384u, cb64 = (uint32_t)(c & 63) * 2u;
+            uint32_t u[16], w2[16];
+            tmem_ld16(tb + lq + TM_W + 32 * hf, u);
+            tmem_ld16(tb + lq + TM_W + 32 * hf + 16, w2);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                *reinterpret_cast<__half *>(sm + SM_WQ + w64 + sw(32 * hf + j, cb64)) = __float2half_rn(__uint_as_float(u[j]));
+                *reinterpret_cast<__half *>(sm + SM_WQ + w64 + sw(32 * hf + 16 + j, cb64)) = __float2half_rn(__uint_as_float(w2[j]));
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- phase 8a: D1 = S~^T [w ; q^ e^G]^T  (A = S~^T from TMEM) ----
+        if (tid == 0) {
+            const uint32_t swq = smem_u32(sm + SM_WQ);
+            const uint32_t id = idesc(128, 128, kF16, kF16, false, false);
+#pragma unroll
+            for (int st = 0; st < 8; ++st)
+                mma_f16_ts(tb + TM_D1, tb + TM_SS + st * 8,
+                           desc_sw128(swq + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024), id, st > 0);
+            mma_commit(&bars->mma);
+        }
+        ok = __syncthreads_and(wait_or_flag(&bars->mma, mma_phase, 4));
+        mma_phase ^= 1;
+        tc_fence_after();
+        if (!ok) break;
+
+        // ---- phase 8b: U^T = u^T - sigma D1[:, 0:64]; U~ = U / tau -> fp16 A operand.
+        //      Thread = (v, tokens 32 hf ..); tau from both halves' maxima ----
+        float tau;
+        {
+            float U[32];
+#pragma unroll
+            for (int t0 = 0; t0 < 32; t0 += 16) {
+                uint32_t a[16], b[16];
+                tmem_ld16(tb + lq + TM_D1 + 32 * hf + t0, a);
+                tmem_ld16(tb + lq + TM_U + 32 * hf + t0, b);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) U[t0 + j] = __uint_as_float(b[j]) - sigma * __uint_as_float(a[j]);
+            }
+            float mx = 0.f;
+#pragma unroll
+            for (int t = 0; t < 32; ++t) mx = fmaxf(mx, fabsf(U[t]));
+            xmax[hf * 128 + vcol] = mx;
+            tc_fence_before();
+            __syncthreads();  // every D1 column is read before U~ overwrites columns 0..31
+            tc_fence_after();
+            tau = pow2_ceil(fmaxf(xmax[vcol], xmax[128 + vcol]));
+            const float inv = 1.f / tau;
+            uint32_t r[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) r[j] = pack_f16(U[2 * j] * inv, U[2 * j + 1] * inv);
+            tmem_st16(tb + lq + TM_D1 + 16 * hf, r);
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---- phase 8c: dS^T = U~^T k' (N = 128), (P U~)^T = U~^T P^T (N = 64) ----
+        if (tid == 0) {
+            const uint32_t skp = smem_u32(sm + SM_KP), sp = smem_u32(sm + SM_P);
+            const uint32_t id2 = idesc(128, 128, kF16, kF16, false, true);
+            const uint32_t id3 = idesc(128, 64, kF16, kF16, false, false);
+#pragma unroll
+            for (int st = 0; st < 4; ++st)
+                mma_f16_ts(tb + TM_D2, tb + TM_D1 + st * 8, desc_sw128(skp + st * 2048, 8192, 1024), id2, st > 0);
+#pragma unroll
+            for (int st = 0; st < 4; ++st)
+                mma_f16_ts(tb + TM_D3, tb + TM_D1 + st * 8, desc_sw128(sp + st * 32, 16, 1024), id3, st > 0);
+            mma_commit(&bars->mma);
+        }
+        ok = __syncthreads_and(wait_or_flag(&bars->mma, mma_phase, 5));
+        mma_phase ^= 1;
+        tc_fence_after();
+        if (!ok) break;
+
+        // ---- phase 8d: O = scale (sigma D1[:, 64:128] + tau D3) -> bf16 tile in shared
+        //      memory (row t, column v), then 16-byte row stores of the valid tokens ----
+        {
+#pragma unroll
+            for (int t0 = 0; t0 < 32; t0 += 16) {
+                uint32_t a[16], b[16];
+                tmem_ld16(tb + lq + TM_D1 + 64 + 32 * hf + t0, a);
+                tmem_ld16(tb + lq + TM_D3 + 32 * hf + t0, b);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float o = p.scale * (sigma * __uint_as_float(a[j]) + tau * __uint_as_float(b[j]));
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + SM_O + (32 * hf + t0 + j) * 256 + vcol * 2) =
+                        __float2bfloat16_rn(o);
+                }
+            }
+            __syncthreads();
+            __nv_bfloat16 *ob = p.out + (ctok * H + h) * kHead;
+#pragma unroll
+            for (int e = tid; e < C * 16; e += NT) {
+                const int t = e >> 4, ch = e & 15;
+                if (t < L)
+                    *reinterpret_cast<uint4 *>(ob + (int64_t)t * rstride + ch * 8) =
+                        *reinterpret_cast<const uint4 *>(sm + SM_O + t * 256 + ch * 16);
+            }
+        }
+
+        // ---- phase 8e: S = Diag(gamma) S + tau dS; new S~ = S / sigma' -> TMEM A operand.
+        //      Thread = (v, k in 64 hf .. 64 hf + 63) ----
+        {
+            float mx = 0.f;
+#pragma unroll
+            for (int k0 = 0; k0 < 64; k0 += 16) {
+                const int kk = 64 * hf + k0;
+                uint32_t a[16], b[16];
+                tmem_ld16(tb + lq + TM_S + kk, a);
+                tmem_ld16(tb + lq + TM_D2 + kk, b);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float sn = gam_s[kk + j] * __uint_as_float(a[j]) + tau * __uint_as_float(b[j]);
+                    mx = fmaxf(mx, fabsf(sn));
+                    a[j] = __float_as_uint(sn);
+                }
+                tmem_st16(tb + lq + TM_S + kk, a);
+            }
+            tmem_wait_st();
+            xmax[hf * 128 + vcol] = mx;
+            tc_fence_before();
+            __syncthreads();  // every dS column is read before S~ overwrites columns 0..63
+            tc_fence_after();
+            sigma = pow2_ceil(fmaxf(xmax[vcol], xmax[128 + vcol]));
+            const float inv = 1.f / sigma;
+#pragma unroll
+            for (int k0 = 0; k0 < 64; k0 += 32) {
+                const int kk = 64 * hf + k0;
+                uint32_t a[16], b[16], r[16];
+                tmem_ld16(tb + lq + TM_S + kk, a);
+                tmem_ld16(tb + lq + TM_S + kk + 16, b);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    r[j] = pack_f16(__uint_as_float(a[2 * j]) * inv, __uint_as_float(a[2 * j + 1]) * inv);
+                    r[8 + j] = pack_f16(__uint_as_float(b[2 * j]) * inv, __uint_as_float(b[2 * j + 1]) * inv);
+                }
+                tmem_st16(tb + lq + TM_SS + kk / 2, r);
+            }
+            tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+
+    // ---- final state: thread (v, half) writes S[64 half .. 64 half + 63][v] ----
+    if (ok && p.final_state) {
+        float *dst = p.final_state + soff + vcol;
+        for (int k0 = 64 * hf; k0 < 64 * hf + 64; k0 += 16) {
+            uint32_t a[16];
+            tmem_ld16(tb + lq + TM_S + k0, a);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) dst[(size_t)(k0 + j) * kHead] = __uint_as_float(a[j]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tb, 512);
+}
+
+// Driver entry point for cuTensorMapEncodeTiled, resolved once through the runtime.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+}  // namespace
+
+int launch_chunked(const FwdParams &p, cudaStream_t stream)
+{
+    const int64_t ctas = p.N * p.H;
+    if (ctas <= 0) return 0;
+    if (ctas > (int64_t)INT32_MAX) return KDA_ERR_SHAPE;
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return KDA_ERR_CUDA;
+    // q, k, g, v viewed as 2-D bf16 tensors [tokens][H * 128]; box [64 tokens][64
+    // channels] with the 128-byte swizzle; rows past the end read as zeros.
+    TMaps tm;
+    const int64_t rows = p.B * p.T;
+    cuuint64_t dims[2] = {(cuuint64_t)(p.H * kHead), (cuuint64_t)(rows > 0 ? rows : 1)};
+    cuuint64_t strides[1] = {(cuuint64_t)(p.H * kHead * 2)};
+    cuuint32_t box[2] = {64, (cuuint32_t)C};
+    cuuint32_t estr[2] = {1, 1};
+    const __nv_bfloat16 *src[4] = {p.q, p.k, p.g, p.v};
+    CUtensorMap *dst[4] = {&tm.q, &tm.k, &tm.g, &tm.v};
+    for (int i = 0; i < 4; ++i) {
+        if (enc(dst[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<__nv_bfloat16 *>(src[i]),
+                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return KDA_ERR_CUDA;
+    }
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 SMEM_ALLOC) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        attr_set = true;
+    }
+    chunk_kernel<<<(unsigned)ctas, NT, SMEM_ALLOC, stream>>>(p, tm);
+    return cudaGetLastError() == cudaSuccess ? 1 : KDA_ERR_CUDA;
+}
+
+int chunked_device_error(bool reset)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_chunk_error, sizeof(int)) != cudaSuccess) return -1;
+    if (reset && v) {
+        const int z = 0;
+        cudaMemcpyToSymbol(g_chunk_error, &z, sizeof(int));
+    }
+    return v;
+}
+
+}  // namespace kda

@@ -24,5 +24,8 @@ struct FwdParams {
 // Kernel launchers; each returns the number of kernels it enqueued (>= 0) or a
 // negative KDA_ERR_* code.
 int launch_tokenwise(const FwdParams &p, cudaStream_t stream);
+int launch_chunked(const FwdParams &p, cudaStream_t stream);
+// Error word the chunked kernel sets when a bounded wait gives up (0 = none).
+int chunked_device_error(bool reset);
 
 }  // namespace kda

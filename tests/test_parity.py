@@ -30,6 +30,7 @@ def dev(inp):
 def run_gpu(inp):
     out, fin = kda.kda_fwd(**dev(inp))
     torch.cuda.synchronize()
+    assert kda.kda_device_status(reset=True) == 0, "a bounded wait in the kernel gave up"
     return out.float().cpu().numpy().astype(np.float64), fin.cpu().numpy().astype(np.float64)
 
 
