@@ -5,7 +5,10 @@
 // Delta...?"; chunk_kda flags on github.zuobiaodaohang.com "FlashKDA：用CUTLASS
 // fused kernel 给 Kimi Delta Attention 提速 3-5 倍", section "作为 FLA 后端的用法").
 //
-// One CTA per (sequence, head).  Tokens are processed in chunks of C = 64.  For a
+// One CTA per (sequence, head), two warp roles working one chunk apart: warps
+// 0..7 prepare chunk n+1 (activations, intra-chunk products, triangular solve)
+// while warps 8..11 run the sequential state pass over chunk n.  Tokens are
+// processed in chunks of C = 64.  For a
 // chunk starting from state S0 (K x V), with q^, k^ L2-normalised, b = sigmoid(beta),
 // lam = clamped log-decay and G the inclusive in-chunk cumulative sum of lam:
 //   A_ij = sum_c k^_i k^_j e^{G_i - G_j}   (j <  i)      decay-weighted k k^T
@@ -25,7 +28,8 @@
 // first block's columns.  These products run in tf32; the rest in fp16 (bounded
 // operands) or bf16 (the raw v tile with T split into a bf16 hi + lo pair).  The
 // state operand S and U are scaled by a power of two per value column before
-// the fp16 cast; the state itself stays fp32 in TMEM.
+// the fp16 cast; the state itself stays fp32 in TMEM, stored divided by the
+// current power-of-two scale of U so that the state update accumulates in place.
 //
 // Orientation: the inter-chunk products are computed transposed (M = value
 // column v on the 128 TMEM lanes), so S^T and U^T are tensor-core A operands
@@ -44,8 +48,11 @@ namespace {
 
 using namespace sm100;
 
-constexpr int C = 64;       // chunk length
-constexpr int NT = 256;     // threads per CTA: 8 warps, two per TMEM lane quadrant
+constexpr int C = 64;        // chunk length
+constexpr int NT_IN = 256;   // in-chunk warpgroups: warps 0..7
+constexpr int NT_ST = 128;   // state warpgroup: warps 8..11 (thread v <-> TMEM lane v)
+constexpr int NT = NT_IN + NT_ST;
+constexpr uint32_t BAR_IN = 1, BAR_ST = 2;  // named barriers of the two roles
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -59,33 +66,33 @@ constexpr uint32_t SM_V = 48 * 1024;        // 16 KB
 // A/P operands for one half of the channels (the product runs in two K rounds):
 constexpr uint32_t SM_APA = 64 * 1024;      // 32 KB  [k^ rho ; q^ rho] tf32, K-major [128][64]
 constexpr uint32_t SM_APB = 96 * 1024;      // 24 KB  [k^ sig ; k^ e^{G_47-G}] tf32, K-major [96][64]
-//   reused once the A/P product has completed (solve), then for the output tile:
+//   reused once the A/P product has completed (solve):
 constexpr uint32_t SM_X = SM_APA;                 // fp32 [64][LST] X = (I + Diag(b) A)^-1
 constexpr uint32_t SM_L = SM_APA + 17 * 1024;     // fp32 [64][LST] Diag(b) A (strict lower)
 constexpr uint32_t SM_Y = SM_APA + 34 * 1024;     // fp32 3 x [16][16] block products
 constexpr uint32_t SM_T16 = SM_APA + 17 * 1024;   // 8 KB fp16 T, K-major [64 i][64 j] (over L)
 constexpr uint32_t SM_THI = SM_APA + 25 * 1024;   // 8 KB bf16 high part of T
 constexpr uint32_t SM_TLO = SM_APA + 33 * 1024;   // 8 KB bf16 low part of T
-constexpr uint32_t SM_O = SM_APA;                 // 16 KB bf16 output tile [64 t][128 v]
 constexpr uint32_t SM_KG = 120 * 1024;      // 16 KB  k^ e^G fp16, MN-major (M = channel, K = token)
+// handed to the state warpgroup:
 constexpr uint32_t SM_WQ = 136 * 1024;      // 32 KB  [w ; q^ e^G] fp16, K-major [128][128]
 constexpr uint32_t SM_KP = 168 * 1024;      // 16 KB  k^ e^{G_last - G} fp16, MN-major (K = token)
 constexpr uint32_t SM_P = 184 * 1024;       // 8 KB   P fp16, K-major [64 i][64 j]
-constexpr uint32_t SM_MISC = 192 * 1024;    // norms, beta, gamma, octant sums, maxima, barriers
-constexpr uint32_t SM_BYTES = 200 * 1024;
+constexpr uint32_t SM_O = 192 * 1024;       // 16 KB  bf16 output tile [64 t][128 v] (state role)
+constexpr uint32_t SM_MISC = 208 * 1024;    // norms, beta, gamma x2, octant sums, barriers
+constexpr uint32_t SM_BYTES = 216 * 1024;
 constexpr uint32_t SMEM_ALLOC = SM_BYTES + 1024;  // + alignment slack
 constexpr int LST = 68;                     // row stride (floats) of the solve matrices
 
 // ---- tensor memory columns (512 allocated) ----
-constexpr uint32_t TM_S = 0;     // fp32 state S, lane v, column k            (128)
-constexpr uint32_t TM_D1 = 128;  // [w S~^T | (q^ e^G) S~^T] per lane v        (128)
-                                 //   cols 0..31 then hold U~^T (fp16 pairs)
-constexpr uint32_t TM_AP = 128;  // A/P product, lanes = rows, cols = 96      (aliases D1)
-constexpr uint32_t TM_D2 = 256;  // (k'^T U~)^T = dS^T per lane v              (128)
-constexpr uint32_t TM_SS = 256;  // S~^T fp16 pairs (A operand), 64 cols      (aliases D2)
-constexpr uint32_t TM_W = 320;   // w^T: lanes = channel, cols = token        (64)
-constexpr uint32_t TM_D3 = 384;  // (P U~)^T per lane v                        (64)
-constexpr uint32_t TM_U = 448;   // u^T: lanes = v, cols = token              (64)
+constexpr uint32_t TM_AP = 0;    // A/P product, lanes = rows, 96 cols        (in-chunk role)
+constexpr uint32_t TM_W = 0;     // w^T: lanes = channel, cols = token (64)   (aliases AP)
+constexpr uint32_t TM_S = 128;   // state S / tau, lane v, column k  (128)    (state role)
+constexpr uint32_t TM_D1 = 256;  // [w S~^T | (q^ e^G) S~^T] per lane v (128); cols 0..31
+                                 //   then hold U~^T (fp16 pairs)
+constexpr uint32_t TM_D3 = 384;  // (P U~)^T per lane v (64)
+constexpr uint32_t TM_SS = 384;  // S~^T fp16 pairs (A operand), 64 cols      (aliases D3)
+constexpr uint32_t TM_U = 448;   // u^T: lanes = v, cols = token (64)         (in-chunk -> state)
 
 __device__ __forceinline__ uint32_t sw(uint32_t row, uint32_t colbyte) { return sw128_offset(row, colbyte); }
 
@@ -139,13 +146,27 @@ __device__ __forceinline__ float pow2_ceil(float m)
 }
 
 struct Bars {
-    uint64_t mma;  // tcgen05.commit arrivals
-    uint64_t qkg;  // TMA q, k, g tiles
-    uint64_t v;    // TMA v tile
+    uint64_t qkg;      // TMA q, k, g tiles                    (tx bytes)
+    uint64_t v;        // TMA v tile                           (tx bytes)
+    uint64_t mma_in;   // in-chunk role's tensor-core work     (commit)
+    uint64_t mma_st;   // state role's tensor-core work        (commit)
+    uint64_t full;     // chunk operands ready for the state role (1 arrival)
+    uint64_t wq_free;  // [w ; q^ e^G] consumed                (commit)
+    uint64_t kp_free;  // k', P consumed                       (commit)
+    uint64_t u_free;   // u^T read out of TMEM                 (128 arrivals)
 };
 
 struct TMaps {
     CUtensorMap q, k, g, v;  // 2-D [tokens][H*128] bf16, box [64][64], 128-byte swizzle
+};
+
+struct Ctx {
+    uint8_t *sm;
+    float *rq_s, *rk_s, *b_s, *gam_s /* [2][128] */, *osum /* [8][128] */;
+    Bars *bars;
+    uint32_t tb;  // TMEM base
+    int64_t h, H, tok0, len, rstride;
+    int nchunks;
 };
 
 __device__ __forceinline__ bool wait_or_flag(uint64_t *bar, uint32_t parity, int code)
@@ -168,125 +189,42 @@ __device__ __forceinline__ uint32_t tile_off(int t, int c)
     return (uint32_t)(c >> 6) * 8192u + sw(t, (c & 63) * 2);
 }
 
-__global__ void __launch_bounds__(NT, 1)
-chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
+// =====================================================================================
+// In-chunk role (warps 0..7): for every chunk, the per-token activations, the
+// decay-weighted products A and P (tf32), the triangular solve for T, and the
+// products w = T (k^ e^G), u = T v; hands [w ; q^ e^G], k', P, u^T and gamma over.
+// =====================================================================================
+__device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx)
 {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
-    float *rq_s = reinterpret_cast<float *>(sm + SM_MISC);
-    float *rk_s = rq_s + 64;
-    float *b_s = rk_s + 64;
-    float *gam_s = b_s + 64;      // [128]
-    float *osum = gam_s + 128;    // [8][128] octant sums of the log-decay
-    float *xmax = osum + 1024;    // [2][128] partial maxima of the two column halves
-    Bars *bars = reinterpret_cast<Bars *>(xmax + 256);
-    uint32_t *tbase_s = reinterpret_cast<uint32_t *>(bars + 1);
+    uint8_t *sm = cx.sm;
+    Bars *bars = cx.bars;
+    const uint32_t tb = cx.tb;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int ln = tid & 127, hf = tid >> 7;
+    const uint32_t lq = (uint32_t)((warp & 3) * 32) << 16;
     float *Lm = reinterpret_cast<float *>(sm + SM_L);
     float *Xm = reinterpret_cast<float *>(sm + SM_X);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int ln = tid & 127, hf = tid >> 7;  // TMEM lane of this thread, column half
-    const int64_t H = p.H;
-    const int64_t s = blockIdx.x / H, h = blockIdx.x % H;
-    int64_t tok0, len;
-    if (p.cu) {
-        tok0 = p.cu[s];
-        len = p.cu[s + 1] - tok0;
-        if (len < 0) len = 0;
-    } else {
-        tok0 = s * p.T;
-        len = p.T;
-    }
-    const int64_t rstride = H * kHead;  // elements between consecutive tokens of one head
-    const int nchunks = (int)((len + C - 1) / C);
-
-    if (tid == 0) {
-        mbar_init(&bars->mma, 1);
-        mbar_init(&bars->qkg, 1);
-        mbar_init(&bars->v, 1);
-        fence_mbar_init();
-    }
-    if (warp == 0) {
-        tmem_alloc(tbase_s, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (tid == 0 && nchunks > 0) {  // first chunk's tiles
-        mbar_arrive_expect_tx(&bars->qkg, 3 * 16384);
-        load_tile(sm + SM_Q, &tm.q, &bars->qkg, h, tok0);
-        load_tile(sm + SM_K, &tm.k, &bars->qkg, h, tok0);
-        load_tile(sm + SM_G, &tm.g, &bars->qkg, h, tok0);
-        mbar_arrive_expect_tx(&bars->v, 16384);
-        load_tile(sm + SM_V, &tm.v, &bars->v, h, tok0);
-    }
-    const uint32_t tb = *tbase_s;
-    const uint32_t lq = (uint32_t)((warp & 3) * 32) << 16;  // this warp's TMEM lane quadrant
-    uint32_t mma_phase = 0, qkg_phase = 0, v_phase = 0;
+    const int64_t H = cx.H, h = cx.h, rstride = cx.rstride;
+    const float aexp = (cx.len > 0) ? ex2(p.A_log[h] * kLog2e) : 0.f;
+    uint32_t mma_cnt = 0;  // completed phases of bars->mma_in waited on so far
     bool ok = true;
 
-    // ---- initial state: thread (v, half) loads S0[64 half .. 64 half + 63][v] into TMEM,
-    //      then S~^T = S / sigma (sigma: power of two >= max_k |S[k][v]|) as fp16 pairs ----
-    const size_t soff = (size_t)(s * H + h) * kHead * kHead;
-    const int vcol = ln;
-    float sigma;  // S~ = S / sigma for the current chunk
-    {
-        float mx = 0.f;
-        for (int k0 = 64 * hf; k0 < 64 * hf + 64; k0 += 16) {
-            uint32_t r[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                float x = 0.f;
-                if (p.init && p.init_dtype == KDA_STATE_F32)
-                    x = reinterpret_cast<const float *>(p.init)[soff + (size_t)(k0 + j) * kHead + vcol];
-                else if (p.init)
-                    x = bf2f(reinterpret_cast<const __nv_bfloat16 *>(p.init)[soff + (size_t)(k0 + j) * kHead + vcol]);
-                mx = fmaxf(mx, fabsf(x));
-                r[j] = __float_as_uint(x);
-            }
-            tmem_st16(tb + lq + TM_S + k0, r);
-        }
-        xmax[hf * 128 + vcol] = mx;
-        tmem_wait_st();
-        __syncthreads();
-        sigma = pow2_ceil(fmaxf(xmax[vcol], xmax[128 + vcol]));
-        const float inv = 1.f / sigma;
-        for (int k0 = 64 * hf; k0 < 64 * hf + 64; k0 += 32) {
-            uint32_t a[16], b[16], r[16];
-            tmem_ld16(tb + lq + TM_S + k0, a);
-            tmem_ld16(tb + lq + TM_S + k0 + 16, b);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                r[j] = pack_f16(__uint_as_float(a[2 * j]) * inv, __uint_as_float(a[2 * j + 1]) * inv);
-                r[8 + j] = pack_f16(__uint_as_float(b[2 * j]) * inv, __uint_as_float(b[2 * j + 1]) * inv);
-            }
-            tmem_st16(tb + lq + TM_SS + k0 / 2, r);
-        }
-        tmem_wait_st();
-    }
-
-    const float aexp = (len > 0) ? ex2(p.A_log[h] * kLog2e) : 0.f;
-
-    for (int n = 0; n < nchunks && ok; ++n) {
-        const int64_t ctok = tok0 + (int64_t)n * C;
-        const int64_t rem = len - (int64_t)n * C;
+    for (int n = 0; n < cx.nchunks && ok; ++n) {
+        const int64_t ctok = cx.tok0 + (int64_t)n * C;
+        const int64_t rem = cx.len - (int64_t)n * C;
         const int L = (int)(rem < C ? rem : C);
-        const bool has_next = n + 1 < nchunks;
+        const bool has_next = n + 1 < cx.nchunks;
+        const uint32_t par = (uint32_t)n & 1u, ppar = (uint32_t)(n - 1) & 1u;
 
-        ok = __syncthreads_and(wait_or_flag(&bars->qkg, qkg_phase, 6));
-        qkg_phase ^= 1;
+        ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->qkg, par, 6));
         if (!ok) break;
 
-        // ---- phase 1: per-token L2 norms (thread: token tid/4, channels 32 (tid%4) ..+31)
-        //      and beta ----
+        // ---- norms (thread: token tid/4, channels 32 (tid%4) ..+31) and beta ----
         {
             const int t = tid >> 2, qq = tid & 3;
             float sq = 0.f, sk = 0.f;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {  // 4 x 16 bytes = 32 channels
+            for (int ch = 0; ch < 4; ++ch) {
                 const uint32_t off = (uint32_t)(qq >> 1) * 8192u + sw(t, (qq & 1) * 64 + ch * 16);
                 const uint4 qr = *reinterpret_cast<const uint4 *>(sm + SM_Q + off);
                 const uint4 kr = *reinterpret_cast<const uint4 *>(sm + SM_K + off);
@@ -303,8 +241,8 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
             sq += __shfl_xor_sync(0xffffffffu, sq, 2);
             sk += __shfl_xor_sync(0xffffffffu, sk, 2);
             if (qq == 0) {
-                rq_s[t] = (t < L) ? rsqrtf(sq + 1e-6f) : 0.f;
-                rk_s[t] = (t < L) ? rsqrtf(sk + 1e-6f) : 0.f;
+                cx.rq_s[t] = (t < L) ? rsqrtf(sq + 1e-6f) : 0.f;
+                cx.rk_s[t] = (t < L) ? rsqrtf(sk + 1e-6f) : 0.f;
             }
             if (tid < C) {
                 float bb = 0.f;
@@ -312,12 +250,12 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
                     const float x = bf2f(p.beta[(ctok + tid) * H + h]);
                     bb = 1.f / (1.f + ex2(-x * kLog2e));
                 }
-                b_s[tid] = bb;
+                cx.b_s[tid] = bb;
             }
         }
-        __syncthreads();
+        named_bar(BAR_IN, NT_IN);
 
-        // ---- phase 2: channel pass in two rounds of 64 channels.  Thread = (channel pair
+        // ---- channel pass in two rounds of 64 channels.  Thread = (channel pair
         //      2cp, 2cp+1 of the round, token octant oc = warp: tokens 8oc..8oc+7).
         //      Block 0 = tokens 0..31 (reference token 15), block 1 = 32..63 (reference 47).
         {
@@ -346,11 +284,11 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
                     G1[j] = run1;
                 }
                 // octant sums -> chunk prefix sums and the reference values G15, G31, G47, G63
-                *reinterpret_cast<float2 *>(osum + oc * 128 + c0) = make_float2(run0, run1);
-                __syncthreads();
+                *reinterpret_cast<float2 *>(cx.osum + oc * 128 + c0) = make_float2(run0, run1);
+                named_bar(BAR_IN, NT_IN);
                 float2 os[8];
 #pragma unroll
-                for (int o = 0; o < 8; ++o) os[o] = *reinterpret_cast<const float2 *>(osum + o * 128 + c0);
+                for (int o = 0; o < 8; ++o) os[o] = *reinterpret_cast<const float2 *>(cx.osum + o * 128 + c0);
                 float pre0 = 0.f, pre1 = 0.f;
 #pragma unroll
                 for (int o = 0; o < 8; ++o)
@@ -365,9 +303,9 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
                 }
 #pragma unroll
                 for (int j = 0; j < 8; ++j) { G0[j] += pre0; G1[j] += pre1; }
-                if (oc == 7) {
-                    gam_s[c0] = ex2(ref0[3] * kLog2e);
-                    gam_s[c0 + 1] = ex2(ref1[3] * kLog2e);
+                if (oc == 7) {  // gamma = e^{G63} of this chunk (double-buffered by chunk parity)
+                    cx.gam_s[par * 128 + c0] = ex2(ref0[3] * kLog2e);
+                    cx.gam_s[par * 128 + c0 + 1] = ex2(ref1[3] * kLog2e);
                 }
                 // per-channel factors (each a decay over at most 32 tokens, so >= e^-160):
                 //   block 0: e^{G_t} = rho e^{G15};  e^{G31-G_t} = sig e^{G31-G15} (=: s1 <= 1)
@@ -390,11 +328,13 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
                         fc[e] = ex2((G63 - G47) * kLog2e);
                     }
                 }
-                if (round == 1) {  // A/P operands of round 0 must be consumed first
-                    ok = __syncthreads_and(wait_or_flag(&bars->mma, mma_phase, 1));
-                    mma_phase ^= 1;
-                    if (!ok) break;
-                }
+                bool wok = true;
+                if (round == 1)  // A/P operands of round 0 must be consumed first
+                    wok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 1);
+                else if (n > 0)  // q^ e^G and k' of the previous chunk must be consumed
+                    wok = wait_or_flag(&bars->wq_free, ppar, 7) && wait_or_flag(&bars->kp_free, ppar, 8);
+                ok = named_bar_and(BAR_IN, NT_IN, wok);
+                if (!ok) break;
                 const int cl = 2 * cp;  // channel within this round's operand half
                 const uint32_t a32 = (uint32_t)(cl >> 5) * 16384u, cb32 = (uint32_t)(cl & 31) * 4u;
                 const uint32_t b32 = (uint32_t)(cl >> 5) * 12288u;
@@ -407,7 +347,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
                     if (t < L) {
                         const float2 k2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_K + tile_off(t, c0)));
                         const float2 q2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_Q + tile_off(t, c0)));
-                        const float rk = rk_s[t], rq = rq_s[t];
+                        const float rk = cx.rk_s[t], rq = cx.rq_s[t];
                         k0 = k2.x * rk; k1 = k2.y * rk;
                         q0 = q2.x * rq; q1 = q2.y * rq;
                     }
@@ -437,7 +377,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
                 }
                 fence_async_smem();
                 tc_fence_before();
-                __syncthreads();
+                named_bar(BAR_IN, NT_IN);
                 tc_fence_after();
                 // A/P += [k^ rho ; q^ rho] [k^ sig ; k^ e^{G47-G}]^T over this round's 64 channels
                 if (tid == 0) {
@@ -449,7 +389,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
                         const uint64_t db = desc_sw128(sb + (st >> 2) * 12288 + (st & 3) * 32, 16, 1024);
                         mma_tf32_ss(tb + TM_AP, da, db, id, (round > 0 || st > 0) ? 1u : 0u);
                     }
-                    mma_commit(&bars->mma);
+                    mma_commit(&bars->mma_in);
                 }
             }
         }
@@ -461,13 +401,12 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
             load_tile(sm + SM_K, &tm.k, &bars->qkg, h, ctok + C);
             load_tile(sm + SM_G, &tm.g, &bars->qkg, h, ctok + C);
         }
-        ok = __syncthreads_and(wait_or_flag(&bars->mma, mma_phase, 1));
-        mma_phase ^= 1;
+        ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 1));
         tc_fence_after();
         if (!ok) break;
 
-        // ---- phase 4: select the valid blocks of the A/P product.  Thread = (row ln,
-        //      column half hf).  Rows 0..63: Diag(b) A -> fp32 (solve); rows 64..127: P -> fp16.
+        // ---- select the valid blocks of the A/P product.  Thread = (row ln, column
+        //      half hf).  Rows 0..63: Diag(b) A -> fp32 (solve); rows 64..127: P -> fp16.
         {
             const int i = ln & 63;
             const bool ib1 = i >= 32;
@@ -487,7 +426,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
             }
             const int jb = 32 * hf;
             if (ln < 64) {
-                const float bi = b_s[i];
+                const float bi = cx.b_s[i];
 #pragma unroll
                 for (int j0 = 0; j0 < 32; j0 += 4) {
                     float e4[4];
@@ -508,12 +447,12 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
             }
         }
         tc_fence_before();
-        __syncthreads();
+        named_bar(BAR_IN, NT_IN);
         tc_fence_after();
 
-        // ---- phase 5: X = (I + Diag(b) A)^-1 by blocked forward substitution on 16 x 16
-        //      blocks: diagonal blocks first, then X_IJ = -X_II sum_{K=J}^{I-1} L_IK X_KJ
-        //      by block diagonals; T = X Diag(b) ----
+        // ---- X = (I + Diag(b) A)^-1 by blocked forward substitution on 16 x 16 blocks:
+        //      diagonal blocks first, then X_IJ = -X_II sum_{K=J}^{I-1} L_IK X_KJ by block
+        //      diagonals; T = X Diag(b) ----
         if (tid < 64) {
             const int I = tid >> 4, j = tid & 15, base = 16 * I;
             float x[16];
@@ -529,14 +468,14 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
             for (int i = 0; i < 16; ++i) Xm[(base + i) * LST + base + j] = x[i];
         } else {
             // zero the blocks above the block diagonal
-            for (int e = tid - 64; e < 6 * 256; e += NT - 64) {
+            for (int e = tid - 64; e < 6 * 256; e += NT_IN - 64) {
                 const int blkid = e >> 8, r = (e >> 4) & 15, cc = e & 15;
                 const int I = blkid < 3 ? 0 : (blkid < 5 ? 1 : 2);
                 const int J = blkid < 3 ? blkid + 1 : (blkid < 5 ? blkid - 1 : 3);
                 Xm[(16 * I + r) * LST + 16 * J + cc] = 0.f;
             }
         }
-        __syncthreads();
+        named_bar(BAR_IN, NT_IN);
         {
             float *Ys = reinterpret_cast<float *>(sm + SM_Y);
             for (int d = 1; d < 4; ++d) {
@@ -563,7 +502,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
                     *reinterpret_cast<float4 *>(Yb) = make_float4(y[0], y[1], y[2], y[3]);
                     *reinterpret_cast<float4 *>(Yb + 4) = make_float4(y[4], y[5], y[6], y[7]);
                 }
-                __syncthreads();
+                named_bar(BAR_IN, NT_IN);
                 if (act) {
                     float xo[8];
 #pragma unroll
@@ -581,7 +520,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
                     *reinterpret_cast<float4 *>(Xo) = make_float4(xo[0], xo[1], xo[2], xo[3]);
                     *reinterpret_cast<float4 *>(Xo + 4) = make_float4(xo[4], xo[5], xo[6], xo[7]);
                 }
-                __syncthreads();
+                named_bar(BAR_IN, NT_IN);
             }
         }
         // T = X Diag(b): fp16 copy (for w) and bf16 hi + lo pair (for u = T v).
@@ -598,7 +537,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
 #pragma unroll
                     for (int q2 = 0; q2 < 2; ++q2) {
                         const int j = jq + j0 + e + q2;
-                        tv[q2] = Xm[i * LST + j] * b_s[j];
+                        tv[q2] = Xm[i * LST + j] * cx.b_s[j];
                         hv[q2] = __float2bfloat16_rn(tv[q2]);
                         lv[q2] = __float2bfloat16_rn(tv[q2] - __bfloat162float(hv[q2]));
                     }
@@ -616,13 +555,14 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
+        named_bar(BAR_IN, NT_IN);
         tc_fence_after();
 
-        // ---- phase 6: w^T = (k^ e^G)^T T^T (fp16), u^T = v^T (T_hi + T_lo)^T (bf16) ----
+        // ---- w^T = (k^ e^G)^T T^T (fp16), u^T = v^T (T_hi + T_lo)^T (bf16) ----
         if (tid == 0) {
-            ok = wait_or_flag(&bars->v, v_phase, 2);
-            if (ok) {
+            bool w = wait_or_flag(&bars->v, par, 2);
+            if (w && n > 0) w = wait_or_flag(&bars->u_free, ppar, 9);  // u^T of chunk n-1 read
+            if (w) {
                 tc_fence_after();
                 const uint32_t skg = smem_u32(sm + SM_KG), st16 = smem_u32(sm + SM_T16);
                 const uint32_t sv = smem_u32(sm + SM_V), shi = smem_u32(sm + SM_THI),
@@ -641,14 +581,13 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
                 for (int st = 0; st < 4; ++st)
                     mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
                                desc_sw128(slo + st * 32, 16, 1024), idu, 1);
-                mma_commit(&bars->mma);
+                mma_commit(&bars->mma_in);
             }
+            ok = w;
         }
-        v_phase ^= 1;
-        ok = __syncthreads_and(ok);
+        ok = named_bar_and(BAR_IN, NT_IN, ok);
         if (!ok) break;
-        ok = __syncthreads_and(wait_or_flag(&bars->mma, mma_phase, 3));
-        mma_phase ^= 1;
+        ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 3));
         tc_fence_after();
         if (!ok) break;
         if (tid == 0 && has_next) {  // the v tile is consumed: prefetch the next chunk's
@@ -656,8 +595,8 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
             load_tile(sm + SM_V, &tm.v, &bars->v, h, ctok + C);
         }
 
-        // ---- phase 7: w (lanes = channel) -> fp16 rows of [w ; q^ e^G]; thread = (channel
-        //      ln, tokens 32 hf .. 32 hf + 31) ----
+        // ---- w (lanes = channel) -> fp16 rows of [w ; q^ e^G]; thread = (channel ln,
+        //      tokens 32 hf .. 32 hf + 31) ----
         {
             const int c = ln;
             const uint32_t w64 = (uint32_t)(c >> 6) * 16384u, cb64 = (uint32_t)(c & 63) * 2u;
@@ -673,163 +612,284 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
         }
         fence_async_smem();
         tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
+        named_bar(BAR_IN, NT_IN);
+        if (tid == 0) mbar_arrive(&bars->full);  // chunk n handed to the state role
+    }
+}
 
-        // ---- phase 8a: D1 = S~^T [w ; q^ e^G]^T  (A = S~^T from TMEM) ----
-        if (tid == 0) {
+// =====================================================================================
+// State role (warps 8..11, thread v <-> TMEM lane v): the sequential pass over the
+// chunks.  TMEM column block TM_S holds S / tau (tau = the scale of the current U~).
+// Per chunk:  S~ = S / sigma -> MMA1: D1 = S~^T [w ; q^ e^G]^T -> U = u - sigma D1[:,0:64]
+//   -> U~ = U / tau' -> TM_S <- (gamma * TM_S) tau / tau' -> MMA2: TM_S += U~^T k',
+//   D3 = U~^T P^T -> out = scale (sigma D1[:,64:128] + tau' D3).
+// =====================================================================================
+__device__ void state_role(const FwdParams &p, const Ctx &cx)
+{
+    uint8_t *sm = cx.sm;
+    Bars *bars = cx.bars;
+    const uint32_t tb = cx.tb;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int v = tid - NT_IN;  // value column = TMEM lane
+    const uint32_t lq = (uint32_t)((warp & 3) * 32) << 16;
+    const bool leader = (v == 0);
+    const int64_t H = cx.H, h = cx.h, rstride = cx.rstride;
+    const int64_t sidx = blockIdx.x;  // (sequence, head) unit = sequence * H + head
+    const size_t state_off = (size_t)sidx * kHead * kHead;
+    uint32_t mma_cnt = 0;
+    bool ok = true;
+
+    // initial state (column v) -> TM_S with tau = 1
+    float tau = 1.f;
+    for (int k0 = 0; k0 < kHead; k0 += 16) {
+        uint32_t r[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            float x = 0.f;
+            if (p.init && p.init_dtype == KDA_STATE_F32)
+                x = reinterpret_cast<const float *>(p.init)[state_off + (size_t)(k0 + j) * kHead + v];
+            else if (p.init)
+                x = bf2f(reinterpret_cast<const __nv_bfloat16 *>(p.init)[state_off + (size_t)(k0 + j) * kHead + v]);
+            r[j] = __float_as_uint(x);
+        }
+        tmem_st16(tb + lq + TM_S + k0, r);
+    }
+    tmem_wait_st();
+
+    for (int n = 0; n < cx.nchunks && ok; ++n) {
+        const int64_t ctok = cx.tok0 + (int64_t)n * C;
+        const int64_t rem = cx.len - (int64_t)n * C;
+        const int L = (int)(rem < C ? rem : C);
+        const uint32_t par = (uint32_t)n & 1u;
+
+        // ---- S~^T = (tau TM_S) / sigma as fp16 pairs into TM_SS ----
+        float sigma;
+        {
+            float mx = 0.f;
+#pragma unroll
+            for (int k0 = 0; k0 < kHead; k0 += 32) {
+                uint32_t a[32];
+                tmem_ld32(tb + lq + TM_S + k0, a);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) mx = fmaxf(mx, fabsf(__uint_as_float(a[j])));
+            }
+            sigma = pow2_ceil(mx * tau);
+            const float f = tau / sigma;
+#pragma unroll
+            for (int k0 = 0; k0 < kHead; k0 += 32) {
+                uint32_t a[32], r[16];
+                tmem_ld32(tb + lq + TM_S + k0, a);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    r[j] = pack_f16(__uint_as_float(a[2 * j]) * f, __uint_as_float(a[2 * j + 1]) * f);
+                tmem_st16(tb + lq + TM_SS + k0 / 2, r);
+            }
+            tmem_wait_st();
+        }
+
+        // ---- wait for the chunk's operands; MMA1: D1 = S~^T [w ; q^ e^G]^T ----
+        ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(&bars->full, par, 10));
+        if (!ok) break;
+        tc_fence_before();
+        named_bar(BAR_ST, NT_ST);
+        tc_fence_after();
+        if (leader) {
             const uint32_t swq = smem_u32(sm + SM_WQ);
             const uint32_t id = idesc(128, 128, kF16, kF16, false, false);
 #pragma unroll
             for (int st = 0; st < 8; ++st)
                 mma_f16_ts(tb + TM_D1, tb + TM_SS + st * 8,
                            desc_sw128(swq + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024), id, st > 0);
-            mma_commit(&bars->mma);
+            mma_commit(&bars->mma_st);
+            mma_commit(&bars->wq_free);
         }
-        ok = __syncthreads_and(wait_or_flag(&bars->mma, mma_phase, 4));
-        mma_phase ^= 1;
+        ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(&bars->mma_st, (mma_cnt++) & 1u, 4));
         tc_fence_after();
         if (!ok) break;
 
-        // ---- phase 8b: U^T = u^T - sigma D1[:, 0:64]; U~ = U / tau -> fp16 A operand.
-        //      Thread = (v, tokens 32 hf ..); tau from both halves' maxima ----
-        float tau;
+        // ---- U = u - sigma D1[:, 0:64]; tau' = pow2 >= max|U|; U~^T -> D1 cols 0..31 ----
+        float tau_n;
         {
-            float U[32];
+            float U[C];
 #pragma unroll
-            for (int t0 = 0; t0 < 32; t0 += 16) {
-                uint32_t a[16], b[16];
-                tmem_ld16(tb + lq + TM_D1 + 32 * hf + t0, a);
-                tmem_ld16(tb + lq + TM_U + 32 * hf + t0, b);
+            for (int t0 = 0; t0 < C; t0 += 32) {
+                uint32_t a[32], b[32];
+                tmem_ld32(tb + lq + TM_D1 + t0, a);
+                tmem_ld32(tb + lq + TM_U + t0, b);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) U[t0 + j] = __uint_as_float(b[j]) - sigma * __uint_as_float(a[j]);
+                for (int j = 0; j < 32; ++j) U[t0 + j] = __uint_as_float(b[j]) - sigma * __uint_as_float(a[j]);
             }
+            mbar_arrive(&bars->u_free);  // u^T of this chunk is out of TMEM
             float mx = 0.f;
 #pragma unroll
-            for (int t = 0; t < 32; ++t) mx = fmaxf(mx, fabsf(U[t]));
-            xmax[hf * 128 + vcol] = mx;
-            tc_fence_before();
-            __syncthreads();  // every D1 column is read before U~ overwrites columns 0..31
-            tc_fence_after();
-            tau = pow2_ceil(fmaxf(xmax[vcol], xmax[128 + vcol]));
-            const float inv = 1.f / tau;
-            uint32_t r[16];
+            for (int t = 0; t < C; ++t) mx = fmaxf(mx, fabsf(U[t]));
+            tau_n = pow2_ceil(mx);
+            const float inv = 1.f / tau_n;
 #pragma unroll
-            for (int j = 0; j < 16; ++j) r[j] = pack_f16(U[2 * j] * inv, U[2 * j + 1] * inv);
-            tmem_st16(tb + lq + TM_D1 + 16 * hf, r);
+            for (int t0 = 0; t0 < C; t0 += 32) {
+                uint32_t r[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) r[j] = pack_f16(U[t0 + 2 * j] * inv, U[t0 + 2 * j + 1] * inv);
+                tmem_st16(tb + lq + TM_D1 + t0 / 2, r);
+            }
+        }
+        // ---- TM_S <- gamma * TM_S * (tau / tau'), so that MMA2 can accumulate U~^T k' ----
+        {
+            const float f = tau / tau_n;
+            const float *gam = cx.gam_s + par * 128;
+#pragma unroll
+            for (int k0 = 0; k0 < kHead; k0 += 32) {
+                uint32_t a[32];
+                tmem_ld32(tb + lq + TM_S + k0, a);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 g4 = *reinterpret_cast<const float4 *>(gam + k0 + j);
+                    a[j] = __float_as_uint(__uint_as_float(a[j]) * (g4.x * f));
+                    a[j + 1] = __float_as_uint(__uint_as_float(a[j + 1]) * (g4.y * f));
+                    a[j + 2] = __float_as_uint(__uint_as_float(a[j + 2]) * (g4.z * f));
+                    a[j + 3] = __float_as_uint(__uint_as_float(a[j + 3]) * (g4.w * f));
+                }
+                uint32_t lo[16], hi[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) { lo[j] = a[j]; hi[j] = a[16 + j]; }
+                tmem_st16(tb + lq + TM_S + k0, lo);
+                tmem_st16(tb + lq + TM_S + k0 + 16, hi);
+            }
             tmem_wait_st();
         }
+        tau = tau_n;
         tc_fence_before();
-        __syncthreads();
+        named_bar(BAR_ST, NT_ST);
         tc_fence_after();
 
-        // ---- phase 8c: dS^T = U~^T k' (N = 128), (P U~)^T = U~^T P^T (N = 64) ----
-        if (tid == 0) {
+        // ---- MMA2: TM_S += U~^T k' (N = 128), D3 = U~^T P^T (N = 64) ----
+        if (leader) {
             const uint32_t skp = smem_u32(sm + SM_KP), sp = smem_u32(sm + SM_P);
             const uint32_t id2 = idesc(128, 128, kF16, kF16, false, true);
             const uint32_t id3 = idesc(128, 64, kF16, kF16, false, false);
 #pragma unroll
             for (int st = 0; st < 4; ++st)
-                mma_f16_ts(tb + TM_D2, tb + TM_D1 + st * 8, desc_sw128(skp + st * 2048, 8192, 1024), id2, st > 0);
+                mma_f16_ts(tb + TM_S, tb + TM_D1 + st * 8, desc_sw128(skp + st * 2048, 8192, 1024), id2, 1u);
 #pragma unroll
             for (int st = 0; st < 4; ++st)
                 mma_f16_ts(tb + TM_D3, tb + TM_D1 + st * 8, desc_sw128(sp + st * 32, 16, 1024), id3, st > 0);
-            mma_commit(&bars->mma);
+            mma_commit(&bars->mma_st);
+            mma_commit(&bars->kp_free);
         }
-        ok = __syncthreads_and(wait_or_flag(&bars->mma, mma_phase, 5));
-        mma_phase ^= 1;
+        ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(&bars->mma_st, (mma_cnt++) & 1u, 5));
         tc_fence_after();
         if (!ok) break;
 
-        // ---- phase 8d: O = scale (sigma D1[:, 64:128] + tau D3) -> bf16 tile in shared
-        //      memory (row t, column v), then 16-byte row stores of the valid tokens ----
+        // ---- out = scale (sigma D1[:, 64:128] + tau D3) -> bf16 tile -> 16-byte row stores ----
         {
 #pragma unroll
-            for (int t0 = 0; t0 < 32; t0 += 16) {
-                uint32_t a[16], b[16];
-                tmem_ld16(tb + lq + TM_D1 + 64 + 32 * hf + t0, a);
-                tmem_ld16(tb + lq + TM_D3 + 32 * hf + t0, b);
+            for (int t0 = 0; t0 < C; t0 += 32) {
+                uint32_t a[32], b[32];
+                tmem_ld32(tb + lq + TM_D1 + 64 + t0, a);
+                tmem_ld32(tb + lq + TM_D3 + t0, b);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
+                for (int j = 0; j < 32; ++j) {
                     const float o = p.scale * (sigma * __uint_as_float(a[j]) + tau * __uint_as_float(b[j]));
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + SM_O + (32 * hf + t0 + j) * 256 + vcol * 2) =
-                        __float2bfloat16_rn(o);
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + SM_O + (t0 + j) * 256 + v * 2) = __float2bfloat16_rn(o);
                 }
             }
-            __syncthreads();
+            named_bar(BAR_ST, NT_ST);
             __nv_bfloat16 *ob = p.out + (ctok * H + h) * kHead;
-#pragma unroll
-            for (int e = tid; e < C * 16; e += NT) {
+#pragma unroll 4
+            for (int e = v; e < C * 16; e += NT_ST) {
                 const int t = e >> 4, ch = e & 15;
                 if (t < L)
                     *reinterpret_cast<uint4 *>(ob + (int64_t)t * rstride + ch * 8) =
                         *reinterpret_cast<const uint4 *>(sm + SM_O + t * 256 + ch * 16);
             }
+            named_bar(BAR_ST, NT_ST);  // the tile is free for the next chunk
         }
-
-        // ---- phase 8e: S = Diag(gamma) S + tau dS; new S~ = S / sigma' -> TMEM A operand.
-        //      Thread = (v, k in 64 hf .. 64 hf + 63) ----
-        {
-            float mx = 0.f;
-#pragma unroll
-            for (int k0 = 0; k0 < 64; k0 += 16) {
-                const int kk = 64 * hf + k0;
-                uint32_t a[16], b[16];
-                tmem_ld16(tb + lq + TM_S + kk, a);
-                tmem_ld16(tb + lq + TM_D2 + kk, b);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float sn = gam_s[kk + j] * __uint_as_float(a[j]) + tau * __uint_as_float(b[j]);
-                    mx = fmaxf(mx, fabsf(sn));
-                    a[j] = __float_as_uint(sn);
-                }
-                tmem_st16(tb + lq + TM_S + kk, a);
-            }
-            tmem_wait_st();
-            xmax[hf * 128 + vcol] = mx;
-            tc_fence_before();
-            __syncthreads();  // every dS column is read before S~ overwrites columns 0..63
-            tc_fence_after();
-            sigma = pow2_ceil(fmaxf(xmax[vcol], xmax[128 + vcol]));
-            const float inv = 1.f / sigma;
-#pragma unroll
-            for (int k0 = 0; k0 < 64; k0 += 32) {
-                const int kk = 64 * hf + k0;
-                uint32_t a[16], b[16], r[16];
-                tmem_ld16(tb + lq + TM_S + kk, a);
-                tmem_ld16(tb + lq + TM_S + kk + 16, b);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    r[j] = pack_f16(__uint_as_float(a[2 * j]) * inv, __uint_as_float(a[2 * j + 1]) * inv);
-                    r[8 + j] = pack_f16(__uint_as_float(b[2 * j]) * inv, __uint_as_float(b[2 * j + 1]) * inv);
-                }
-                tmem_st16(tb + lq + TM_SS + kk / 2, r);
-            }
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
     }
 
-    // ---- final state: thread (v, half) writes S[64 half .. 64 half + 63][v] ----
+    // ---- final state = tau TM_S (column v) ----
     if (ok && p.final_state) {
-        float *dst = p.final_state + soff + vcol;
-        for (int k0 = 64 * hf; k0 < 64 * hf + 64; k0 += 16) {
-            uint32_t a[16];
-            tmem_ld16(tb + lq + TM_S + k0, a);
+        float *dst = p.final_state + state_off + v;
+        for (int k0 = 0; k0 < kHead; k0 += 32) {
+            uint32_t a[32];
+            tmem_ld32(tb + lq + TM_S + k0, a);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) dst[(size_t)(k0 + j) * kHead] = __uint_as_float(a[j]);
+            for (int j = 0; j < 32; ++j) dst[(size_t)(k0 + j) * kHead] = tau * __uint_as_float(a[j]);
         }
+    }
+}
+
+__global__ void __launch_bounds__(NT, 1)
+chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+    Ctx cx;
+    cx.sm = sm;
+    cx.rq_s = reinterpret_cast<float *>(sm + SM_MISC);
+    cx.rk_s = cx.rq_s + 64;
+    cx.b_s = cx.rk_s + 64;
+    cx.gam_s = cx.b_s + 64;     // [2][128]
+    cx.osum = cx.gam_s + 256;   // [8][128]
+    cx.bars = reinterpret_cast<Bars *>(cx.osum + 1024);
+    uint32_t *tbase_s = reinterpret_cast<uint32_t *>(cx.bars + 1);
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    cx.H = p.H;
+    const int64_t s = blockIdx.x / p.H;
+    cx.h = blockIdx.x % p.H;
+    if (p.cu) {
+        cx.tok0 = p.cu[s];
+        cx.len = p.cu[s + 1] - cx.tok0;
+        if (cx.len < 0) cx.len = 0;
+    } else {
+        cx.tok0 = s * p.T;
+        cx.len = p.T;
+    }
+    cx.rstride = p.H * kHead;
+    cx.nchunks = (int)((cx.len + C - 1) / C);
+
+    if (tid == 0) {
+        Bars *b = cx.bars;
+        mbar_init(&b->qkg, 1);
+        mbar_init(&b->v, 1);
+        mbar_init(&b->mma_in, 1);
+        mbar_init(&b->mma_st, 1);
+        mbar_init(&b->full, 1);
+        mbar_init(&b->wq_free, 1);
+        mbar_init(&b->kp_free, 1);
+        mbar_init(&b->u_free, NT_ST);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tbase_s, 512);
+        tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tb, 512);
+    tc_fence_after();
+    cx.tb = *tbase_s;
+    if (tid == 0 && cx.nchunks > 0) {  // first chunk's tiles
+        mbar_arrive_expect_tx(&cx.bars->qkg, 3 * 16384);
+        load_tile(sm + SM_Q, &tm.q, &cx.bars->qkg, cx.h, cx.tok0);
+        load_tile(sm + SM_K, &tm.k, &cx.bars->qkg, cx.h, cx.tok0);
+        load_tile(sm + SM_G, &tm.g, &cx.bars->qkg, cx.h, cx.tok0);
+        mbar_arrive_expect_tx(&cx.bars->v, 16384);
+        load_tile(sm + SM_V, &tm.v, &cx.bars->v, cx.h, cx.tok0);
+    }
+
+    if (warp < NT_IN / 32) in_chunk_role(p, tm, cx);
+    else state_role(p, cx);
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(cx.tb, 512);
 }
 
 // Driver entry point for cuTensorMapEncodeTiled, resolved once through the runtime.

@@ -234,3 +234,28 @@ __host__ __device__ constexpr uint32_t sw128_offset(uint32_t row, uint32_t col_b
 
 }  // namespace sm100
 }  // namespace kda
+
+namespace kda {
+namespace sm100 {
+
+// Named barrier over `count` threads (multiple of 32); barrier 0 is __syncthreads.
+__device__ __forceinline__ void named_bar(uint32_t id, uint32_t count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier that also returns the AND of `pred` over the participating threads.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
+}
+
+}  // namespace sm100
+}  // namespace kda
