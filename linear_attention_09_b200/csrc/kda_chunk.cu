@@ -54,7 +54,6 @@ constexpr int NT_ST = 128;   // state warpgroup: warps 8..11 (thread v <-> TMEM 
 constexpr int NT = NT_IN + NT_ST;
 constexpr uint32_t BAR_IN = 1, BAR_ST = 2;  // named barriers of the two roles
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLn2 = 0.6931471805599453f;
 
 // ---- shared memory (byte offsets from a 1024-byte aligned base) ----
 // q, k, g, v tiles arrive by TMA as 2 boxes of [64 tokens][64 channels] bf16 with
@@ -65,7 +64,7 @@ constexpr uint32_t SM_G = 32 * 1024;        // 16 KB
 constexpr uint32_t SM_V = 48 * 1024;        // 16 KB
 // A/P operands for one half of the channels (the product runs in two K rounds):
 constexpr uint32_t SM_APA = 64 * 1024;      // 32 KB  [k^ rho ; q^ rho] tf32, K-major [128][64]
-constexpr uint32_t SM_APB = 96 * 1024;      // 24 KB  [k^ sig ; k^ e^{G_47-G}] tf32, K-major [96][64]
+constexpr uint32_t SM_APB = 96 * 1024;      // 32 KB  [k^ sig ; k^ e^{G_47-G}] tf32, K-major [96(+32 pad)][64]
 //   reused once the A/P product has completed (solve):
 constexpr uint32_t SM_X = SM_APA;                 // fp32 [64][LST] X = (I + Diag(b) A)^-1
 constexpr uint32_t SM_L = SM_APA + 17 * 1024;     // fp32 [64][LST] Diag(b) A (strict lower)
@@ -73,14 +72,14 @@ constexpr uint32_t SM_Y = SM_APA + 34 * 1024;     // fp32 3 x [16][16] block pro
 constexpr uint32_t SM_T16 = SM_APA + 17 * 1024;   // 8 KB fp16 T, K-major [64 i][64 j] (over L)
 constexpr uint32_t SM_THI = SM_APA + 25 * 1024;   // 8 KB bf16 high part of T
 constexpr uint32_t SM_TLO = SM_APA + 33 * 1024;   // 8 KB bf16 low part of T
-constexpr uint32_t SM_KG = 120 * 1024;      // 16 KB  k^ e^G fp16, MN-major (M = channel, K = token)
+constexpr uint32_t SM_KG = 128 * 1024;      // 16 KB  k^ e^G fp16, MN-major (M = channel, K = token)
 // handed to the state warpgroup:
-constexpr uint32_t SM_WQ = 136 * 1024;      // 32 KB  [w ; q^ e^G] fp16, K-major [128][128]
-constexpr uint32_t SM_KP = 168 * 1024;      // 16 KB  k^ e^{G_last - G} fp16, MN-major (K = token)
-constexpr uint32_t SM_P = 184 * 1024;       // 8 KB   P fp16, K-major [64 i][64 j]
-constexpr uint32_t SM_O = 192 * 1024;       // 16 KB  bf16 output tile [64 t][128 v] (state role)
-constexpr uint32_t SM_MISC = 208 * 1024;    // norms, beta, gamma x2, octant sums, barriers
-constexpr uint32_t SM_BYTES = 216 * 1024;
+constexpr uint32_t SM_WQ = 144 * 1024;      // 32 KB  [w ; q^ e^G] fp16, K-major [128][128]
+constexpr uint32_t SM_KP = 176 * 1024;      // 16 KB  k^ e^{G_last - G} fp16, MN-major (K = token)
+constexpr uint32_t SM_P = 192 * 1024;       // 8 KB   P fp16, K-major [64 i][64 j]
+constexpr uint32_t SM_O = 200 * 1024;       // 16 KB  bf16 output tile [64 t][128 v] (state role)
+constexpr uint32_t SM_MISC = 216 * 1024;    // norms, beta, gamma x2, octant sums, barriers
+constexpr uint32_t SM_BYTES = 224 * 1024;
 constexpr uint32_t SMEM_ALLOC = SM_BYTES + 1024;  // + alignment slack
 constexpr int LST = 68;                     // row stride (floats) of the solve matrices
 
@@ -162,7 +161,7 @@ struct TMaps {
 
 struct Ctx {
     uint8_t *sm;
-    float *rq_s, *rk_s, *b_s, *gam_s /* [2][128] */, *osum /* [8][128] */;
+    float *rkq_s /* [64][2] */, *b_s, *gam_s /* [2][128] */, *osum /* [8][128] */;
     Bars *bars;
     uint32_t tb;  // TMEM base
     int64_t h, H, tok0, len, rstride;
@@ -183,12 +182,6 @@ __device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *tm, u
     tma_load_2d(dst + 8192, tm, bar, (int32_t)(h * kHead + 64), (int32_t)tok);
 }
 
-// Byte offset of the bf16 pair (t, c), (t, c+1) (c even) in a TMA-loaded tile.
-__device__ __forceinline__ uint32_t tile_off(int t, int c)
-{
-    return (uint32_t)(c >> 6) * 8192u + sw(t, (c & 63) * 2);
-}
-
 // =====================================================================================
 // In-chunk role (warps 0..7): for every chunk, the per-token activations, the
 // decay-weighted products A and P (tf32), the triangular solve for T, and the
@@ -204,10 +197,29 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
     const uint32_t lq = (uint32_t)((warp & 3) * 32) << 16;
     float *Lm = reinterpret_cast<float *>(sm + SM_L);
     float *Xm = reinterpret_cast<float *>(sm + SM_X);
-    const int64_t H = cx.H, h = cx.h, rstride = cx.rstride;
+    const int64_t H = cx.H, h = cx.h;
+    // log-decay in log2 units: lam2 = max(lb log2e, -A log2e max(x,0) - A lg2(1 + 2^(-|x| log2e)))
     const float aexp = (cx.len > 0) ? ex2(p.A_log[h] * kLog2e) : 0.f;
+    const float a2 = aexp * kLog2e, lb2 = p.lower_bound * kLog2e;
     uint32_t mma_cnt = 0;  // completed phases of bars->mma_in waited on so far
     bool ok = true;
+
+    // Channel-pass thread mapping: channel pair 2cp, 2cp+1 (of each 64-channel round),
+    // token octant oc (tokens 8oc..8oc+7; their rows have row % 8 == j).  Swizzled byte
+    // offsets of the pair in row 8oc + j, precomputed once:
+    //   o16[j]: 16-bit tiles and fp16 operands (column byte 4cp within a 128-byte row)
+    //   o32[j]: tf32 operands (column byte 8 (cp % 16) within the atom (cp / 16))
+    const int cp = lane, oc = warp, t0 = oc * 8, blk = oc >> 2;
+    uint32_t o16[8], o32[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        o16[j] = sw((uint32_t)(t0 + j), (uint32_t)cp * 4u);
+        o32[j] = (uint32_t)(cp >> 4) * 16384u + sw((uint32_t)(t0 + j), (uint32_t)(cp & 15) * 8u);
+    }
+
+    // beta logits are read one chunk ahead (thread t < 64 holds token t of the next chunk)
+    float beta_raw = 0.f;
+    if (tid < C && tid < cx.len) beta_raw = bf2f(p.beta[(cx.tok0 + tid) * H + h]);
 
     for (int n = 0; n < cx.nchunks && ok; ++n) {
         const int64_t ctok = cx.tok0 + (int64_t)n * C;
@@ -215,6 +227,9 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         const int L = (int)(rem < C ? rem : C);
         const bool has_next = n + 1 < cx.nchunks;
         const uint32_t par = (uint32_t)n & 1u, ppar = (uint32_t)(n - 1) & 1u;
+        const float beta_cur = beta_raw;
+        if (tid < C && has_next && (int64_t)(n + 1) * C + tid < cx.len)
+            beta_raw = bf2f(p.beta[(ctok + C + tid) * H + h]);
 
         ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->qkg, par, 6));
         if (!ok) break;
@@ -240,157 +255,126 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             sk += __shfl_xor_sync(0xffffffffu, sk, 1);
             sq += __shfl_xor_sync(0xffffffffu, sq, 2);
             sk += __shfl_xor_sync(0xffffffffu, sk, 2);
-            if (qq == 0) {
-                cx.rq_s[t] = (t < L) ? rsqrtf(sq + 1e-6f) : 0.f;
-                cx.rk_s[t] = (t < L) ? rsqrtf(sk + 1e-6f) : 0.f;
-            }
-            if (tid < C) {
-                float bb = 0.f;
-                if (tid < L) {
-                    const float x = bf2f(p.beta[(ctok + tid) * H + h]);
-                    bb = 1.f / (1.f + ex2(-x * kLog2e));
-                }
-                cx.b_s[tid] = bb;
-            }
+            if (qq == 0)  // (1/|k|, 1/|q|) per token, zero past the chunk end
+                *reinterpret_cast<float2 *>(cx.rkq_s + 2 * t) =
+                    (t < L) ? make_float2(rsqrtf(sk + 1e-6f), rsqrtf(sq + 1e-6f)) : make_float2(0.f, 0.f);
+            if (tid < C) cx.b_s[tid] = (tid < L) ? 1.f / (1.f + ex2(-beta_cur * kLog2e)) : 0.f;
         }
         named_bar(BAR_IN, NT_IN);
 
-        // ---- channel pass in two rounds of 64 channels.  Thread = (channel pair
-        //      2cp, 2cp+1 of the round, token octant oc = warp: tokens 8oc..8oc+7).
-        //      Block 0 = tokens 0..31 (reference token 15), block 1 = 32..63 (reference 47).
-        {
-            const int cp = lane, oc = warp, t0 = oc * 8, blk = oc >> 2;
-            const float lb = p.lower_bound;
-            for (int round = 0; round < 2; ++round) {
-                const int c0 = 64 * round + 2 * cp;  // first channel of the pair
-                const float2 dtb = *reinterpret_cast<const float2 *>(p.dt_bias + h * kHead + c0);
-                float G0[8], G1[8];
-                float run0 = 0.f, run1 = 0.f;
+        // ---- channel pass in two rounds of 64 channels.  Block 0 = tokens 0..31
+        //      (reference token 15), block 1 = tokens 32..63 (reference token 47). ----
+        for (int round = 0; round < 2; ++round) {
+            const int c0 = 64 * round + 2 * cp;  // first channel of the pair
+            const uint32_t rb = (uint32_t)round * 8192u;
+            const float2 dtb = *reinterpret_cast<const float2 *>(p.dt_bias + h * kHead + c0);
+            float2 G[8];  // in-chunk cumulative log2-decay of the pair, tokens t0 .. t0+7
+            float2 run = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int t = t0 + j;
-                    float l0 = 0.f, l1 = 0.f;
-                    if (t < L) {
-                        const float2 g2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_G + tile_off(t, c0)));
-                        const float x0 = g2.x + dtb.x, x1 = g2.y + dtb.y;
-                        const float sp0 = fmaxf(x0, 0.f) + kLn2 * lg2(1.f + ex2(-fabsf(x0) * kLog2e));
-                        const float sp1 = fmaxf(x1, 0.f) + kLn2 * lg2(1.f + ex2(-fabsf(x1) * kLog2e));
-                        l0 = fmaxf(lb, -aexp * sp0);
-                        l1 = fmaxf(lb, -aexp * sp1);
-                    }
-                    run0 += l0;
-                    run1 += l1;
-                    G0[j] = run0;
-                    G1[j] = run1;
+            for (int j = 0; j < 8; ++j) {
+                float2 l2 = make_float2(0.f, 0.f);
+                if (t0 + j < L) {
+                    const float2 g2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_G + rb + o16[j]));
+                    const float x0 = g2.x + dtb.x, x1 = g2.y + dtb.y;
+                    const float e0 = lg2(1.f + ex2(-fabsf(x0) * kLog2e));
+                    const float e1 = lg2(1.f + ex2(-fabsf(x1) * kLog2e));
+                    l2.x = fmaxf(lb2, -a2 * fmaxf(x0, 0.f) - aexp * e0);
+                    l2.y = fmaxf(lb2, -a2 * fmaxf(x1, 0.f) - aexp * e1);
                 }
-                // octant sums -> chunk prefix sums and the reference values G15, G31, G47, G63
-                *reinterpret_cast<float2 *>(cx.osum + oc * 128 + c0) = make_float2(run0, run1);
-                named_bar(BAR_IN, NT_IN);
-                float2 os[8];
+                run.x += l2.x;
+                run.y += l2.y;
+                G[j] = run;
+            }
+            // octant sums -> chunk prefix sums and the reference values G15, G31, G47, G63
+            *reinterpret_cast<float2 *>(cx.osum + oc * 128 + c0) = run;
+            named_bar(BAR_IN, NT_IN);
+            float2 os[8];
 #pragma unroll
-                for (int o = 0; o < 8; ++o) os[o] = *reinterpret_cast<const float2 *>(cx.osum + o * 128 + c0);
-                float pre0 = 0.f, pre1 = 0.f;
+            for (int o = 0; o < 8; ++o) os[o] = *reinterpret_cast<const float2 *>(cx.osum + o * 128 + c0);
+            float2 pre = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int o = 0; o < 8; ++o)
-                    if (o < oc) { pre0 += os[o].x; pre1 += os[o].y; }
-                float ref0[4], ref1[4];  // G15, G31, G47, G63 of the two channels
-                ref0[0] = os[0].x + os[1].x;
-                ref1[0] = os[0].y + os[1].y;
+            for (int o = 0; o < 8; ++o)
+                if (o < oc) { pre.x += os[o].x; pre.y += os[o].y; }
+            float2 ref[4];  // G15, G31, G47, G63 (log2 units)
+            ref[0] = make_float2(os[0].x + os[1].x, os[0].y + os[1].y);
 #pragma unroll
-                for (int r2 = 1; r2 < 4; ++r2) {
-                    ref0[r2] = ref0[r2 - 1] + os[2 * r2].x + os[2 * r2 + 1].x;
-                    ref1[r2] = ref1[r2 - 1] + os[2 * r2].y + os[2 * r2 + 1].y;
+            for (int r2 = 1; r2 < 4; ++r2)
+                ref[r2] = make_float2(ref[r2 - 1].x + os[2 * r2].x + os[2 * r2 + 1].x,
+                                      ref[r2 - 1].y + os[2 * r2].y + os[2 * r2 + 1].y);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { G[j].x += pre.x; G[j].y += pre.y; }
+            if (oc == 7)  // gamma = e^{G63} of this chunk (double-buffered by chunk parity)
+                *reinterpret_cast<float2 *>(cx.gam_s + par * 128 + c0) = make_float2(ex2(ref[3].x), ex2(ref[3].y));
+            // per-channel factors (each a decay over at most 32 tokens, so >= e^-160):
+            //   block 0: e^{G_t} = rho e^{G15};  e^{G31-G_t} = sig e^{G31-G15} (=: s1 <= 1)
+            //            e^{G63-G_t} = s1 e^{G63-G31};  e^{G47-G_t} = s1 e^{G47-G31}
+            //   block 1: e^{G_t} = rho e^{G47};  e^{G63-G_t} = sig e^{G63-G47}
+            // (e^{G15}, e^{G47} may underflow only where every factor they scale is below
+            //  e^-12 of the unit-size terms it is added to)
+            const float2 Gr = blk ? ref[2] : ref[0];
+            const float2 fo = make_float2(ex2(ref[2].x - ref[1].x), ex2(ref[2].y - ref[1].y));
+            const float2 fa = make_float2(ex2(Gr.x), ex2(Gr.y));
+            float2 fb = make_float2(1.f, 1.f), fc;
+            if (blk == 0) {
+                fb = make_float2(ex2(ref[1].x - ref[0].x), ex2(ref[1].y - ref[0].y));
+                fc = make_float2(ex2(ref[3].x - ref[1].x), ex2(ref[3].y - ref[1].y));
+            } else {
+                fc = make_float2(ex2(ref[3].x - ref[2].x), ex2(ref[3].y - ref[2].y));
+            }
+            bool wok = true;
+            if (round == 1)  // A/P operands of round 0 must be consumed first
+                wok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 1);
+            else if (n > 0)  // q^ e^G and k' of the previous chunk must be consumed
+                wok = wait_or_flag(&bars->wq_free, ppar, 7) && wait_or_flag(&bars->kp_free, ppar, 8);
+            ok = named_bar_and(BAR_IN, NT_IN, wok);
+            if (!ok) break;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float2 kk = make_float2(0.f, 0.f), qv = make_float2(0.f, 0.f);
+                if (t0 + j < L) {
+                    const float2 rkq = *reinterpret_cast<const float2 *>(cx.rkq_s + 2 * (t0 + j));
+                    kk = mul2(bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_K + rb + o16[j])),
+                              make_float2(rkq.x, rkq.x));
+                    qv = mul2(bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_Q + rb + o16[j])),
+                              make_float2(rkq.y, rkq.y));
                 }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) { G0[j] += pre0; G1[j] += pre1; }
-                if (oc == 7) {  // gamma = e^{G63} of this chunk (double-buffered by chunk parity)
-                    cx.gam_s[par * 128 + c0] = ex2(ref0[3] * kLog2e);
-                    cx.gam_s[par * 128 + c0 + 1] = ex2(ref1[3] * kLog2e);
+                const float d0 = G[j].x - Gr.x, d1 = G[j].y - Gr.y;
+                const float2 rho = make_float2(ex2(d0), ex2(d1));
+                const float2 sig = make_float2(ex2(-d0), ex2(-d1));
+                const float2 kr = mul2(kk, rho), qr = mul2(qv, rho), ks = mul2(kk, sig);
+                st_u64(sm, SM_APA + o32[j], tf32b(kr.x), tf32b(kr.y));
+                st_u64(sm, SM_APA + 8192 + o32[j], tf32b(qr.x), tf32b(qr.y));
+                st_u64(sm, SM_APB + o32[j], tf32b(ks.x), tf32b(ks.y));
+                const float2 gam = mul2(rho, fa);
+                float2 kp;
+                if (blk == 0) {
+                    const float2 s1 = mul2(sig, fb);  // e^{G31 - G_t} <= 1
+                    kp = mul2(s1, fc);
+                    const float2 ko = mul2(kk, mul2(s1, fo));
+                    st_u64(sm, SM_APB + 8192 + o32[j], tf32b(ko.x), tf32b(ko.y));
+                } else {
+                    kp = mul2(sig, fc);
                 }
-                // per-channel factors (each a decay over at most 32 tokens, so >= e^-160):
-                //   block 0: e^{G_t} = rho e^{G15};  e^{G31-G_t} = sig e^{G31-G15} (=: s1 <= 1)
-                //            e^{G63-G_t} = s1 e^{G63-G31};  e^{G47-G_t} = s1 e^{G47-G31}
-                //   block 1: e^{G_t} = (rho e^{G47-G31}) e^{G31};  e^{G63-G_t} = sig e^{G63-G47}
-                float Gr[2], fa[2], fb[2], fc[2], fo[2];
+                const float2 kg = mul2(kk, gam), qg = mul2(qv, gam), kpp = mul2(kk, kp);
+                st_u32(sm, SM_KG + rb + o16[j], pack_f16(kg.x, kg.y));
+                st_u32(sm, SM_WQ + 2 * rb + 8192 + o16[j], pack_f16(qg.x, qg.y));
+                st_u32(sm, SM_KP + rb + o16[j], pack_f16(kpp.x, kpp.y));
+            }
+            fence_async_smem();
+            tc_fence_before();
+            named_bar(BAR_IN, NT_IN);
+            tc_fence_after();
+            // A/P += [k^ rho ; q^ rho] [k^ sig ; k^ e^{G47-G}]^T over this round's 64 channels
+            if (tid == 0) {
+                const uint32_t id = idesc(128, 96, kTF32, kTF32, false, false);
+                const uint32_t sa = smem_u32(sm + SM_APA), sb = smem_u32(sm + SM_APB);
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const float G15 = e ? ref1[0] : ref0[0], G31 = e ? ref1[1] : ref0[1];
-                    const float G47 = e ? ref1[2] : ref0[2], G63 = e ? ref1[3] : ref0[3];
-                    Gr[e] = blk ? G47 : G15;
-                    fo[e] = ex2((G47 - G31) * kLog2e);
-                    if (blk == 0) {
-                        fa[e] = ex2(G15 * kLog2e);
-                        fb[e] = ex2((G31 - G15) * kLog2e);
-                        fc[e] = ex2((G63 - G31) * kLog2e);
-                    } else {
-                        fa[e] = fo[e];
-                        fb[e] = ex2(G31 * kLog2e);
-                        fc[e] = ex2((G63 - G47) * kLog2e);
-                    }
+                for (int st = 0; st < 8; ++st) {
+                    const uint64_t da = desc_sw128(sa + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024);
+                    const uint64_t db = desc_sw128(sb + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024);
+                    mma_tf32_ss(tb + TM_AP, da, db, id, (round > 0 || st > 0) ? 1u : 0u);
                 }
-                bool wok = true;
-                if (round == 1)  // A/P operands of round 0 must be consumed first
-                    wok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 1);
-                else if (n > 0)  // q^ e^G and k' of the previous chunk must be consumed
-                    wok = wait_or_flag(&bars->wq_free, ppar, 7) && wait_or_flag(&bars->kp_free, ppar, 8);
-                ok = named_bar_and(BAR_IN, NT_IN, wok);
-                if (!ok) break;
-                const int cl = 2 * cp;  // channel within this round's operand half
-                const uint32_t a32 = (uint32_t)(cl >> 5) * 16384u, cb32 = (uint32_t)(cl & 31) * 4u;
-                const uint32_t b32 = (uint32_t)(cl >> 5) * 12288u;
-                const uint32_t a64 = (uint32_t)(c0 >> 6) * 8192u, cb64 = (uint32_t)(c0 & 63) * 2u;
-                const uint32_t w64 = (uint32_t)(c0 >> 6) * 16384u;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int t = t0 + j;
-                    float k0 = 0.f, k1 = 0.f, q0 = 0.f, q1 = 0.f;
-                    if (t < L) {
-                        const float2 k2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_K + tile_off(t, c0)));
-                        const float2 q2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_Q + tile_off(t, c0)));
-                        const float rk = cx.rk_s[t], rq = cx.rq_s[t];
-                        k0 = k2.x * rk; k1 = k2.y * rk;
-                        q0 = q2.x * rq; q1 = q2.y * rq;
-                    }
-                    const float rho0 = ex2((G0[j] - Gr[0]) * kLog2e), rho1 = ex2((G1[j] - Gr[1]) * kLog2e);
-                    const float sig0 = ex2((Gr[0] - G0[j]) * kLog2e), sig1 = ex2((Gr[1] - G1[j]) * kLog2e);
-                    st_u64(sm, SM_APA + a32 + sw(t, cb32), tf32b(k0 * rho0), tf32b(k1 * rho1));
-                    st_u64(sm, SM_APA + a32 + sw(64 + t, cb32), tf32b(q0 * rho0), tf32b(q1 * rho1));
-                    st_u64(sm, SM_APB + b32 + sw(t, cb32), tf32b(k0 * sig0), tf32b(k1 * sig1));
-                    float gam0, gam1, kp0, kp1;
-                    if (blk == 0) {
-                        gam0 = rho0 * fa[0];
-                        gam1 = rho1 * fa[1];
-                        const float s10 = sig0 * fb[0], s11 = sig1 * fb[1];  // e^{G31 - G_t} <= 1
-                        kp0 = s10 * fc[0];
-                        kp1 = s11 * fc[1];
-                        st_u64(sm, SM_APB + b32 + sw(64 + t, cb32), tf32b(k0 * (s10 * fo[0])),
-                               tf32b(k1 * (s11 * fo[1])));
-                    } else {
-                        gam0 = (rho0 * fa[0]) * fb[0];
-                        gam1 = (rho1 * fa[1]) * fb[1];
-                        kp0 = sig0 * fc[0];
-                        kp1 = sig1 * fc[1];
-                    }
-                    st_u32(sm, SM_KG + a64 + sw(t, cb64), pack_f16(k0 * gam0, k1 * gam1));
-                    st_u32(sm, SM_WQ + w64 + sw(64 + t, cb64), pack_f16(q0 * gam0, q1 * gam1));
-                    st_u32(sm, SM_KP + a64 + sw(t, cb64), pack_f16(k0 * kp0, k1 * kp1));
-                }
-                fence_async_smem();
-                tc_fence_before();
-                named_bar(BAR_IN, NT_IN);
-                tc_fence_after();
-                // A/P += [k^ rho ; q^ rho] [k^ sig ; k^ e^{G47-G}]^T over this round's 64 channels
-                if (tid == 0) {
-                    const uint32_t id = idesc(128, 96, kTF32, kTF32, false, false);
-                    const uint32_t sa = smem_u32(sm + SM_APA), sb = smem_u32(sm + SM_APB);
-#pragma unroll
-                    for (int st = 0; st < 8; ++st) {
-                        const uint64_t da = desc_sw128(sa + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024);
-                        const uint64_t db = desc_sw128(sb + (st >> 2) * 12288 + (st & 3) * 32, 16, 1024);
-                        mma_tf32_ss(tb + TM_AP, da, db, id, (round > 0 || st > 0) ? 1u : 0u);
-                    }
-                    mma_commit(&bars->mma_in);
-                }
+                mma_commit(&bars->mma_in);
             }
         }
         if (!ok) break;
@@ -414,15 +398,11 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             const uint32_t cbase = hf ? 32u : (ib1 ? 64u : 0u);
             float d[32];
             {
-                uint32_t u[16], w2[16];
-                tmem_ld16(tb + lq + TM_AP + cbase, u);
-                tmem_ld16(tb + lq + TM_AP + cbase + 16, w2);
+                uint32_t u[32];
+                tmem_ld32(tb + lq + TM_AP + cbase, u);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    d[j] = __uint_as_float(u[j]);
-                    d[16 + j] = __uint_as_float(w2[j]);
-                }
+                for (int j = 0; j < 32; ++j) d[j] = __uint_as_float(u[j]);
             }
             const int jb = 32 * hf;
             if (ln < 64) {
@@ -450,19 +430,24 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         named_bar(BAR_IN, NT_IN);
         tc_fence_after();
 
-        // ---- X = (I + Diag(b) A)^-1 by blocked forward substitution on 16 x 16 blocks:
-        //      diagonal blocks first, then X_IJ = -X_II sum_{K=J}^{I-1} L_IK X_KJ by block
-        //      diagonals; T = X Diag(b) ----
+        // ---- X = (I + Diag(b) A)^-1 by blocked forward substitution on 16 x 16 blocks.
+        //      Diagonal blocks: thread = (block I, column j), row sums split four ways.
         if (tid < 64) {
             const int I = tid >> 4, j = tid & 15, base = 16 * I;
             float x[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                float acc = (i == j) ? 1.f : 0.f;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
                 const float *Li = Lm + (base + i) * LST + base;
 #pragma unroll
-                for (int m = 0; m < i; ++m) acc -= Li[m] * x[m];
-                x[i] = acc;
+                for (int m0 = 0; m0 < i; m0 += 4) {
+                    const float4 l4 = *reinterpret_cast<const float4 *>(Li + m0);
+                    acc[0] += l4.x * x[m0];
+                    if (m0 + 1 < i) acc[1] += l4.y * x[m0 + 1];
+                    if (m0 + 2 < i) acc[2] += l4.z * x[m0 + 2];
+                    if (m0 + 3 < i) acc[3] += l4.w * x[m0 + 3];
+                }
+                x[i] = ((i == j) ? 1.f : 0.f) - ((acc[0] + acc[1]) + (acc[2] + acc[3]));
             }
 #pragma unroll
             for (int i = 0; i < 16; ++i) Xm[(base + i) * LST + base + j] = x[i];
@@ -476,49 +461,92 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             }
         }
         named_bar(BAR_IN, NT_IN);
+        //      Off-diagonal blocks by block diagonals d = I - J: warp (d, J) computes
+        //      Y = sum_{K=J}^{I-1} L_IK X_KJ, then X_IJ = -X_II Y, on the tensor cores
+        //      (m16n8k8 tf32 with the 3-pass hi/lo split: fp32-accurate products).
         {
             float *Ys = reinterpret_cast<float *>(sm + SM_Y);
+            const int g = lane >> 2, tq = lane & 3;
             for (int d = 1; d < 4; ++d) {
-                const int nblk = 4 - d;
-                const bool act = tid < 32 * nblk;
-                const int bi = tid >> 5, J = bi, I = J + d;
-                const int r = (tid & 31) >> 1, c0 = (tid & 1) * 8;
-                if (act) {
-                    float y[8];
+                if (warp < 4 - d) {
+                    const int J = warp, I = J + d;
+                    float acc[2][4];
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) y[cc] = 0.f;
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+                    // Y = sum_K L_IK X_KJ
                     for (int K = J; K < I; ++K) {
-                        const float *Lr = Lm + (16 * I + r) * LST + 16 * K;
 #pragma unroll
-                        for (int m = 0; m < 16; ++m) {
-                            const float l = Lr[m];
-                            const float4 xa = *reinterpret_cast<const float4 *>(Xm + (16 * K + m) * LST + 16 * J + c0);
-                            const float4 xb = *reinterpret_cast<const float4 *>(Xm + (16 * K + m) * LST + 16 * J + c0 + 4);
-                            y[0] += l * xa.x; y[1] += l * xa.y; y[2] += l * xa.z; y[3] += l * xa.w;
-                            y[4] += l * xb.x; y[5] += l * xb.y; y[6] += l * xb.z; y[7] += l * xb.w;
+                        for (int ks = 0; ks < 2; ++ks) {
+                            const float *La = Lm + (16 * I + g) * LST + 16 * K + 8 * ks + tq;
+                            const float av[4] = {La[0], La[8 * LST], La[4], La[8 * LST + 4]};
+                            uint32_t ah[4], al[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                ah[e] = cvt_tf32(av[e]);
+                                al[e] = cvt_tf32(av[e] - __uint_as_float(ah[e]));
+                            }
+#pragma unroll
+                            for (int nt = 0; nt < 2; ++nt) {
+                                const float *Xb = Xm + (16 * K + 8 * ks + tq) * LST + 16 * J + 8 * nt + g;
+                                const float bv[2] = {Xb[0], Xb[4 * LST]};
+                                uint32_t bh[2], bl[2];
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    bh[e] = cvt_tf32(bv[e]);
+                                    bl[e] = cvt_tf32(bv[e] - __uint_as_float(bh[e]));
+                                }
+                                mma_tf32_16x8x8(acc[nt], al, bh);
+                                mma_tf32_16x8x8(acc[nt], ah, bl);
+                                mma_tf32_16x8x8(acc[nt], ah, bh);
+                            }
                         }
                     }
-                    float *Yb = Ys + bi * 256 + r * 16 + c0;
-                    *reinterpret_cast<float4 *>(Yb) = make_float4(y[0], y[1], y[2], y[3]);
-                    *reinterpret_cast<float4 *>(Yb + 4) = make_float4(y[4], y[5], y[6], y[7]);
-                }
-                named_bar(BAR_IN, NT_IN);
-                if (act) {
-                    float xo[8];
+                    float *Yw = Ys + warp * 256;  // this warp's 16 x 16 Y
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) xo[cc] = 0.f;
-                    const float *Xr = Xm + (16 * I + r) * LST + 16 * I;
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        const float xi = Xr[m];
-                        const float4 ya = *reinterpret_cast<const float4 *>(Ys + bi * 256 + m * 16 + c0);
-                        const float4 yb = *reinterpret_cast<const float4 *>(Ys + bi * 256 + m * 16 + c0 + 4);
-                        xo[0] -= xi * ya.x; xo[1] -= xi * ya.y; xo[2] -= xi * ya.z; xo[3] -= xi * ya.w;
-                        xo[4] -= xi * yb.x; xo[5] -= xi * yb.y; xo[6] -= xi * yb.z; xo[7] -= xi * yb.w;
+                    for (int nt = 0; nt < 2; ++nt) {
+                        *reinterpret_cast<float2 *>(Yw + g * 16 + 8 * nt + 2 * tq) = make_float2(acc[nt][0], acc[nt][1]);
+                        *reinterpret_cast<float2 *>(Yw + (g + 8) * 16 + 8 * nt + 2 * tq) = make_float2(acc[nt][2], acc[nt][3]);
                     }
-                    float *Xo = Xm + (16 * I + r) * LST + 16 * J + c0;
-                    *reinterpret_cast<float4 *>(Xo) = make_float4(xo[0], xo[1], xo[2], xo[3]);
-                    *reinterpret_cast<float4 *>(Xo + 4) = make_float4(xo[4], xo[5], xo[6], xo[7]);
+                    __syncwarp();
+                    // X_IJ = -X_II Y
+                    float xo[2][4];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) xo[nt][e] = 0.f;
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks) {
+                        const float *Xa = Xm + (16 * I + g) * LST + 16 * I + 8 * ks + tq;
+                        const float av[4] = {Xa[0], Xa[8 * LST], Xa[4], Xa[8 * LST + 4]};
+                        uint32_t ah[4], al[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            ah[e] = cvt_tf32(av[e]);
+                            al[e] = cvt_tf32(av[e] - __uint_as_float(ah[e]));
+                        }
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt) {
+                            const float *Yb = Yw + (8 * ks + tq) * 16 + 8 * nt + g;
+                            const float bv[2] = {Yb[0], Yb[4 * 16]};
+                            uint32_t bh[2], bl[2];
+#pragma unroll
+                            for (int e = 0; e < 2; ++e) {
+                                bh[e] = cvt_tf32(bv[e]);
+                                bl[e] = cvt_tf32(bv[e] - __uint_as_float(bh[e]));
+                            }
+                            mma_tf32_16x8x8(xo[nt], al, bh);
+                            mma_tf32_16x8x8(xo[nt], ah, bl);
+                            mma_tf32_16x8x8(xo[nt], ah, bh);
+                        }
+                    }
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        float *Xo = Xm + (16 * I + g) * LST + 16 * J + 8 * nt + 2 * tq;
+                        *reinterpret_cast<float2 *>(Xo) = make_float2(-xo[nt][0], -xo[nt][1]);
+                        *reinterpret_cast<float2 *>(Xo + 8 * LST) = make_float2(-xo[nt][2], -xo[nt][3]);
+                    }
                 }
                 named_bar(BAR_IN, NT_IN);
             }
@@ -600,15 +628,12 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         {
             const int c = ln;
             const uint32_t w64 = (uint32_t)(c >> 6) * 16384u, cb64 = (uint32_t)(c & 63) * 2u;
-            uint32_t u[16], w2[16];
-            tmem_ld16(tb + lq + TM_W + 32 * hf, u);
-            tmem_ld16(tb + lq + TM_W + 32 * hf + 16, w2);
+            uint32_t u[32];
+            tmem_ld32(tb + lq + TM_W + 32 * hf, u);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
+            for (int j = 0; j < 32; ++j)
                 *reinterpret_cast<__half *>(sm + SM_WQ + w64 + sw(32 * hf + j, cb64)) = __float2half_rn(__uint_as_float(u[j]));
-                *reinterpret_cast<__half *>(sm + SM_WQ + w64 + sw(32 * hf + 16 + j, cb64)) = __float2half_rn(__uint_as_float(w2[j]));
-            }
         }
         fence_async_smem();
         tc_fence_before();
@@ -832,9 +857,8 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
                                               ~uintptr_t(1023));
     Ctx cx;
     cx.sm = sm;
-    cx.rq_s = reinterpret_cast<float *>(sm + SM_MISC);
-    cx.rk_s = cx.rq_s + 64;
-    cx.b_s = cx.rk_s + 64;
+    cx.rkq_s = reinterpret_cast<float *>(sm + SM_MISC);
+    cx.b_s = cx.rkq_s + 128;
     cx.gam_s = cx.b_s + 64;     // [2][128]
     cx.osum = cx.gam_s + 256;   // [8][128]
     cx.bars = reinterpret_cast<Bars *>(cx.osum + 1024);
