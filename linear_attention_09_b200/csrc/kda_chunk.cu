@@ -36,6 +36,8 @@
 // read straight from TMEM, and thread v owns value column v.
 #include <cuda.h>
 
+#include <type_traits>
+
 #include "kda.h"
 #include "kda_internal.cuh"
 #include "sm100.cuh"
@@ -102,17 +104,19 @@ __device__ __forceinline__ float2 bf2x2(uint32_t w)
     return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w));
 }
 
+// 2^x and log2(x) on the special-function unit; results below 2^-126 flush to zero
+// (every such factor here scales terms that are negligible at fp32 precision).
 __device__ __forceinline__ float ex2(float x)
 {
     float y;
-    asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 
 __device__ __forceinline__ float lg2(float x)
 {
     float y;
-    asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 
@@ -272,17 +276,14 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             float2 run = make_float2(0.f, 0.f);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                float2 l2 = make_float2(0.f, 0.f);
-                if (t0 + j < L) {
-                    const float2 g2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_G + rb + o16[j]));
-                    const float x0 = g2.x + dtb.x, x1 = g2.y + dtb.y;
-                    const float e0 = lg2(1.f + ex2(-fabsf(x0) * kLog2e));
-                    const float e1 = lg2(1.f + ex2(-fabsf(x1) * kLog2e));
-                    l2.x = fmaxf(lb2, -a2 * fmaxf(x0, 0.f) - aexp * e0);
-                    l2.y = fmaxf(lb2, -a2 * fmaxf(x1, 0.f) - aexp * e1);
-                }
-                run.x += l2.x;
-                run.y += l2.y;
+                // branch-free: tokens past the chunk end read finite tile data and get lam = 0
+                const float2 g2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_G + rb + o16[j]));
+                const float x0 = g2.x + dtb.x, x1 = g2.y + dtb.y;
+                const float e0 = lg2(1.f + ex2(-fabsf(x0) * kLog2e));
+                const float e1 = lg2(1.f + ex2(-fabsf(x1) * kLog2e));
+                const bool valid = t0 + j < L;
+                run.x += valid ? fmaxf(lb2, -a2 * fmaxf(x0, 0.f) - aexp * e0) : 0.f;
+                run.y += valid ? fmaxf(lb2, -a2 * fmaxf(x1, 0.f) - aexp * e1) : 0.f;
                 G[j] = run;
             }
             // octant sums -> chunk prefix sums and the reference values G15, G31, G47, G63
@@ -328,38 +329,42 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
                 wok = wait_or_flag(&bars->wq_free, ppar, 7) && wait_or_flag(&bars->kp_free, ppar, 8);
             ok = named_bar_and(BAR_IN, NT_IN, wok);
             if (!ok) break;
+            // operand rows of this octant; the block (uniform per warp) is a compile-time
+            // branch of the loop body, and tokens past the chunk end have zero norms.
+            auto operand_rows = [&](auto blk0_tag) {
+                constexpr bool kBlk0 = decltype(blk0_tag)::value;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                float2 kk = make_float2(0.f, 0.f), qv = make_float2(0.f, 0.f);
-                if (t0 + j < L) {
+                for (int j = 0; j < 8; ++j) {
                     const float2 rkq = *reinterpret_cast<const float2 *>(cx.rkq_s + 2 * (t0 + j));
-                    kk = mul2(bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_K + rb + o16[j])),
-                              make_float2(rkq.x, rkq.x));
-                    qv = mul2(bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_Q + rb + o16[j])),
-                              make_float2(rkq.y, rkq.y));
+                    const float2 kk = mul2(bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_K + rb + o16[j])),
+                                           make_float2(rkq.x, rkq.x));
+                    const float2 qv = mul2(bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_Q + rb + o16[j])),
+                                           make_float2(rkq.y, rkq.y));
+                    const float d0 = G[j].x - Gr.x, d1 = G[j].y - Gr.y;
+                    const float2 rho = make_float2(ex2(d0), ex2(d1));
+                    const float2 sig = make_float2(ex2(-d0), ex2(-d1));
+                    const float2 kr = mul2(kk, rho), qr = mul2(qv, rho), ks = mul2(kk, sig);
+                    st_u64(sm, SM_APA + o32[j], tf32b(kr.x), tf32b(kr.y));
+                    st_u64(sm, SM_APA + 8192 + o32[j], tf32b(qr.x), tf32b(qr.y));
+                    st_u64(sm, SM_APB + o32[j], tf32b(ks.x), tf32b(ks.y));
+                    const float2 gam = mul2(rho, fa);
+                    float2 kp;
+                    if (kBlk0) {
+                        const float2 s1 = mul2(sig, fb);  // e^{G31 - G_t} <= 1
+                        kp = mul2(s1, fc);
+                        const float2 ko = mul2(kk, mul2(s1, fo));
+                        st_u64(sm, SM_APB + 8192 + o32[j], tf32b(ko.x), tf32b(ko.y));
+                    } else {
+                        kp = mul2(sig, fc);
+                    }
+                    const float2 kg = mul2(kk, gam), qg = mul2(qv, gam), kpp = mul2(kk, kp);
+                    st_u32(sm, SM_KG + rb + o16[j], pack_f16(kg.x, kg.y));
+                    st_u32(sm, SM_WQ + 2 * rb + 8192 + o16[j], pack_f16(qg.x, qg.y));
+                    st_u32(sm, SM_KP + rb + o16[j], pack_f16(kpp.x, kpp.y));
                 }
-                const float d0 = G[j].x - Gr.x, d1 = G[j].y - Gr.y;
-                const float2 rho = make_float2(ex2(d0), ex2(d1));
-                const float2 sig = make_float2(ex2(-d0), ex2(-d1));
-                const float2 kr = mul2(kk, rho), qr = mul2(qv, rho), ks = mul2(kk, sig);
-                st_u64(sm, SM_APA + o32[j], tf32b(kr.x), tf32b(kr.y));
-                st_u64(sm, SM_APA + 8192 + o32[j], tf32b(qr.x), tf32b(qr.y));
-                st_u64(sm, SM_APB + o32[j], tf32b(ks.x), tf32b(ks.y));
-                const float2 gam = mul2(rho, fa);
-                float2 kp;
-                if (blk == 0) {
-                    const float2 s1 = mul2(sig, fb);  // e^{G31 - G_t} <= 1
-                    kp = mul2(s1, fc);
-                    const float2 ko = mul2(kk, mul2(s1, fo));
-                    st_u64(sm, SM_APB + 8192 + o32[j], tf32b(ko.x), tf32b(ko.y));
-                } else {
-                    kp = mul2(sig, fc);
-                }
-                const float2 kg = mul2(kk, gam), qg = mul2(qv, gam), kpp = mul2(kk, kp);
-                st_u32(sm, SM_KG + rb + o16[j], pack_f16(kg.x, kg.y));
-                st_u32(sm, SM_WQ + 2 * rb + 8192 + o16[j], pack_f16(qg.x, qg.y));
-                st_u32(sm, SM_KP + rb + o16[j], pack_f16(kpp.x, kpp.y));
-            }
+            };
+            if (blk == 0) operand_rows(std::true_type{});
+            else operand_rows(std::false_type{});
             fence_async_smem();
             tc_fence_before();
             named_bar(BAR_IN, NT_IN);
@@ -470,11 +475,14 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             for (int d = 1; d < 4; ++d) {
                 if (warp < 4 - d) {
                     const int J = warp, I = J + d;
-                    float acc[2][4];
+                    // separate accumulators per hi/lo term keep the mma chains short
+                    float acc[3][2][4];
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
+                    for (int q3 = 0; q3 < 3; ++q3)
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) acc[q3][nt][e] = 0.f;
                     // Y = sum_K L_IK X_KJ
                     for (int K = J; K < I; ++K) {
 #pragma unroll
@@ -497,25 +505,30 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
                                     bh[e] = cvt_tf32(bv[e]);
                                     bl[e] = cvt_tf32(bv[e] - __uint_as_float(bh[e]));
                                 }
-                                mma_tf32_16x8x8(acc[nt], al, bh);
-                                mma_tf32_16x8x8(acc[nt], ah, bl);
-                                mma_tf32_16x8x8(acc[nt], ah, bh);
+                                mma_tf32_16x8x8(acc[0][nt], al, bh);
+                                mma_tf32_16x8x8(acc[1][nt], ah, bl);
+                                mma_tf32_16x8x8(acc[2][nt], ah, bh);
                             }
                         }
                     }
                     float *Yw = Ys + warp * 256;  // this warp's 16 x 16 Y
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
-                        *reinterpret_cast<float2 *>(Yw + g * 16 + 8 * nt + 2 * tq) = make_float2(acc[nt][0], acc[nt][1]);
-                        *reinterpret_cast<float2 *>(Yw + (g + 8) * 16 + 8 * nt + 2 * tq) = make_float2(acc[nt][2], acc[nt][3]);
+                        float y4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) y4[e] = (acc[0][nt][e] + acc[1][nt][e]) + acc[2][nt][e];
+                        *reinterpret_cast<float2 *>(Yw + g * 16 + 8 * nt + 2 * tq) = make_float2(y4[0], y4[1]);
+                        *reinterpret_cast<float2 *>(Yw + (g + 8) * 16 + 8 * nt + 2 * tq) = make_float2(y4[2], y4[3]);
                     }
                     __syncwarp();
                     // X_IJ = -X_II Y
-                    float xo[2][4];
+                    float xo[3][2][4];
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
+                    for (int q3 = 0; q3 < 3; ++q3)
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) xo[nt][e] = 0.f;
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) xo[q3][nt][e] = 0.f;
 #pragma unroll
                     for (int ks = 0; ks < 2; ++ks) {
                         const float *Xa = Xm + (16 * I + g) * LST + 16 * I + 8 * ks + tq;
@@ -536,16 +549,19 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
                                 bh[e] = cvt_tf32(bv[e]);
                                 bl[e] = cvt_tf32(bv[e] - __uint_as_float(bh[e]));
                             }
-                            mma_tf32_16x8x8(xo[nt], al, bh);
-                            mma_tf32_16x8x8(xo[nt], ah, bl);
-                            mma_tf32_16x8x8(xo[nt], ah, bh);
+                            mma_tf32_16x8x8(xo[0][nt], al, bh);
+                            mma_tf32_16x8x8(xo[1][nt], ah, bl);
+                            mma_tf32_16x8x8(xo[2][nt], ah, bh);
                         }
                     }
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
+                        float x4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) x4[e] = -((xo[0][nt][e] + xo[1][nt][e]) + xo[2][nt][e]);
                         float *Xo = Xm + (16 * I + g) * LST + 16 * J + 8 * nt + 2 * tq;
-                        *reinterpret_cast<float2 *>(Xo) = make_float2(-xo[nt][0], -xo[nt][1]);
-                        *reinterpret_cast<float2 *>(Xo + 8 * LST) = make_float2(-xo[nt][2], -xo[nt][3]);
+                        *reinterpret_cast<float2 *>(Xo) = make_float2(x4[0], x4[1]);
+                        *reinterpret_cast<float2 *>(Xo + 8 * LST) = make_float2(x4[2], x4[3]);
                     }
                 }
                 named_bar(BAR_IN, NT_IN);

@@ -263,17 +263,10 @@ __device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t count, bool 
 namespace kda {
 namespace sm100 {
 
-// Packed fp32 pair multiply (one f32x2 instruction).
-__device__ __forceinline__ float2 mul2(float2 a, float2 b)
-{
-    uint64_t ra, rb, rc;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(ra) : "f"(a.x), "f"(a.y));
-    asm("mov.b64 %0, {%1, %2};" : "=l"(rb) : "f"(b.x), "f"(b.y));
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(rc) : "l"(ra), "l"(rb));
-    float2 r;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(rc));
-    return r;
-}
+// Componentwise product of two fp32 pairs (two scalar multiplies: on sm_100 these
+// issue at full rate, while the packed f32x2 form with its register moves measured
+// slower).
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return make_float2(a.x * b.x, a.y * b.y); }
 
 // fp32 -> tf32 (round to nearest, ties away), as a 32-bit pattern.
 __device__ __forceinline__ uint32_t cvt_tf32(float x)
