@@ -44,6 +44,12 @@ BYTES_PER_TOKEN_HEAD = 4 * 256 + 2 + 256  # q,k,v,g + beta in, out written (bf16
 STATE_BYTES = 128 * 128 * 4  # fp32 final state per (sequence, head)
 FLOPS_PER_TOKEN_HEAD = 140629  # chunked algorithm at C=64, D=128 (triangles halved)
 FALLBACK_HBM_GBS = 6650.0
+KERNEL = "chunk_kernel"  # the one kernel of a kda_fwd call
+KERNEL_SRC = ["linear_attention_09_b200/csrc/kda_chunk.cu", "linear_attention_09_b200/csrc/sm100.cuh"]
+PROFILE = "chunk_kernel_long_B4_T32768_H32.md"  # ncu summary: traffic per launch + source hash
+# arithmetic of the path: bf16 in/out; tf32, fp16 and bf16 tensor-core products with fp32
+# accumulation; fp32 activations, solve and state
+DTYPE = "bf16-io/tf32+fp16+bf16-mma/fp32-acc"
 
 
 def parse():
@@ -160,7 +166,7 @@ class ClockSampler:
 
 def profile_traffic(kernel_source):
     """Per-launch DRAM bytes from the committed ncu summary, if the kernel is unchanged."""
-    path = os.path.join(ROOT, "profiles", "kda_fwd_chunked_long_B4_T32768_H32.md")
+    path = os.path.join(ROOT, "profiles", PROFILE)
     try:
         txt = open(path).read()
     except OSError:
@@ -302,8 +308,7 @@ def main():
     peak, peak_src = peaks()
     bytes_launch = algorithmic_bytes(B, T, H, B)
     achieved = bytes_launch / (ms_local / args.steps / launches_per_step / 1e3) / 1e9
-    kernel_src = ["linear_attention_09_b200/csrc/kda_tokenwise.cu"]
-    traffic, _ = profile_traffic(kernel_src)
+    traffic, _ = profile_traffic(KERNEL_SRC)
 
     # end to end: host (pinned) buffers through kda_fwd_host, copies inside the timed region
     host = {n: inp[n].cpu().pin_memory() for n in ("q", "k", "v", "g", "beta")}
@@ -340,7 +345,7 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
             "config": {"workload": w["name"], "global_batch": B * world, "seq_len": T, "heads": H,
                        "head_dim": 128, "parallelism": f"dp{world}",
                        "l2": "inputs 5.4 GB per step > 126 MB L2 (no flush needed)"},
@@ -348,7 +353,7 @@ def main():
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": peak_src,
                          "alg_bytes_per_launch": bytes_launch,
-                         "kernel": "tokenwise_kernel"},
+                         "kernel": KERNEL},
             "tflops": FLOPS_PER_TOKEN_HEAD * tokens * H * world * args.steps / (ms / 1e3) / 1e12,
             "clocks": clk.summary(),
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,

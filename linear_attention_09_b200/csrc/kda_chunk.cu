@@ -165,7 +165,7 @@ struct TMaps {
 
 struct Ctx {
     uint8_t *sm;
-    float *rkq_s /* [64][2] */, *b_s, *gam_s /* [2][128] */, *osum /* [8][128] */;
+    float *rkq_s /* [64][2] */, *b_s, *gam_s /* [2][128] */, *osum /* [8][128] */, *dtb_s /* [128] */;
     Bars *bars;
     uint32_t tb;  // TMEM base
     int64_t h, H, tok0, len, rstride;
@@ -221,9 +221,12 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         o32[j] = (uint32_t)(cp >> 4) * 16384u + sw((uint32_t)(t0 + j), (uint32_t)(cp & 15) * 8u);
     }
 
-    // beta logits are read one chunk ahead (thread t < 64 holds token t of the next chunk)
-    float beta_raw = 0.f;
-    if (tid < C && tid < cx.len) beta_raw = bf2f(p.beta[(cx.tok0 + tid) * H + h]);
+    // beta logits are read one chunk ahead as raw bf16 bits (thread t < 64 holds token t
+    // of the next chunk); converting them only when the next chunk starts keeps the
+    // global load off the critical path
+    const uint16_t *beta_g = reinterpret_cast<const uint16_t *>(p.beta);
+    uint16_t beta_bits = 0;
+    if (tid < C && tid < cx.len) beta_bits = beta_g[(cx.tok0 + tid) * H + h];
 
     for (int n = 0; n < cx.nchunks && ok; ++n) {
         const int64_t ctok = cx.tok0 + (int64_t)n * C;
@@ -231,9 +234,9 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         const int L = (int)(rem < C ? rem : C);
         const bool has_next = n + 1 < cx.nchunks;
         const uint32_t par = (uint32_t)n & 1u, ppar = (uint32_t)(n - 1) & 1u;
-        const float beta_cur = beta_raw;
+        const float beta_cur = __uint_as_float((uint32_t)beta_bits << 16);
         if (tid < C && has_next && (int64_t)(n + 1) * C + tid < cx.len)
-            beta_raw = bf2f(p.beta[(ctok + C + tid) * H + h]);
+            beta_bits = beta_g[(ctok + C + tid) * H + h];
 
         ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->qkg, par, 6));
         if (!ok) break;
@@ -262,7 +265,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             if (qq == 0)  // (1/|k|, 1/|q|) per token, zero past the chunk end
                 *reinterpret_cast<float2 *>(cx.rkq_s + 2 * t) =
                     (t < L) ? make_float2(rsqrtf(sk + 1e-6f), rsqrtf(sq + 1e-6f)) : make_float2(0.f, 0.f);
-            if (tid < C) cx.b_s[tid] = (tid < L) ? 1.f / (1.f + ex2(-beta_cur * kLog2e)) : 0.f;
+            if (tid < C) cx.b_s[tid] = (tid < L) ? __fdividef(1.f, 1.f + ex2(-beta_cur * kLog2e)) : 0.f;
         }
         named_bar(BAR_IN, NT_IN);
 
@@ -271,7 +274,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         for (int round = 0; round < 2; ++round) {
             const int c0 = 64 * round + 2 * cp;  // first channel of the pair
             const uint32_t rb = (uint32_t)round * 8192u;
-            const float2 dtb = *reinterpret_cast<const float2 *>(p.dt_bias + h * kHead + c0);
+            const float2 dtb = *reinterpret_cast<const float2 *>(cx.dtb_s + c0);
             float2 G[8];  // in-chunk cumulative log2-decay of the pair, tokens t0 .. t0+7
             float2 run = make_float2(0.f, 0.f);
 #pragma unroll
@@ -466,106 +469,98 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             }
         }
         named_bar(BAR_IN, NT_IN);
-        //      Off-diagonal blocks by block diagonals d = I - J: warp (d, J) computes
-        //      Y = sum_{K=J}^{I-1} L_IK X_KJ, then X_IJ = -X_II Y, on the tensor cores
-        //      (m16n8k8 tf32 with the 3-pass hi/lo split: fp32-accurate products).
+        //      Blocks below the diagonal by recursive doubling in fp32, all 256 threads:
+        //        X_(2B+1)(2B) = -X_(2B+1)(2B+1) L_(2B+1)(2B) X_(2B)(2B)   (16 x 16, B = 0, 1)
+        //        X_hl         = -X_hh L_hl X_ll                          (32 x 32 halves)
+        //      where h, l are the token halves 32..63 and 0..31.  Every X_II is lower
+        //      triangular and the blocks above the diagonal are zero, which bounds the
+        //      inner loops below.
         {
-            float *Ys = reinterpret_cast<float *>(sm + SM_Y);
-            const int g = lane >> 2, tq = lane & 3;
-            for (int d = 1; d < 4; ++d) {
-                if (warp < 4 - d) {
-                    const int J = warp, I = J + d;
-                    // separate accumulators per hi/lo term keep the mma chains short
-                    float acc[3][2][4];
+            float *Zs = reinterpret_cast<float *>(sm + SM_Y);  // 2 x [16][16]: L_(2B+1)(2B) X_(2B)(2B)
+            float *Zb = Zs + 512;                              // [32][ZST]:   L_hl X_ll
+            constexpr int ZST = 36;
+            {
+                // thread = (B, row r, columns c, c + 1)
+                const int B = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2, o = 32 * B;
+                const float *Ar = Lm + (o + 16 + r) * LST + o;
+                const float *Bc = Xm + o * LST + o + c;
+                float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int q3 = 0; q3 < 3; ++q3)
+                for (int m = 0; m < 16; m += 4) {
+                    const float4 a = *reinterpret_cast<const float4 *>(Ar + m);
+                    const float2 b0 = *reinterpret_cast<const float2 *>(Bc + (m + 0) * LST);
+                    const float2 b1 = *reinterpret_cast<const float2 *>(Bc + (m + 1) * LST);
+                    const float2 b2 = *reinterpret_cast<const float2 *>(Bc + (m + 2) * LST);
+                    const float2 b3 = *reinterpret_cast<const float2 *>(Bc + (m + 3) * LST);
+                    a0.x += a.x * b0.x; a0.y += a.x * b0.y;
+                    a1.x += a.y * b1.x; a1.y += a.y * b1.y;
+                    a0.x += a.z * b2.x; a0.y += a.z * b2.y;
+                    a1.x += a.w * b3.x; a1.y += a.w * b3.y;
+                }
+                *reinterpret_cast<float2 *>(Zs + B * 256 + r * 16 + c) = make_float2(a0.x + a1.x, a0.y + a1.y);
+                named_bar(BAR_IN, NT_IN);
+                const float *Xr = Xm + (o + 16 + r) * LST + o + 16;
+                const float *Zc = Zs + B * 256 + c;
+                a0 = make_float2(0.f, 0.f);
+                a1 = make_float2(0.f, 0.f);
 #pragma unroll
-                        for (int nt = 0; nt < 2; ++nt)
+                for (int m = 0; m < 16; m += 4) {
+                    const float4 a = *reinterpret_cast<const float4 *>(Xr + m);
+                    const float2 b0 = *reinterpret_cast<const float2 *>(Zc + (m + 0) * 16);
+                    const float2 b1 = *reinterpret_cast<const float2 *>(Zc + (m + 1) * 16);
+                    const float2 b2 = *reinterpret_cast<const float2 *>(Zc + (m + 2) * 16);
+                    const float2 b3 = *reinterpret_cast<const float2 *>(Zc + (m + 3) * 16);
+                    a0.x += a.x * b0.x; a0.y += a.x * b0.y;
+                    a1.x += a.y * b1.x; a1.y += a.y * b1.y;
+                    a0.x += a.z * b2.x; a0.y += a.z * b2.y;
+                    a1.x += a.w * b3.x; a1.y += a.w * b3.y;
+                }
+                *reinterpret_cast<float2 *>(Xm + (o + 16 + r) * LST + o + c) =
+                    make_float2(-(a0.x + a1.x), -(a0.y + a1.y));
+            }
+            named_bar(BAR_IN, NT_IN);
+            {
+                // Zb = L_hl X_ll: thread = (row r = lane, columns 4 warp ..+3); rows m < 4 warp
+                // of X_ll are zero in these columns
+                const int r = lane, c4 = 4 * warp;
+                const float *Ar = Lm + (32 + r) * LST;
+                float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+                for (int m = c4; m < 32; m += 4) {
+                    const float4 a = *reinterpret_cast<const float4 *>(Ar + m);
+                    const float4 b0 = *reinterpret_cast<const float4 *>(Xm + (m + 0) * LST + c4);
+                    const float4 b1 = *reinterpret_cast<const float4 *>(Xm + (m + 1) * LST + c4);
+                    const float4 b2 = *reinterpret_cast<const float4 *>(Xm + (m + 2) * LST + c4);
+                    const float4 b3 = *reinterpret_cast<const float4 *>(Xm + (m + 3) * LST + c4);
+                    a0.x += a.x * b0.x; a0.y += a.x * b0.y; a0.z += a.x * b0.z; a0.w += a.x * b0.w;
+                    a1.x += a.y * b1.x; a1.y += a.y * b1.y; a1.z += a.y * b1.z; a1.w += a.y * b1.w;
+                    a0.x += a.z * b2.x; a0.y += a.z * b2.y; a0.z += a.z * b2.z; a0.w += a.z * b2.w;
+                    a1.x += a.w * b3.x; a1.y += a.w * b3.y; a1.z += a.w * b3.z; a1.w += a.w * b3.w;
+                }
+                *reinterpret_cast<float4 *>(Zb + r * ZST + c4) =
+                    make_float4(a0.x + a1.x, a0.y + a1.y, a0.z + a1.z, a0.w + a1.w);
+            }
+            named_bar(BAR_IN, NT_IN);
+            {
+                // X_hl = -X_hh Zb: thread = (rows 4 warp ..+3 of the half, column c = lane);
+                // X_hh is lower triangular, so row r needs m <= r only
+                const int r4 = 4 * warp, c = lane;
+                float a[4] = {0.f, 0.f, 0.f, 0.f}, b[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int m = 0; m < r4 + 4; m += 4) {
+                    const float z0 = Zb[(m + 0) * ZST + c], z1 = Zb[(m + 1) * ZST + c];
+                    const float z2 = Zb[(m + 2) * ZST + c], z3 = Zb[(m + 3) * ZST + c];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) acc[q3][nt][e] = 0.f;
-                    // Y = sum_K L_IK X_KJ
-                    for (int K = J; K < I; ++K) {
-#pragma unroll
-                        for (int ks = 0; ks < 2; ++ks) {
-                            const float *La = Lm + (16 * I + g) * LST + 16 * K + 8 * ks + tq;
-                            const float av[4] = {La[0], La[8 * LST], La[4], La[8 * LST + 4]};
-                            uint32_t ah[4], al[4];
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                ah[e] = cvt_tf32(av[e]);
-                                al[e] = cvt_tf32(av[e] - __uint_as_float(ah[e]));
-                            }
-#pragma unroll
-                            for (int nt = 0; nt < 2; ++nt) {
-                                const float *Xb = Xm + (16 * K + 8 * ks + tq) * LST + 16 * J + 8 * nt + g;
-                                const float bv[2] = {Xb[0], Xb[4 * LST]};
-                                uint32_t bh[2], bl[2];
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    bh[e] = cvt_tf32(bv[e]);
-                                    bl[e] = cvt_tf32(bv[e] - __uint_as_float(bh[e]));
-                                }
-                                mma_tf32_16x8x8(acc[0][nt], al, bh);
-                                mma_tf32_16x8x8(acc[1][nt], ah, bl);
-                                mma_tf32_16x8x8(acc[2][nt], ah, bh);
-                            }
-                        }
-                    }
-                    float *Yw = Ys + warp * 256;  // this warp's 16 x 16 Y
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        float y4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) y4[e] = (acc[0][nt][e] + acc[1][nt][e]) + acc[2][nt][e];
-                        *reinterpret_cast<float2 *>(Yw + g * 16 + 8 * nt + 2 * tq) = make_float2(y4[0], y4[1]);
-                        *reinterpret_cast<float2 *>(Yw + (g + 8) * 16 + 8 * nt + 2 * tq) = make_float2(y4[2], y4[3]);
-                    }
-                    __syncwarp();
-                    // X_IJ = -X_II Y
-                    float xo[3][2][4];
-#pragma unroll
-                    for (int q3 = 0; q3 < 3; ++q3)
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) xo[q3][nt][e] = 0.f;
-#pragma unroll
-                    for (int ks = 0; ks < 2; ++ks) {
-                        const float *Xa = Xm + (16 * I + g) * LST + 16 * I + 8 * ks + tq;
-                        const float av[4] = {Xa[0], Xa[8 * LST], Xa[4], Xa[8 * LST + 4]};
-                        uint32_t ah[4], al[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            ah[e] = cvt_tf32(av[e]);
-                            al[e] = cvt_tf32(av[e] - __uint_as_float(ah[e]));
-                        }
-#pragma unroll
-                        for (int nt = 0; nt < 2; ++nt) {
-                            const float *Yb = Yw + (8 * ks + tq) * 16 + 8 * nt + g;
-                            const float bv[2] = {Yb[0], Yb[4 * 16]};
-                            uint32_t bh[2], bl[2];
-#pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                bh[e] = cvt_tf32(bv[e]);
-                                bl[e] = cvt_tf32(bv[e] - __uint_as_float(bh[e]));
-                            }
-                            mma_tf32_16x8x8(xo[0][nt], al, bh);
-                            mma_tf32_16x8x8(xo[1][nt], ah, bl);
-                            mma_tf32_16x8x8(xo[2][nt], ah, bh);
-                        }
-                    }
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        float x4[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) x4[e] = -((xo[0][nt][e] + xo[1][nt][e]) + xo[2][nt][e]);
-                        float *Xo = Xm + (16 * I + g) * LST + 16 * J + 8 * nt + 2 * tq;
-                        *reinterpret_cast<float2 *>(Xo) = make_float2(x4[0], x4[1]);
-                        *reinterpret_cast<float2 *>(Xo + 8 * LST) = make_float2(x4[2], x4[3]);
+                    for (int rr = 0; rr < 4; ++rr) {
+                        const float4 x = *reinterpret_cast<const float4 *>(Xm + (32 + r4 + rr) * LST + 32 + m);
+                        a[rr] += x.x * z0;
+                        b[rr] += x.y * z1;
+                        a[rr] += x.z * z2;
+                        b[rr] += x.w * z3;
                     }
                 }
-                named_bar(BAR_IN, NT_IN);
+#pragma unroll
+                for (int rr = 0; rr < 4; ++rr) Xm[(32 + r4 + rr) * LST + c] = -(a[rr] + b[rr]);
             }
+            named_bar(BAR_IN, NT_IN);
         }
         // T = X Diag(b): fp16 copy (for w) and bf16 hi + lo pair (for u = T v).
         // Thread = (row i = tid / 4, 16 columns 16 (tid % 4) ..)
@@ -879,6 +874,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
     cx.osum = cx.gam_s + 256;   // [8][128]
     cx.bars = reinterpret_cast<Bars *>(cx.osum + 1024);
     uint32_t *tbase_s = reinterpret_cast<uint32_t *>(cx.bars + 1);
+    cx.dtb_s = reinterpret_cast<float *>(sm + SM_MISC + 7168);
 
     const int tid = threadIdx.x, warp = tid >> 5;
     cx.H = p.H;
@@ -911,6 +907,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
         tmem_alloc(tbase_s, 512);
         tmem_relinquish();
     }
+    if (tid < kHead && cx.nchunks > 0) cx.dtb_s[tid] = p.dt_bias[cx.h * kHead + tid];
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

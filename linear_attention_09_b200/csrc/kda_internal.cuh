@@ -21,9 +21,8 @@ struct FwdParams {
     int64_t B, T, H, N;      // N = number of sequences
 };
 
-// Kernel launchers; each returns the number of kernels it enqueued (>= 0) or a
-// negative KDA_ERR_* code.
-int launch_tokenwise(const FwdParams &p, cudaStream_t stream);
+// Kernel launcher; returns the number of kernels it enqueued (>= 0) or a negative
+// KDA_ERR_* code.
 int launch_chunked(const FwdParams &p, cudaStream_t stream);
 // Error word the chunked kernel sets when a bounded wait gives up (0 = none).
 int chunked_device_error(bool reset);
