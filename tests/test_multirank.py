@@ -1,0 +1,70 @@
+"""Multi-rank host logic of bench.py on the CPU: world size 2 over gloo.
+
+The data path has no collective (the (sequence, head) units are independent), so the
+multi-rank part is the harness: process-group setup from the torchrun environment,
+the barrier around the timed region, the max-over-ranks time, and the reference arm
+where rank 0 alone runs and prints.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, outdir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      LOCAL_RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import bench
+    import torch.distributed as dist
+    w, r, _ = bench.dist_setup(world)
+    assert (w, r) == (world, rank)
+    bench.barrier(w)
+    t = bench.max_over_ranks(1.5 * (rank + 1), w)  # ranks report 1.5 and 3.0
+    with open(os.path.join(outdir, f"r{rank}.txt"), "w") as f:
+        f.write(repr(t))
+    bench.barrier(w)
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo(tmp_path):
+    ctx = mp.get_context("spawn")
+    port = free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, str(tmp_path))) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    for r in range(2):
+        assert float((tmp_path / f"r{r}.txt").read_text()) == 3.0
+
+
+def test_reference_arm_two_ranks_prints_once():
+    """torchrun with 2 ranks: rank 0 times the oracle and prints one JSON line; rank 1
+    exits 0 without work."""
+    port = free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl",
+           "reference", "--gpus", "2", "--steps", "1", "--warmup", "0", "--seqlen", "256"]
+    res = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
+    assert d["value"] > 0 and d["unit"] == "tokens/s"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
