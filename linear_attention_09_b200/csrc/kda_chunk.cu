@@ -267,7 +267,8 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
                     (t < L) ? make_float2(rsqrtf(sk + 1e-6f), rsqrtf(sq + 1e-6f)) : make_float2(0.f, 0.f);
             if (tid < C) cx.b_s[tid] = (tid < L) ? __fdividef(1.f, 1.f + ex2(-beta_cur * kLog2e)) : 0.f;
         }
-        named_bar(BAR_IN, NT_IN);
+        // (no barrier: the gate loop does not read the norms; the octant-sum barrier
+        //  below publishes both)
 
         // ---- channel pass in two rounds of 64 channels.  Block 0 = tokens 0..31
         //      (reference token 15), block 1 = tokens 32..63 (reference token 47). ----
@@ -325,13 +326,13 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             } else {
                 fc = make_float2(ex2(ref[3].x - ref[2].x), ex2(ref[3].y - ref[2].y));
             }
+            // every thread waits for the buffers it is about to overwrite; a wait that
+            // gives up is combined into the barrier after the operand rows
             bool wok = true;
             if (round == 1)  // A/P operands of round 0 must be consumed first
                 wok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 1);
             else if (n > 0)  // q^ e^G and k' of the previous chunk must be consumed
                 wok = wait_or_flag(&bars->wq_free, ppar, 7) && wait_or_flag(&bars->kp_free, ppar, 8);
-            ok = named_bar_and(BAR_IN, NT_IN, wok);
-            if (!ok) break;
             // operand rows of this octant; the block (uniform per warp) is a compile-time
             // branch of the loop body, and tokens past the chunk end have zero norms.
             auto operand_rows = [&](auto blk0_tag) {
@@ -370,8 +371,9 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             else operand_rows(std::false_type{});
             fence_async_smem();
             tc_fence_before();
-            named_bar(BAR_IN, NT_IN);
+            ok = named_bar_and(BAR_IN, NT_IN, wok);
             tc_fence_after();
+            if (!ok) break;
             // A/P += [k^ rho ; q^ rho] [k^ sig ; k^ e^{G47-G}]^T over this round's 64 channels
             if (tid == 0) {
                 const uint32_t id = idesc(128, 96, kTF32, kTF32, false, false);
@@ -563,28 +565,29 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             named_bar(BAR_IN, NT_IN);
         }
         // T = X Diag(b): fp16 copy (for w) and bf16 hi + lo pair (for u = T v).
-        // Thread = (row i = tid / 4, 16 columns 16 (tid % 4) ..)
+        // Thread = (row i = tid % 64, columns 16 (tid / 64) ..+15): the lanes of a warp
+        // take consecutive rows, so the float4 reads of X (row stride 68 floats) and the
+        // swizzled 16-byte stores are free of bank conflicts.
         {
-            const int i = tid >> 2, jq = (tid & 3) * 16;
+            const int i = tid & 63, jq = (tid >> 6) * 16;
+            const float *Xr = Xm + i * LST + jq;
 #pragma unroll
             for (int j0 = 0; j0 < 16; j0 += 8) {
+                const float4 x0 = *reinterpret_cast<const float4 *>(Xr + j0);
+                const float4 x1 = *reinterpret_cast<const float4 *>(Xr + j0 + 4);
+                const float4 b0 = *reinterpret_cast<const float4 *>(cx.b_s + jq + j0);
+                const float4 b1 = *reinterpret_cast<const float4 *>(cx.b_s + jq + j0 + 4);
+                const float tv[8] = {x0.x * b0.x, x0.y * b0.y, x0.z * b0.z, x0.w * b0.w,
+                                     x1.x * b1.x, x1.y * b1.y, x1.z * b1.z, x1.w * b1.w};
                 uint32_t p16[4], phi[4], plo[4];
 #pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    float tv[2];
-                    __nv_bfloat16 hv[2], lv[2];
-#pragma unroll
-                    for (int q2 = 0; q2 < 2; ++q2) {
-                        const int j = jq + j0 + e + q2;
-                        tv[q2] = Xm[i * LST + j] * cx.b_s[j];
-                        hv[q2] = __float2bfloat16_rn(tv[q2]);
-                        lv[q2] = __float2bfloat16_rn(tv[q2] - __bfloat162float(hv[q2]));
-                    }
-                    p16[e / 2] = pack_f16(tv[0], tv[1]);
-                    __nv_bfloat162 hh2 = __halves2bfloat162(hv[0], hv[1]);
-                    __nv_bfloat162 ll2 = __halves2bfloat162(lv[0], lv[1]);
-                    phi[e / 2] = *reinterpret_cast<uint32_t *>(&hh2);
-                    plo[e / 2] = *reinterpret_cast<uint32_t *>(&ll2);
+                for (int e = 0; e < 4; ++e) {
+                    p16[e] = pack_f16(tv[2 * e], tv[2 * e + 1]);
+                    const __nv_bfloat162 hh = __floats2bfloat162_rn(tv[2 * e], tv[2 * e + 1]);
+                    const float2 hf = __bfloat1622float2(hh);
+                    const __nv_bfloat162 ll = __floats2bfloat162_rn(tv[2 * e] - hf.x, tv[2 * e + 1] - hf.y);
+                    phi[e] = *reinterpret_cast<const uint32_t *>(&hh);
+                    plo[e] = *reinterpret_cast<const uint32_t *>(&ll);
                 }
                 const uint32_t off = sw(i, (jq + j0) * 2);
                 *reinterpret_cast<uint4 *>(sm + SM_T16 + off) = make_uint4(p16[0], p16[1], p16[2], p16[3]);
