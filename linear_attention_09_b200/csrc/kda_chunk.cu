@@ -241,13 +241,14 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->qkg, par, 6));
         if (!ok) break;
 
-        // ---- norms (thread: token tid/4, channels 32 (tid%4) ..+31) and beta ----
+        // ---- norms (thread: token tid/4, 16-byte chunks 2 (tid%4), 2 (tid%4) + 1 of both
+        //      64-channel boxes; each 8-lane phase then reads 8 distinct bank groups) and beta ----
         {
             const int t = tid >> 2, qq = tid & 3;
             float sq = 0.f, sk = 0.f;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
-                const uint32_t off = (uint32_t)(qq >> 1) * 8192u + sw(t, (qq & 1) * 64 + ch * 16);
+                const uint32_t off = (uint32_t)(ch >> 1) * 8192u + sw(t, (2 * qq + (ch & 1)) * 16);
                 const uint4 qr = *reinterpret_cast<const uint4 *>(sm + SM_Q + off);
                 const uint4 kr = *reinterpret_cast<const uint4 *>(sm + SM_K + off);
                 const uint32_t qw[4] = {qr.x, qr.y, qr.z, qr.w}, kw[4] = {kr.x, kr.y, kr.z, kr.w};
@@ -867,8 +868,10 @@ __global__ void __launch_bounds__(NT, 1)
 chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
 {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~uintptr_t(1023));
+    // 1024-byte alignment by pointer arithmetic on the shared array itself, so that the
+    // compiler keeps every access through sm in the shared space (32-bit addresses,
+    // shared loads/stores) instead of falling back to generic ones
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Ctx cx;
     cx.sm = sm;
     cx.rkq_s = reinterpret_cast<float *>(sm + SM_MISC);
