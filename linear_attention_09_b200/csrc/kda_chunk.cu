@@ -53,7 +53,8 @@ using namespace sm100;
 constexpr int C = 64;        // chunk length
 constexpr int NT_IN = 256;   // in-chunk warpgroups: warps 0..7
 constexpr int NT_ST = 128;   // state warpgroup: warps 8..11 (thread v <-> TMEM lane v)
-constexpr int NT = NT_IN + NT_ST;
+constexpr int NT_MMA = 32;   // tensor-core issue warp for the in-chunk products: warp 12
+constexpr int NT = NT_IN + NT_ST + NT_MMA;
 constexpr uint32_t BAR_IN = 1, BAR_ST = 2;  // named barriers of the two roles
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -77,9 +78,9 @@ constexpr uint32_t SM_TLO = SM_APA + 33 * 1024;   // 8 KB bf16 low part of T
 constexpr uint32_t SM_KG = 128 * 1024;      // 16 KB  k^ e^G fp16, MN-major (M = channel, K = token)
 // handed to the state warpgroup:
 constexpr uint32_t SM_WQ = 144 * 1024;      // 32 KB  [w ; q^ e^G] fp16, K-major [128][128]
-constexpr uint32_t SM_KP = 176 * 1024;      // 16 KB  k^ e^{G_last - G} fp16, MN-major (K = token)
+constexpr uint32_t SM_KP0 = 176 * 1024;     // 16 KB  k' = k^ e^{G_last - G} fp16, MN-major (K = token),
+constexpr uint32_t SM_KP1 = 200 * 1024;     // 16 KB    two buffers by chunk parity
 constexpr uint32_t SM_P = 192 * 1024;       // 8 KB   P fp16, K-major [64 i][64 j]
-constexpr uint32_t SM_O = 200 * 1024;       // 16 KB  bf16 output tile [64 t][128 v] (state role)
 constexpr uint32_t SM_MISC = 216 * 1024;    // norms, beta, gamma x2, octant sums, barriers
 constexpr uint32_t SM_BYTES = 224 * 1024;
 constexpr uint32_t SMEM_ALLOC = SM_BYTES + 1024;  // + alignment slack
@@ -155,8 +156,11 @@ struct Bars {
     uint64_t mma_st;   // state role's tensor-core work        (commit)
     uint64_t full;     // chunk operands ready for the state role (1 arrival)
     uint64_t wq_free;  // [w ; q^ e^G] consumed                (commit)
-    uint64_t kp_free;  // k', P consumed                       (commit)
+    uint64_t kp_free[2];  // k' buffer b, gamma slot b and P consumed (commit after the
+                          // state role's second product of a chunk of parity b)
     uint64_t u_free;   // u^T read out of TMEM                 (128 arrivals)
+    uint64_t ops;      // operands of the next in-chunk product written (one arrival per
+                       // in-chunk warp); the issue warp waits on it
 };
 
 struct TMaps {
@@ -222,78 +226,112 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
     }
 
     // beta logits are read one chunk ahead as raw bf16 bits (thread t < 64 holds token t
-    // of the next chunk); converting them only when the next chunk starts keeps the
-    // global load off the critical path
+    // of the chunk after the one being prepared); converting them only when that chunk
+    // starts keeps the global load off the critical path
     const uint16_t *beta_g = reinterpret_cast<const uint16_t *>(p.beta);
     uint16_t beta_bits = 0;
-    if (tid < C && tid < cx.len) beta_bits = beta_g[(cx.tok0 + tid) * H + h];
+    auto chunk_len = [&](int m) {
+        const int64_t rem = cx.len - (int64_t)m * C;
+        return (int)(rem < C ? rem : C);
+    };
+    auto load_beta = [&](int m) {  // raw beta of chunk m (zero past the sequence end)
+        beta_bits = 0;
+        if (tid < C && m < cx.nchunks && (int64_t)m * C + tid < cx.len)
+            beta_bits = beta_g[(cx.tok0 + (int64_t)m * C + tid) * H + h];
+    };
+
+    // ---- norms (thread: token tid/4, 16-byte chunks 2 (tid%4), 2 (tid%4) + 1 of both
+    //      64-channel boxes; each 8-lane phase then reads 8 distinct bank groups) and beta
+    //      of the chunk whose tiles are in shared memory, of length Lc ----
+    auto norms = [&](int Lc) {
+        const float beta_c = __uint_as_float((uint32_t)beta_bits << 16);
+        const int t = tid >> 2, qq = tid & 3;
+        float sq = 0.f, sk = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+            const uint32_t off = (uint32_t)(ch >> 1) * 8192u + sw(t, (2 * qq + (ch & 1)) * 16);
+            const uint4 qr = *reinterpret_cast<const uint4 *>(sm + SM_Q + off);
+            const uint4 kr = *reinterpret_cast<const uint4 *>(sm + SM_K + off);
+            const uint32_t qw[4] = {qr.x, qr.y, qr.z, qr.w}, kw[4] = {kr.x, kr.y, kr.z, kr.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 qf = bf2x2(qw[e]), kf = bf2x2(kw[e]);
+                sq += qf.x * qf.x + qf.y * qf.y;
+                sk += kf.x * kf.x + kf.y * kf.y;
+            }
+        }
+        sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+        sk += __shfl_xor_sync(0xffffffffu, sk, 1);
+        sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+        sk += __shfl_xor_sync(0xffffffffu, sk, 2);
+        if (qq == 0)  // (1/|k|, 1/|q|) per token, zero past the chunk end
+            *reinterpret_cast<float2 *>(cx.rkq_s + 2 * t) =
+                (t < Lc) ? make_float2(rsqrtf(sk + 1e-6f), rsqrtf(sq + 1e-6f)) : make_float2(0.f, 0.f);
+        if (tid < C) cx.b_s[tid] = (tid < Lc) ? __fdividef(1.f, 1.f + ex2(-beta_c * kLog2e)) : 0.f;
+    };
+
+    // ---- gate of one 64-channel round: in-octant cumulative log2-decay of the pair
+    //      (tokens t0 .. t0+7) and the octant sums for the prefix ----
+    auto gate_round = [&](int round, int Lc, float2 (&Gq)[8]) {
+        const int c0 = 64 * round + 2 * cp;
+        const uint32_t rb = (uint32_t)round * 8192u;
+        const float2 dtb = *reinterpret_cast<const float2 *>(cx.dtb_s + c0);
+        float2 run = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            // branch-free: tokens past the chunk end read finite tile data and get lam = 0
+            const float2 g2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_G + rb + o16[j]));
+            const float x0 = g2.x + dtb.x, x1 = g2.y + dtb.y;
+            const float e0 = lg2(1.f + ex2(-fabsf(x0) * kLog2e));
+            const float e1 = lg2(1.f + ex2(-fabsf(x1) * kLog2e));
+            const bool valid = t0 + j < Lc;
+            run.x += valid ? fmaxf(lb2, -a2 * fmaxf(x0, 0.f) - aexp * e0) : 0.f;
+            run.y += valid ? fmaxf(lb2, -a2 * fmaxf(x1, 0.f) - aexp * e1) : 0.f;
+            Gq[j] = run;
+        }
+        *reinterpret_cast<float2 *>(cx.osum + oc * 128 + c0) = run;
+    };
+
+    // Chunk 0's norms and round-0 gate run here; those of chunk n+1 run while the w/u
+    // products of chunk n are on the tensor cores (the octant-sum barrier at the top of
+    // the round publishes them).
+    float2 G0[8];  // round-0 gate of the chunk about to be processed
+    if (cx.nchunks > 0) {
+        load_beta(0);
+        ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->qkg, 0, 6));
+        if (ok) {
+            norms(chunk_len(0));
+            gate_round(0, chunk_len(0), G0);
+            load_beta(1);
+        }
+    }
 
     for (int n = 0; n < cx.nchunks && ok; ++n) {
         const int64_t ctok = cx.tok0 + (int64_t)n * C;
-        const int64_t rem = cx.len - (int64_t)n * C;
-        const int L = (int)(rem < C ? rem : C);
+        const int L = chunk_len(n);
         const bool has_next = n + 1 < cx.nchunks;
         const uint32_t par = (uint32_t)n & 1u, ppar = (uint32_t)(n - 1) & 1u;
-        const float beta_cur = __uint_as_float((uint32_t)beta_bits << 16);
-        if (tid < C && has_next && (int64_t)(n + 1) * C + tid < cx.len)
-            beta_bits = beta_g[(ctok + C + tid) * H + h];
-
-        ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->qkg, par, 6));
-        if (!ok) break;
-
-        // ---- norms (thread: token tid/4, 16-byte chunks 2 (tid%4), 2 (tid%4) + 1 of both
-        //      64-channel boxes; each 8-lane phase then reads 8 distinct bank groups) and beta ----
-        {
-            const int t = tid >> 2, qq = tid & 3;
-            float sq = 0.f, sk = 0.f;
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                const uint32_t off = (uint32_t)(ch >> 1) * 8192u + sw(t, (2 * qq + (ch & 1)) * 16);
-                const uint4 qr = *reinterpret_cast<const uint4 *>(sm + SM_Q + off);
-                const uint4 kr = *reinterpret_cast<const uint4 *>(sm + SM_K + off);
-                const uint32_t qw[4] = {qr.x, qr.y, qr.z, qr.w}, kw[4] = {kr.x, kr.y, kr.z, kr.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 qf = bf2x2(qw[e]), kf = bf2x2(kw[e]);
-                    sq += qf.x * qf.x + qf.y * qf.y;
-                    sk += kf.x * kf.x + kf.y * kf.y;
-                }
-            }
-            sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-            sk += __shfl_xor_sync(0xffffffffu, sk, 1);
-            sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-            sk += __shfl_xor_sync(0xffffffffu, sk, 2);
-            if (qq == 0)  // (1/|k|, 1/|q|) per token, zero past the chunk end
-                *reinterpret_cast<float2 *>(cx.rkq_s + 2 * t) =
-                    (t < L) ? make_float2(rsqrtf(sk + 1e-6f), rsqrtf(sq + 1e-6f)) : make_float2(0.f, 0.f);
-            if (tid < C) cx.b_s[tid] = (tid < L) ? __fdividef(1.f, 1.f + ex2(-beta_cur * kLog2e)) : 0.f;
-        }
-        // (no barrier: the gate loop does not read the norms; the octant-sum barrier
-        //  below publishes both)
+        const uint32_t skp = par ? SM_KP1 : SM_KP0;  // this chunk's k' buffer
 
         // ---- channel pass in two rounds of 64 channels.  Block 0 = tokens 0..31
         //      (reference token 15), block 1 = tokens 32..63 (reference token 47). ----
         for (int round = 0; round < 2; ++round) {
             const int c0 = 64 * round + 2 * cp;  // first channel of the pair
             const uint32_t rb = (uint32_t)round * 8192u;
-            const float2 dtb = *reinterpret_cast<const float2 *>(cx.dtb_s + c0);
             float2 G[8];  // in-chunk cumulative log2-decay of the pair, tokens t0 .. t0+7
-            float2 run = make_float2(0.f, 0.f);
+            if (round == 0) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                // branch-free: tokens past the chunk end read finite tile data and get lam = 0
-                const float2 g2 = bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_G + rb + o16[j]));
-                const float x0 = g2.x + dtb.x, x1 = g2.y + dtb.y;
-                const float e0 = lg2(1.f + ex2(-fabsf(x0) * kLog2e));
-                const float e1 = lg2(1.f + ex2(-fabsf(x1) * kLog2e));
-                const bool valid = t0 + j < L;
-                run.x += valid ? fmaxf(lb2, -a2 * fmaxf(x0, 0.f) - aexp * e0) : 0.f;
-                run.y += valid ? fmaxf(lb2, -a2 * fmaxf(x1, 0.f) - aexp * e1) : 0.f;
-                G[j] = run;
+                for (int j = 0; j < 8; ++j) G[j] = G0[j];
+            } else {
+                gate_round(1, L, G);
             }
+            // Round 0 first waits until chunk n-2, the previous user of this chunk's k'
+            // buffer and gamma slot (both indexed by chunk parity), is fully consumed.
+            bool kok = true;
+            if (round == 0 && n >= 2) kok = wait_or_flag(&bars->kp_free[par], (uint32_t)((n >> 1) - 1) & 1u, 8);
             // octant sums -> chunk prefix sums and the reference values G15, G31, G47, G63
-            *reinterpret_cast<float2 *>(cx.osum + oc * 128 + c0) = run;
-            named_bar(BAR_IN, NT_IN);
+            ok = named_bar_and(BAR_IN, NT_IN, kok);
+            if (!ok) break;
             float2 os[8];
 #pragma unroll
             for (int o = 0; o < 8; ++o) os[o] = *reinterpret_cast<const float2 *>(cx.osum + o * 128 + c0);
@@ -332,8 +370,8 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             bool wok = true;
             if (round == 1)  // A/P operands of round 0 must be consumed first
                 wok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 1);
-            else if (n > 0)  // q^ e^G and k' of the previous chunk must be consumed
-                wok = wait_or_flag(&bars->wq_free, ppar, 7) && wait_or_flag(&bars->kp_free, ppar, 8);
+            else if (n > 0)  // q^ e^G of the previous chunk must be consumed
+                wok = wait_or_flag(&bars->wq_free, ppar, 7);
             // operand rows of this octant; the block (uniform per warp) is a compile-time
             // branch of the loop body, and tokens past the chunk end have zero norms.
             auto operand_rows = [&](auto blk0_tag) {
@@ -365,28 +403,18 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
                     const float2 kg = mul2(kk, gam), qg = mul2(qv, gam), kpp = mul2(kk, kp);
                     st_u32(sm, SM_KG + rb + o16[j], pack_f16(kg.x, kg.y));
                     st_u32(sm, SM_WQ + 2 * rb + 8192 + o16[j], pack_f16(qg.x, qg.y));
-                    st_u32(sm, SM_KP + rb + o16[j], pack_f16(kpp.x, kpp.y));
+                    st_u32(sm, skp + rb + o16[j], pack_f16(kpp.x, kpp.y));
                 }
             };
             if (blk == 0) operand_rows(std::true_type{});
             else operand_rows(std::false_type{});
+            // hand this round's operands to the issue warp (A/P += [k^ rho ; q^ rho]
+            // [k^ sig ; k^ e^{G47-G}]^T over the round's 64 channels)
             fence_async_smem();
-            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->ops);
             ok = named_bar_and(BAR_IN, NT_IN, wok);
-            tc_fence_after();
             if (!ok) break;
-            // A/P += [k^ rho ; q^ rho] [k^ sig ; k^ e^{G47-G}]^T over this round's 64 channels
-            if (tid == 0) {
-                const uint32_t id = idesc(128, 96, kTF32, kTF32, false, false);
-                const uint32_t sa = smem_u32(sm + SM_APA), sb = smem_u32(sm + SM_APB);
-#pragma unroll
-                for (int st = 0; st < 8; ++st) {
-                    const uint64_t da = desc_sw128(sa + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024);
-                    const uint64_t db = desc_sw128(sb + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024);
-                    mma_tf32_ss(tb + TM_AP, da, db, id, (round > 0 || st > 0) ? 1u : 0u);
-                }
-                mma_commit(&bars->mma_in);
-            }
         }
         if (!ok) break;
         // q, k, g tiles are consumed: prefetch the next chunk's
@@ -396,7 +424,13 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             load_tile(sm + SM_K, &tm.k, &bars->qkg, h, ctok + C);
             load_tile(sm + SM_G, &tm.g, &bars->qkg, h, ctok + C);
         }
-        ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 1));
+        {
+            // the A/P product is complete, and chunk n-1's second state product (the last
+            // reader of the single P tile) is done before P is overwritten
+            const bool aok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 1);
+            const bool pok = n < 1 || wait_or_flag(&bars->kp_free[ppar], (uint32_t)((n - 1) >> 1) & 1u, 11);
+            ok = named_bar_and(BAR_IN, NT_IN, aok && pok);
+        }
         tc_fence_after();
         if (!ok) break;
 
@@ -596,41 +630,30 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
                 *reinterpret_cast<uint4 *>(sm + SM_TLO + off) = make_uint4(plo[0], plo[1], plo[2], plo[3]);
             }
         }
+        // hand T to the issue warp (w^T = (k^ e^G)^T T^T, u^T = v^T (T_hi + T_lo)^T); the
+        // barrier keeps b_s of this chunk alive until every warp has written T
         fence_async_smem();
         tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->ops);
         named_bar(BAR_IN, NT_IN);
-        tc_fence_after();
 
-        // ---- w^T = (k^ e^G)^T T^T (fp16), u^T = v^T (T_hi + T_lo)^T (bf16) ----
-        if (tid == 0) {
-            bool w = wait_or_flag(&bars->v, par, 2);
-            if (w && n > 0) w = wait_or_flag(&bars->u_free, ppar, 9);  // u^T of chunk n-1 read
-            if (w) {
-                tc_fence_after();
-                const uint32_t skg = smem_u32(sm + SM_KG), st16 = smem_u32(sm + SM_T16);
-                const uint32_t sv = smem_u32(sm + SM_V), shi = smem_u32(sm + SM_THI),
-                               slo = smem_u32(sm + SM_TLO);
-                const uint32_t idw = idesc(128, 64, kF16, kF16, true, false);
-                const uint32_t idu = idesc(128, 64, kBF16, kBF16, true, false);
-#pragma unroll
-                for (int st = 0; st < 4; ++st)
-                    mma_f16_ss(tb + TM_W, desc_sw128(skg + st * 2048, 8192, 1024),
-                               desc_sw128(st16 + st * 32, 16, 1024), idw, st > 0);
-#pragma unroll
-                for (int st = 0; st < 4; ++st)
-                    mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
-                               desc_sw128(shi + st * 32, 16, 1024), idu, st > 0);
-#pragma unroll
-                for (int st = 0; st < 4; ++st)
-                    mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
-                               desc_sw128(slo + st * 32, 16, 1024), idu, 1);
-                mma_commit(&bars->mma_in);
-            }
-            ok = w;
+        // ---- w^T = (k^ e^G)^T T^T (fp16), u^T = v^T (T_hi + T_lo)^T (bf16) run on the issue warp ----
+        // ---- while the w/u products run: the next chunk's norms and round-0 gate (its
+        //      tiles were requested after this chunk's channel pass; b_s and the norms of
+        //      this chunk are no longer read) ----
+        bool sok = true;
+        if (has_next) {
+            sok = wait_or_flag(&bars->qkg, par ^ 1u, 6);
+            norms(chunk_len(n + 1));
+            gate_round(0, chunk_len(n + 1), G0);
+            load_beta(n + 2);
         }
-        ok = named_bar_and(BAR_IN, NT_IN, ok);
-        if (!ok) break;
-        ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 3));
+        {
+            // (if the issue warp gave up, this bounded wait runs out)
+            const bool mok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 3);
+            ok = named_bar_and(BAR_IN, NT_IN, sok && mok);
+        }
         tc_fence_after();
         if (!ok) break;
         if (tid == 0 && has_next) {  // the v tile is consumed: prefetch the next chunk's
@@ -654,6 +677,58 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         tc_fence_before();
         named_bar(BAR_IN, NT_IN);
         if (tid == 0) mbar_arrive(&bars->full);  // chunk n handed to the state role
+    }
+}
+
+// =====================================================================================
+// Issue role (warp 12, one thread): the in-chunk role's tensor-core products.  For each
+// chunk it waits for the operands of A/P round 0, A/P round 1 and the w/u products
+// (the `ops` barrier, one arrival per in-chunk warp) and commits each group to
+// `mma_in`.  The in-chunk warps never stall on issuing.
+// =====================================================================================
+__device__ void mma_role(const Ctx &cx)
+{
+    if ((threadIdx.x & 31) != 0) return;
+    uint8_t *sm = cx.sm;
+    Bars *bars = cx.bars;
+    const uint32_t tb = cx.tb;
+    const uint32_t sa = smem_u32(sm + SM_APA), sb = smem_u32(sm + SM_APB);
+    const uint32_t skg = smem_u32(sm + SM_KG), st16 = smem_u32(sm + SM_T16);
+    const uint32_t sv = smem_u32(sm + SM_V), shi = smem_u32(sm + SM_THI), slo = smem_u32(sm + SM_TLO);
+    const uint32_t idap = idesc(128, 96, kTF32, kTF32, false, false);
+    const uint32_t idw = idesc(128, 64, kF16, kF16, true, false);
+    const uint32_t idu = idesc(128, 64, kBF16, kBF16, true, false);
+    uint32_t ops_cnt = 0;
+    for (int n = 0; n < cx.nchunks; ++n) {
+        const uint32_t par = (uint32_t)n & 1u, ppar = (uint32_t)(n - 1) & 1u;
+        for (int round = 0; round < 2; ++round) {
+            if (!wait_or_flag(&bars->ops, (ops_cnt++) & 1u, 12)) return;
+            tc_fence_after();
+#pragma unroll
+            for (int st = 0; st < 8; ++st) {
+                const uint64_t da = desc_sw128(sa + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024);
+                const uint64_t db = desc_sw128(sb + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024);
+                mma_tf32_ss(tb + TM_AP, da, db, idap, (round > 0 || st > 0) ? 1u : 0u);
+            }
+            mma_commit(&bars->mma_in);
+        }
+        if (!wait_or_flag(&bars->ops, (ops_cnt++) & 1u, 12)) return;
+        if (!wait_or_flag(&bars->v, par, 2)) return;
+        if (n > 0 && !wait_or_flag(&bars->u_free, ppar, 9)) return;  // u^T of chunk n-1 read
+        tc_fence_after();
+#pragma unroll
+        for (int st = 0; st < 4; ++st)
+            mma_f16_ss(tb + TM_W, desc_sw128(skg + st * 2048, 8192, 1024),
+                       desc_sw128(st16 + st * 32, 16, 1024), idw, st > 0);
+#pragma unroll
+        for (int st = 0; st < 4; ++st)
+            mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
+                       desc_sw128(shi + st * 32, 16, 1024), idu, st > 0);
+#pragma unroll
+        for (int st = 0; st < 4; ++st)
+            mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
+                       desc_sw128(slo + st * 32, 16, 1024), idu, 1);
+        mma_commit(&bars->mma_in);
     }
 }
 
@@ -762,6 +837,7 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
 #pragma unroll
                 for (int j = 0; j < 32; ++j) U[t0 + j] = __uint_as_float(b[j]) - sigma * __uint_as_float(a[j]);
             }
+            tc_fence_before();
             mbar_arrive(&bars->u_free);  // u^T of this chunk is out of TMEM
             float mx = 0.f;
 #pragma unroll
@@ -808,7 +884,7 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
 
         // ---- MMA2: TM_S += U~^T k' (N = 128), D3 = U~^T P^T (N = 64) ----
         if (leader) {
-            const uint32_t skp = smem_u32(sm + SM_KP), sp = smem_u32(sm + SM_P);
+            const uint32_t skp = smem_u32(sm + (par ? SM_KP1 : SM_KP0)), sp = smem_u32(sm + SM_P);
             const uint32_t id2 = idesc(128, 128, kF16, kF16, false, true);
             const uint32_t id3 = idesc(128, 64, kF16, kF16, false, false);
 #pragma unroll
@@ -818,36 +894,29 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
             for (int st = 0; st < 4; ++st)
                 mma_f16_ts(tb + TM_D3, tb + TM_D1 + st * 8, desc_sw128(sp + st * 32, 16, 1024), id3, st > 0);
             mma_commit(&bars->mma_st);
-            mma_commit(&bars->kp_free);
+            mma_commit(&bars->kp_free[par]);
         }
         ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(&bars->mma_st, (mma_cnt++) & 1u, 5));
         tc_fence_after();
         if (!ok) break;
 
-        // ---- out = scale (sigma D1[:, 64:128] + tau D3) -> bf16 tile -> 16-byte row stores ----
+        // ---- out = scale (sigma D1[:, 64:128] + tau D3): thread v stores column v of each
+        //      token; a warp's 32 columns are 64 contiguous bytes of the token's row ----
         {
-#pragma unroll
-            for (int t0 = 0; t0 < C; t0 += 32) {
-                uint32_t a[32], b[32];
-                tmem_ld32(tb + lq + TM_D1 + 64 + t0, a);
-                tmem_ld32(tb + lq + TM_D3 + t0, b);
+            __nv_bfloat16 *op = p.out + (ctok * H + h) * kHead + v;
+            const float fs = p.scale * sigma, ft = p.scale * tau;
+#pragma unroll 1
+            for (int t0 = 0; t0 < C; t0 += 16) {
+                uint32_t a[16], b[16];
+                tmem_ld16(tb + lq + TM_D1 + 64 + t0, a);
+                tmem_ld16(tb + lq + TM_D3 + t0, b);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const float o = p.scale * (sigma * __uint_as_float(a[j]) + tau * __uint_as_float(b[j]));
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + SM_O + (t0 + j) * 256 + v * 2) = __float2bfloat16_rn(o);
+                for (int j = 0; j < 16; ++j) {
+                    if (t0 + j < L) *op = __float2bfloat16_rn(fs * __uint_as_float(a[j]) + ft * __uint_as_float(b[j]));
+                    op += rstride;
                 }
             }
-            named_bar(BAR_ST, NT_ST);
-            __nv_bfloat16 *ob = p.out + (ctok * H + h) * kHead;
-#pragma unroll 4
-            for (int e = v; e < C * 16; e += NT_ST) {
-                const int t = e >> 4, ch = e & 15;
-                if (t < L)
-                    *reinterpret_cast<uint4 *>(ob + (int64_t)t * rstride + ch * 8) =
-                        *reinterpret_cast<const uint4 *>(sm + SM_O + t * 256 + ch * 16);
-            }
-            named_bar(BAR_ST, NT_ST);  // the tile is free for the next chunk
         }
     }
 
@@ -905,8 +974,10 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
         mbar_init(&b->mma_st, 1);
         mbar_init(&b->full, 1);
         mbar_init(&b->wq_free, 1);
-        mbar_init(&b->kp_free, 1);
+        mbar_init(&b->kp_free[0], 1);
+        mbar_init(&b->kp_free[1], 1);
         mbar_init(&b->u_free, NT_ST);
+        mbar_init(&b->ops, NT_IN / 32);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -928,7 +999,8 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
     }
 
     if (warp < NT_IN / 32) in_chunk_role(p, tm, cx);
-    else state_role(p, cx);
+    else if (warp < (NT_IN + NT_ST) / 32) state_role(p, cx);
+    else mma_role(cx);
 
     tc_fence_before();
     __syncthreads();
