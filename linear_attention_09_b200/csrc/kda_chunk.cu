@@ -150,7 +150,7 @@ __device__ __forceinline__ float pow2_ceil(float m)
 }
 
 struct Bars {
-    uint64_t qkg;      // TMA q, k, g tiles                    (tx bytes)
+    uint64_t qkg[2];   // TMA q, k, g 64-channel box b         (tx bytes)
     uint64_t v;        // TMA v tile                           (tx bytes)
     uint64_t mma_in;   // in-chunk role's tensor-core work     (commit)
     uint64_t mma_st;   // state role's tensor-core work        (commit)
@@ -181,6 +181,17 @@ __device__ __forceinline__ bool wait_or_flag(uint64_t *bar, uint32_t parity, int
     if (mbar_wait(bar, parity)) return true;
     atomicExch(&g_chunk_error, code);
     return false;
+}
+
+// q, k and g box b (channels 64b..64b+63) of the chunk starting at token tok
+__device__ __forceinline__ void load_qkg_box(uint8_t *sm, const TMaps &tm, uint64_t *bar, int64_t h,
+                                             int64_t tok, int b)
+{
+    mbar_arrive_expect_tx(bar, 3 * 8192);
+    const int32_t x = (int32_t)(h * kHead + 64 * b), y = (int32_t)tok;
+    tma_load_2d(sm + SM_Q + 8192 * b, &tm.q, bar, x, y);
+    tma_load_2d(sm + SM_K + 8192 * b, &tm.k, bar, x, y);
+    tma_load_2d(sm + SM_G + 8192 * b, &tm.g, bar, x, y);
 }
 
 __device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *tm, uint64_t *bar,
@@ -292,13 +303,13 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         *reinterpret_cast<float2 *>(cx.osum + oc * 128 + c0) = run;
     };
 
-    // Chunk 0's norms and round-0 gate run here; those of chunk n+1 run while the w/u
-    // products of chunk n are on the tensor cores (the octant-sum barrier at the top of
-    // the round publishes them).
+    // Chunk 0's norms and round-0 gate run here.  For chunk n+1, the round-0 gate runs
+    // while chunk n's second A/P product is on the tensor cores and the norms while its
+    // w/u products are (the octant-sum barrier at the top of the round publishes them).
     float2 G0[8];  // round-0 gate of the chunk about to be processed
     if (cx.nchunks > 0) {
         load_beta(0);
-        ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->qkg, 0, 6));
+        ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->qkg[0], 0, 6) && wait_or_flag(&bars->qkg[1], 0, 13));
         if (ok) {
             norms(chunk_len(0));
             gate_round(0, chunk_len(0), G0);
@@ -415,21 +426,23 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             if (lane == 0) mbar_arrive(&bars->ops);
             ok = named_bar_and(BAR_IN, NT_IN, wok);
             if (!ok) break;
+            // this round's box of q, k, g is consumed: prefetch the next chunk's
+            if (tid == 0 && has_next) load_qkg_box(sm, tm, &bars->qkg[round], h, ctok + C, round);
         }
         if (!ok) break;
-        // q, k, g tiles are consumed: prefetch the next chunk's
-        if (tid == 0 && has_next) {
-            mbar_arrive_expect_tx(&bars->qkg, 3 * 16384);
-            load_tile(sm + SM_Q, &tm.q, &bars->qkg, h, ctok + C);
-            load_tile(sm + SM_K, &tm.k, &bars->qkg, h, ctok + C);
-            load_tile(sm + SM_G, &tm.g, &bars->qkg, h, ctok + C);
+        // ---- while the round-1 A/P product runs: the next chunk's round-0 gate (its
+        //      first box was requested after this chunk's round 0) ----
+        bool gok = true;
+        if (has_next) {
+            gok = wait_or_flag(&bars->qkg[0], par ^ 1u, 6);
+            gate_round(0, chunk_len(n + 1), G0);
         }
         {
             // the A/P product is complete, and chunk n-1's second state product (the last
             // reader of the single P tile) is done before P is overwritten
             const bool aok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 1);
             const bool pok = n < 1 || wait_or_flag(&bars->kp_free[ppar], (uint32_t)((n - 1) >> 1) & 1u, 11);
-            ok = named_bar_and(BAR_IN, NT_IN, aok && pok);
+            ok = named_bar_and(BAR_IN, NT_IN, aok && pok && gok);
         }
         tc_fence_after();
         if (!ok) break;
@@ -639,14 +652,13 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         named_bar(BAR_IN, NT_IN);
 
         // ---- w^T = (k^ e^G)^T T^T (fp16), u^T = v^T (T_hi + T_lo)^T (bf16) run on the issue warp ----
-        // ---- while the w/u products run: the next chunk's norms and round-0 gate (its
-        //      tiles were requested after this chunk's channel pass; b_s and the norms of
-        //      this chunk are no longer read) ----
+        // ---- while the w/u products run: the next chunk's norms (its second box was
+        //      requested after this chunk's round 1; b_s and the norms of this chunk are
+        //      no longer read) ----
         bool sok = true;
         if (has_next) {
-            sok = wait_or_flag(&bars->qkg, par ^ 1u, 6);
+            sok = wait_or_flag(&bars->qkg[1], par ^ 1u, 13);
             norms(chunk_len(n + 1));
-            gate_round(0, chunk_len(n + 1), G0);
             load_beta(n + 2);
         }
         {
@@ -968,7 +980,8 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
 
     if (tid == 0) {
         Bars *b = cx.bars;
-        mbar_init(&b->qkg, 1);
+        mbar_init(&b->qkg[0], 1);
+        mbar_init(&b->qkg[1], 1);
         mbar_init(&b->v, 1);
         mbar_init(&b->mma_in, 1);
         mbar_init(&b->mma_st, 1);
@@ -990,10 +1003,8 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
     tc_fence_after();
     cx.tb = *tbase_s;
     if (tid == 0 && cx.nchunks > 0) {  // first chunk's tiles
-        mbar_arrive_expect_tx(&cx.bars->qkg, 3 * 16384);
-        load_tile(sm + SM_Q, &tm.q, &cx.bars->qkg, cx.h, cx.tok0);
-        load_tile(sm + SM_K, &tm.k, &cx.bars->qkg, cx.h, cx.tok0);
-        load_tile(sm + SM_G, &tm.g, &cx.bars->qkg, cx.h, cx.tok0);
+        load_qkg_box(sm, tm, &cx.bars->qkg[0], cx.h, cx.tok0, 0);
+        load_qkg_box(sm, tm, &cx.bars->qkg[1], cx.h, cx.tok0, 1);
         mbar_arrive_expect_tx(&cx.bars->v, 16384);
         load_tile(sm + SM_V, &tm.v, &cx.bars->v, cx.h, cx.tok0);
     }
