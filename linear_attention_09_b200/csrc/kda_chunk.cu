@@ -159,6 +159,7 @@ struct Bars {
     uint64_t kp_free[2];  // k' buffer b, gamma slot b and P consumed (commit after the
                           // state role's second product of a chunk of parity b)
     uint64_t u_free;   // u^T read out of TMEM                 (128 arrivals)
+    uint64_t u_ready;  // u^T of the chunk in TMEM             (commit)
     uint64_t ops;      // operands of the next in-chunk product written (one arrival per
                        // in-chunk warp); the issue warp waits on it
 };
@@ -732,6 +733,7 @@ __device__ void mma_role(const Ctx &cx)
         for (int st = 0; st < 4; ++st)
             mma_f16_ss(tb + TM_W, desc_sw128(skg + st * 2048, 8192, 1024),
                        desc_sw128(st16 + st * 32, 16, 1024), idw, st > 0);
+        mma_commit(&bars->mma_in);  // the in-chunk role needs only w; u goes to the state role
 #pragma unroll
         for (int st = 0; st < 4; ++st)
             mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
@@ -740,7 +742,7 @@ __device__ void mma_role(const Ctx &cx)
         for (int st = 0; st < 4; ++st)
             mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
                        desc_sw128(slo + st * 32, 16, 1024), idu, 1);
-        mma_commit(&bars->mma_in);
+        mma_commit(&bars->u_ready);
     }
 }
 
@@ -817,11 +819,10 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
         }
 
         // ---- wait for the chunk's operands; MMA1: D1 = S~^T [w ; q^ e^G]^T ----
+        tc_fence_before();  // the S~ stores above precede MMA1
         ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(&bars->full, par, 10));
-        if (!ok) break;
-        tc_fence_before();
-        named_bar(BAR_ST, NT_ST);
         tc_fence_after();
+        if (!ok) break;
         if (leader) {
             const uint32_t swq = smem_u32(sm + SM_WQ);
             const uint32_t id = idesc(128, 128, kF16, kF16, false, false);
@@ -832,7 +833,12 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
             mma_commit(&bars->mma_st);
             mma_commit(&bars->wq_free);
         }
-        ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(&bars->mma_st, (mma_cnt++) & 1u, 4));
+        {
+            // MMA1 done, and u^T of this chunk (issued after w by the issue warp) is in TMEM
+            const bool m1 = wait_or_flag(&bars->mma_st, (mma_cnt++) & 1u, 4);
+            const bool uo = wait_or_flag(&bars->u_ready, par, 14);
+            ok = named_bar_and(BAR_ST, NT_ST, m1 && uo);
+        }
         tc_fence_after();
         if (!ok) break;
 
@@ -991,6 +997,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
         mbar_init(&b->kp_free[1], 1);
         mbar_init(&b->u_free, NT_ST);
         mbar_init(&b->ops, NT_IN / 32);
+        mbar_init(&b->u_ready, 1);
         fence_mbar_init();
     }
     if (warp == 0) {
