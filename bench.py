@@ -64,6 +64,9 @@ def parse():
     # profiling aids: a smaller batch / sequence of the same workload (default: the full one)
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--seqlen", type=int, default=None)
+    # the decode step (one token per sequence, state in HBM) instead of the prefill
+    ap.add_argument("--op", default="prefill", choices=["prefill", "decode"])
+    ap.add_argument("--decode-seqs", type=int, default=256)
     a = ap.parse_args()
     if a.batch:
         WORKLOAD["B"] = a.batch
@@ -260,9 +263,75 @@ def run_reference(args, world, rank):
     return 0
 
 
+DECODE_BYTES_PER_TOKEN_HEAD = 2 * 128 * 128 * 4 + 4 * 128 * 2 + 2 + 128 * 2  # state r+w, q k v g, beta, out
+
+
+def run_decode_bench(args, world, rank, local):
+    """Decode step: N sequences x H heads, one token each, fp32 state updated in place."""
+    import linear_attention_09_b200 as kda
+    from linear_attention_09_b200 import build as kbuild
+    kbuild.build()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    N, H = args.decode_seqs, WORKLOAD["H"]
+    gen = torch.Generator(device=device)
+    gen.manual_seed(args.seed + 1000 * rank)
+    rnd = lambda *shape, std=1.0: (torch.randn(*shape, device=device, generator=gen) * std)
+    q, k, v = (rnd(N, H, 128).to(torch.bfloat16) for _ in range(3))
+    g = rnd(N, H, 128, std=WORKLOAD["g_std"]).to(torch.bfloat16)
+    beta = rnd(N, H).to(torch.bfloat16)
+    A_log = torch.empty(H, device=device).uniform_(1.0, 16.0, generator=gen).log_()
+    dt_bias = rnd(H, 128, std=0.1)
+    state = rnd(N, H, 128, 128, std=0.05)
+    out = torch.empty((N, H, 128), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        kda.kda_decode(q, k, v, g, beta, 1.0 / math.sqrt(128), A_log, dt_bias, -5.0, state,
+                       out=out, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_local, world)
+    peak, peak_src = peaks()
+    bytes_launch = N * H * DECODE_BYTES_PER_TOKEN_HEAD
+    achieved = bytes_launch / (ms_local / args.steps / 1e3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": "KDA decode step token-heads/s (H=32, K=V=128, fp32 state in HBM)",
+            "value": N * H * world * args.steps / (ms / 1e3), "unit": "token-heads/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16-io/fp32", "data": "synthetic",
+            "config": {"workload": f"decode_N{N}_H{H}", "sequences": N * world, "heads": H,
+                       "l2": f"state {N * H * 64 // 1024} MB per rank > 126 MB L2"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
+                         "alg_bytes_per_launch": bytes_launch, "kernel": "decode_kernel"},
+            "clocks": clk.summary(), "gpu_launches": args.steps}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args.gpus)
+    if args.op == "decode" and args.impl == "ours":
+        rc = run_decode_bench(args, world, rank, local)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
     if args.impl == "reference":
         rc = run_reference(args, world, rank)
         if world > 1:

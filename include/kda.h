@@ -69,6 +69,12 @@ typedef struct CUstream_st *kda_stream_t;
 #define KDA_ERR_WORKSPACE (-10)   /* workspace missing or too small */
 #define KDA_ERR_DEVICE (-11)      /* no usable sm_100 device for this call */
 #define KDA_ERR_SCALE (-12)       /* scale is not finite */
+#define KDA_ERR_LAYOUT (-13)      /* state_layout is not KV / VK */
+
+/* State layouts (kda_fwd_ex).  The FLA call on the pages passes
+ * transpose_state_layout=True, i.e. per (sequence, head) the state stored value-major. */
+#define KDA_LAYOUT_KV 0 /* S[k][v] at ((n*H + h)*K + k)*V + v   (kda_fwd's layout) */
+#define KDA_LAYOUT_VK 1 /* S[v][k] at ((n*H + h)*V + v)*K + k   (transposed)       */
 
 /*
  * kda_fwd -- the forward/prefill pass on device buffers.
@@ -92,6 +98,27 @@ int kda_fwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_b
             float lower_bound, const void *initial_state, int initial_state_dtype,
             float *final_state, const int64_t *cu_seqlens, int64_t num_seqs, kda_bf16 *out,
             int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, kda_stream_t stream);
+
+/*
+ * kda_fwd_ex -- kda_fwd with the state variants of the operator statement (FlashKDA de
+ * código abierto de Moonshot AI, 7minutos.es, section "Debajo del capó: CUTLASS en
+ * Hopper": optional initial and final states in bf16 or fp32; the transposed layout
+ * is the transpose_state_layout flag of the chunk_kda call on
+ * github.zuobiaodaohang.com, section "作为 FLA 后端的用法").
+ *
+ * final_state: device pointer or NULL; final_state_dtype is KDA_STATE_F32 or
+ *   KDA_STATE_BF16 (bf16 is the fp32 state rounded to nearest even).
+ * state_layout: KDA_LAYOUT_KV or KDA_LAYOUT_VK, for both initial and final state.
+ * Everything else as kda_fwd; kda_fwd(...) == kda_fwd_ex(..., final_state,
+ * KDA_STATE_F32, KDA_LAYOUT_KV, ...).  Extra return code: KDA_ERR_LAYOUT; a
+ * final_state_dtype other than F32/BF16 with a final_state gives KDA_ERR_STATE_DTYPE.
+ */
+int kda_fwd_ex(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
+               const kda_bf16 *beta, float scale, const float *A_log, const float *dt_bias,
+               float lower_bound, const void *initial_state, int initial_state_dtype,
+               void *final_state, int final_state_dtype, int state_layout,
+               const int64_t *cu_seqlens, int64_t num_seqs, kda_bf16 *out, int64_t B, int64_t T,
+               int64_t H, int64_t K, int64_t V, kda_stream_t stream);
 
 /*
  * kda_fwd_host_workspace_size -- bytes of device memory kda_fwd_host needs for a
@@ -119,6 +146,25 @@ int kda_fwd_host(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const 
                  float *final_state, const int64_t *cu_seqlens, int64_t num_seqs,
                  kda_bf16 *out, int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
                  void *workspace, size_t workspace_bytes, kda_stream_t stream);
+
+/*
+ * kda_decode -- one decode step: a single new token for each of N sequences, the
+ * same operator as kda_fwd with T = 1 and the state carried in HBM between calls
+ * (the generation step that follows prefill; FlashKDA pages, 7minutos.es, "¿Qué es
+ * la atención Kimi Delta y por qué es importante?").
+ *
+ *   q, k, g   [N, H, K] bf16     v, out  [N, H, V] bf16     beta  [N, H] bf16
+ *   A_log [H], dt_bias [H, K] fp32; scale and lower_bound as kda_fwd
+ *   state_in  fp32 [N, H, K, V], S[k][v]; state_out fp32 [N, H, K, V], may be the
+ *             same buffer as state_in (update in place)
+ * Device pointers; asynchronous on stream.  N == 0 is a no-op.  Returns KDA_OK or a
+ * negative code (head size, NULL pointers, alignment: 16 bytes for the states, 2 for
+ * the bf16 vectors, 4 for A_log / dt_bias; lower_bound; scale; shape; device).
+ */
+int kda_decode(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
+               const kda_bf16 *beta, float scale, const float *A_log, const float *dt_bias,
+               float lower_bound, const float *state_in, float *state_out, kda_bf16 *out,
+               int64_t N, int64_t H, int64_t K, int64_t V, kda_stream_t stream);
 
 /* Human-readable text of a return code (static storage; never NULL). */
 const char *kda_strerror(int code);

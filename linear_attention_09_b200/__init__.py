@@ -5,7 +5,7 @@ Argument marshalling only: every step of the pass runs in the CUDA kernels of
 PyTorch fallback: if the library cannot be loaded, the calls raise.
 
 The functions mirror the C ABI in ``include/kda.h``:
-  kda_fwd, kda_fwd_host, kda_fwd_host_workspace_size, kda_strerror,
+  kda_fwd, kda_fwd_ex, kda_decode, kda_fwd_host, kda_fwd_host_workspace_size, kda_strerror,
   kda_last_launch_count, kda_device_status.
 """
 from __future__ import annotations
@@ -21,6 +21,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libkda.so")
 
 KDA_STATE_NONE, KDA_STATE_F32, KDA_STATE_BF16 = 0, 1, 2
+KDA_LAYOUT_KV, KDA_LAYOUT_VK = 0, 1
+_LAYOUTS = {"kv": KDA_LAYOUT_KV, "vk": KDA_LAYOUT_VK}
 HEAD = 128
 
 _lib = None
@@ -48,6 +50,11 @@ def lib() -> ctypes.CDLL:
             L.kda_fwd.argtypes = [P, P, P, P, P, F, P, P, F, P, I, P, P, I64, P, I64, I64, I64,
                                   I64, I64, P]
             L.kda_fwd.restype = I
+            L.kda_fwd_ex.argtypes = [P, P, P, P, P, F, P, P, F, P, I, P, I, I, P, I64, P, I64,
+                                     I64, I64, I64, I64, P]
+            L.kda_fwd_ex.restype = I
+            L.kda_decode.argtypes = [P, P, P, P, P, F, P, P, F, P, P, P, I64, I64, I64, I64, P]
+            L.kda_decode.restype = I
             L.kda_fwd_host.argtypes = [P, P, P, P, P, F, P, P, F, P, I, P, P, I64, P, I64, I64,
                                        I64, I64, I64, P, SZ, P]
             L.kda_fwd_host.restype = I
@@ -127,6 +134,52 @@ def kda_fwd(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, initial_state=
     if rc != 0:
         raise KDAError(rc, "kda_fwd")
     return out, final_state
+
+
+def kda_fwd_ex(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, initial_state=None,
+               final_state=None, cu_seqlens=None, out=None, output_final_state=True,
+               state_layout="kv", final_state_dtype=torch.float32, stream=None):
+    """``kda_fwd`` with the state variants: ``state_layout`` "kv" (S[k][v]) or "vk"
+    (S[v][k], the transposed layout) for both states, and a bf16 or fp32 final state
+    (``final_state_dtype``, or the dtype of a given ``final_state``)."""
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = B if cu_seqlens is None else num_seqs
+    layout = _LAYOUTS.get(state_layout, -1) if isinstance(state_layout, str) else int(state_layout)
+    if out is None:
+        out = torch.empty((B, T, H, V), dtype=torch.bfloat16, device=q.device)
+    if final_state is None and output_final_state:
+        shape = (N, H, K, V) if layout != KDA_LAYOUT_VK else (N, H, V, K)
+        final_state = torch.empty(shape, dtype=final_state_dtype, device=q.device)
+    rc = lib().kda_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                          _ptr(A_log), _ptr(dt_bias), float(lower_bound), _ptr(initial_state),
+                          _state_dtype(initial_state), _ptr(final_state),
+                          _state_dtype(final_state) if final_state is not None else KDA_STATE_F32,
+                          layout, _ptr(cu_seqlens), num_seqs, _ptr(out), B, T, H, K, V,
+                          _stream_handle(stream, q.device))
+    if rc != 0:
+        raise KDAError(rc, "kda_fwd_ex")
+    return out, final_state
+
+
+def kda_decode(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, state, state_out=None,
+               out=None, stream=None):
+    """One decode step on CUDA tensors: q, k, g bf16 [N,H,128], v bf16 [N,H,128], beta
+    bf16 [N,H]; ``state`` fp32 [N,H,128,128] (S[k][v]) is updated in place unless
+    ``state_out`` is given.  Returns (out [N,H,128] bf16, new state)."""
+    N, H, K = q.shape
+    V = v.shape[2]
+    if state_out is None:
+        state_out = state
+    if out is None:
+        out = torch.empty((N, H, V), dtype=torch.bfloat16, device=q.device)
+    rc = lib().kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                          _ptr(A_log), _ptr(dt_bias), float(lower_bound), _ptr(state),
+                          _ptr(state_out), _ptr(out), N, H, K, V, _stream_handle(stream, q.device))
+    if rc != 0:
+        raise KDAError(rc, "kda_decode")
+    return out, state_out
 
 
 def kda_fwd_raw(*args) -> int:

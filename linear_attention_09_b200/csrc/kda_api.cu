@@ -35,7 +35,7 @@ int check_device()
 // Validation shared by kda_fwd and kda_fwd_host (pointer kinds aside).
 int validate(const void *q, const void *k, const void *v, const void *g, const void *beta,
              float scale, const float *A_log, const float *dt_bias, float lower_bound,
-             const void *init, int init_dtype, const float *final_state, const int64_t *cu,
+             const void *init, int init_dtype, const void *final_state, const int64_t *cu,
              int64_t num_seqs, const void *out, int64_t B, int64_t T, int64_t H, int64_t K,
              int64_t V, int64_t *N_out)
 {
@@ -114,6 +114,7 @@ extern "C" const char *kda_strerror(int code)
     case KDA_ERR_WORKSPACE: return "workspace missing or too small";
     case KDA_ERR_DEVICE: return "no usable sm_100 (B200) device";
     case KDA_ERR_SCALE: return "scale must be finite";
+    case KDA_ERR_LAYOUT: return "state_layout must be KDA_LAYOUT_KV or KDA_LAYOUT_VK";
     default: return "unknown kda error code";
     }
 }
@@ -122,18 +123,22 @@ extern "C" int kda_last_launch_count(void) { return g_last_launches; }
 
 extern "C" int kda_device_status(int reset) { return kda::chunked_device_error(reset != 0); }
 
-extern "C" int kda_fwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
-                       const kda_bf16 *beta, float scale, const float *A_log,
-                       const float *dt_bias, float lower_bound, const void *initial_state,
-                       int initial_state_dtype, float *final_state, const int64_t *cu_seqlens,
-                       int64_t num_seqs, kda_bf16 *out, int64_t B, int64_t T, int64_t H,
-                       int64_t K, int64_t V, kda_stream_t stream)
+extern "C" int kda_fwd_ex(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v,
+                          const kda_bf16 *g, const kda_bf16 *beta, float scale,
+                          const float *A_log, const float *dt_bias, float lower_bound,
+                          const void *initial_state, int initial_state_dtype, void *final_state,
+                          int final_state_dtype, int state_layout, const int64_t *cu_seqlens,
+                          int64_t num_seqs, kda_bf16 *out, int64_t B, int64_t T, int64_t H,
+                          int64_t K, int64_t V, kda_stream_t stream)
 {
     int64_t N = 0;
     int rc = validate(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, initial_state,
                       initial_state_dtype, final_state, cu_seqlens, num_seqs, out, B, T, H, K, V,
                       &N);
     if (rc != KDA_OK) return rc;
+    if (state_layout != KDA_LAYOUT_KV && state_layout != KDA_LAYOUT_VK) return KDA_ERR_LAYOUT;
+    if (final_state && final_state_dtype != KDA_STATE_F32 && final_state_dtype != KDA_STATE_BF16)
+        return KDA_ERR_STATE_DTYPE;
     if ((rc = check_device()) != KDA_OK) return rc;
     kda::FwdParams p{};
     p.q = reinterpret_cast<const __nv_bfloat16 *>(q);
@@ -146,6 +151,8 @@ extern "C" int kda_fwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, 
     p.init = initial_state;
     p.init_dtype = initial_state_dtype;
     p.final_state = final_state;
+    p.final_dtype = final_state_dtype;
+    p.state_layout = state_layout;
     p.cu = cu_seqlens;
     p.out = reinterpret_cast<__nv_bfloat16 *>(out);
     p.scale = scale;
@@ -161,6 +168,62 @@ extern "C" int kda_fwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, 
         return KDA_OK;
     }
     const int n = kda::launch_chunked(p, st);
+    if (n < 0) return n;
+    g_last_launches = n;
+    return KDA_OK;
+}
+
+extern "C" int kda_fwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
+                       const kda_bf16 *beta, float scale, const float *A_log,
+                       const float *dt_bias, float lower_bound, const void *initial_state,
+                       int initial_state_dtype, float *final_state, const int64_t *cu_seqlens,
+                       int64_t num_seqs, kda_bf16 *out, int64_t B, int64_t T, int64_t H,
+                       int64_t K, int64_t V, kda_stream_t stream)
+{
+    return kda_fwd_ex(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, initial_state,
+                      initial_state_dtype, final_state, KDA_STATE_F32, KDA_LAYOUT_KV, cu_seqlens,
+                      num_seqs, out, B, T, H, K, V, stream);
+}
+
+extern "C" int kda_decode(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v,
+                          const kda_bf16 *g, const kda_bf16 *beta, float scale,
+                          const float *A_log, const float *dt_bias, float lower_bound,
+                          const float *state_in, float *state_out, kda_bf16 *out, int64_t N,
+                          int64_t H, int64_t K, int64_t V, kda_stream_t stream)
+{
+    if (K != kda::kHead || V != kda::kHead) return KDA_ERR_HEAD_DIM;
+    if (N < 0 || H < 1 || N > (int64_t(1) << 40) / H || N * H > (int64_t(1) << 31) - 1)
+        return KDA_ERR_SHAPE;
+    if (!(lower_bound >= -5.0f && lower_bound <= 0.0f)) return KDA_ERR_LOWER_BOUND;
+    if (!std::isfinite(scale)) return KDA_ERR_SCALE;
+    if (N == 0) {
+        g_last_launches = 0;
+        return KDA_OK;
+    }
+    if (!q || !k || !v || !g || !beta || !A_log || !dt_bias || !state_in || !state_out || !out)
+        return KDA_ERR_NULL;
+    if (!aligned(q, 2) || !aligned(k, 2) || !aligned(v, 2) || !aligned(g, 2) || !aligned(beta, 2) ||
+        !aligned(out, 2) || !aligned(A_log, 4) || !aligned(dt_bias, 4) || !aligned(state_in, 16) ||
+        !aligned(state_out, 16))
+        return KDA_ERR_ALIGN;
+    int rc = check_device();
+    if (rc != KDA_OK) return rc;
+    kda::DecodeParams p{};
+    p.q = reinterpret_cast<const __nv_bfloat16 *>(q);
+    p.k = reinterpret_cast<const __nv_bfloat16 *>(k);
+    p.v = reinterpret_cast<const __nv_bfloat16 *>(v);
+    p.g = reinterpret_cast<const __nv_bfloat16 *>(g);
+    p.beta = reinterpret_cast<const __nv_bfloat16 *>(beta);
+    p.A_log = A_log;
+    p.dt_bias = dt_bias;
+    p.state_in = state_in;
+    p.state_out = state_out;
+    p.out = reinterpret_cast<__nv_bfloat16 *>(out);
+    p.scale = scale;
+    p.lower_bound = lower_bound;
+    p.N = N;
+    p.H = H;
+    const int n = kda::launch_decode(p, reinterpret_cast<cudaStream_t>(stream));
     if (n < 0) return n;
     g_last_launches = n;
     return KDA_OK;

@@ -768,6 +768,13 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
     uint32_t mma_cnt = 0;
     bool ok = true;
 
+    // element (k, v) of a state in either layout: S[k][v] (rows of the KV layout are
+    // read and written coalesced across threads v) or S[v][k] (thread v owns a row)
+    const bool vk = p.state_layout == KDA_LAYOUT_VK;
+    auto st_idx = [&](int kk) -> size_t {
+        return state_off + (vk ? (size_t)v * kHead + kk : (size_t)kk * kHead + v);
+    };
+
     // initial state (column v) -> TM_S with tau = 1
     float tau = 1.f;
     for (int k0 = 0; k0 < kHead; k0 += 16) {
@@ -776,9 +783,9 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
         for (int j = 0; j < 16; ++j) {
             float x = 0.f;
             if (p.init && p.init_dtype == KDA_STATE_F32)
-                x = reinterpret_cast<const float *>(p.init)[state_off + (size_t)(k0 + j) * kHead + v];
+                x = reinterpret_cast<const float *>(p.init)[st_idx(k0 + j)];
             else if (p.init)
-                x = bf2f(reinterpret_cast<const __nv_bfloat16 *>(p.init)[state_off + (size_t)(k0 + j) * kHead + v]);
+                x = bf2f(reinterpret_cast<const __nv_bfloat16 *>(p.init)[st_idx(k0 + j)]);
             r[j] = __float_as_uint(x);
         }
         tmem_st16(tb + lq + TM_S + k0, r);
@@ -938,15 +945,19 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
         }
     }
 
-    // ---- final state = tau TM_S (column v) ----
+    // ---- final state = tau TM_S (column v), fp32 or bf16 (round to nearest even) ----
     if (ok && p.final_state) {
-        float *dst = p.final_state + state_off + v;
+        const bool bf = p.final_dtype == KDA_STATE_BF16;
         for (int k0 = 0; k0 < kHead; k0 += 32) {
             uint32_t a[32];
             tmem_ld32(tb + lq + TM_S + k0, a);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) dst[(size_t)(k0 + j) * kHead] = tau * __uint_as_float(a[j]);
+            for (int j = 0; j < 32; ++j) {
+                const float x = tau * __uint_as_float(a[j]);
+                if (bf) reinterpret_cast<__nv_bfloat16 *>(p.final_state)[st_idx(k0 + j)] = __float2bfloat16_rn(x);
+                else reinterpret_cast<float *>(p.final_state)[st_idx(k0 + j)] = x;
+            }
         }
     }
 }

@@ -12,14 +12,29 @@ constexpr int kHead = 128;  // K = V = 128 (the pages' only supported head size)
 struct FwdParams {
     const __nv_bfloat16 *q, *k, *v, *g, *beta;
     const float *A_log, *dt_bias;
-    const void *init;        // fp32 or bf16 [N,H,K,V] or nullptr
+    const void *init;        // fp32 or bf16 state per (sequence, head) or nullptr
     int init_dtype;          // KDA_STATE_*
-    float *final_state;      // fp32 [N,H,K,V] or nullptr
+    void *final_state;       // fp32 or bf16 state per (sequence, head) or nullptr
+    int final_dtype;         // KDA_STATE_F32 / KDA_STATE_BF16
+    int state_layout;        // KDA_LAYOUT_KV / KDA_LAYOUT_VK (both states)
     const int64_t *cu;       // [N+1] or nullptr
     __nv_bfloat16 *out;
     float scale, lower_bound;
     int64_t B, T, H, N;      // N = number of sequences
 };
+
+// One decode step: one token per (sequence, head), state updated in HBM.
+struct DecodeParams {
+    const __nv_bfloat16 *q, *k, *v, *g, *beta;  // [N,H,K], [N,H,K], [N,H,V], [N,H,K], [N,H]
+    const float *A_log, *dt_bias;
+    const float *state_in;   // fp32 [N,H,K,V] (S[k][v])
+    float *state_out;        // fp32 [N,H,K,V]; may equal state_in
+    __nv_bfloat16 *out;      // [N,H,V]
+    float scale, lower_bound;
+    int64_t N, H;
+};
+
+int launch_decode(const DecodeParams &p, cudaStream_t stream);
 
 // Kernel launcher; returns the number of kernels it enqueued (>= 0) or a negative
 // KDA_ERR_* code.

@@ -68,7 +68,7 @@ def test_invalid_arguments_rejected_on_host(L, over, code):
 
 
 def test_error_strings(L):
-    for c in range(-12, 1):
+    for c in range(-13, 1):
         s = kda.kda_strerror(c)
         assert isinstance(s, str) and s
     assert kda.kda_strerror(0) == "ok"
@@ -92,3 +92,65 @@ def test_host_workspace_size(L):
 def test_binding_has_no_fallback():
     src = open(os.path.join(ROOT, "linear_attention_09_b200", "__init__.py")).read()
     assert "oracle" not in src and "import numpy" not in src
+
+
+def call_ex(final_dtype=1, layout=0, **over):
+    args = dict(q=A16, k=A16 + 0x100, v=A16 + 0x200, g=A16 + 0x300, beta=A16 + 0x400, scale=0.1,
+                A_log=A16 + 0x500, dt_bias=A16 + 0x600, lb=-5.0, init=None, init_dtype=0,
+                final=A16 + 0xA00, cu=None, num_seqs=0, out=A16 + 0x700, B=1, T=64, H=2, K=128,
+                V=128, stream=None)
+    args.update(over)
+    a = args
+    return int(kda.lib().kda_fwd_ex(a["q"], a["k"], a["v"], a["g"], a["beta"],
+                                    ctypes.c_float(a["scale"]), a["A_log"], a["dt_bias"],
+                                    ctypes.c_float(a["lb"]), a["init"], a["init_dtype"], a["final"],
+                                    final_dtype, layout, a["cu"], a["num_seqs"], a["out"], a["B"],
+                                    a["T"], a["H"], a["K"], a["V"], a["stream"]))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(layout=2), -13), (dict(layout=-1), -13),
+    (dict(final_dtype=0), -6), (dict(final_dtype=3), -6),
+    (dict(K=64), -1), (dict(lb=1.0), -5), (dict(final=A16 + 4), -7),
+])
+def test_ex_invalid_arguments_rejected_on_host(L, kw, code):
+    assert call_ex(**kw) == code
+
+
+def test_ex_valid_arguments_without_device(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; the GPU tests cover valid calls")
+    for layout in (0, 1):
+        for fd in (1, 2):
+            assert call_ex(final_dtype=fd, layout=layout) == -11
+    # no final state: its dtype is not looked at
+    assert call_ex(final=None, final_dtype=0) == -11
+
+
+def call_decode(**over):
+    a = dict(q=A16, k=A16 + 0x100, v=A16 + 0x200, g=A16 + 0x300, beta=A16 + 0x400, scale=0.1,
+             A_log=A16 + 0x500, dt_bias=A16 + 0x600, lb=-5.0, sin=A16 + 0x800, sout=A16 + 0x800,
+             out=A16 + 0x700, N=4, H=2, K=128, V=128, stream=None)
+    a.update(over)
+    return int(kda.lib().kda_decode(a["q"], a["k"], a["v"], a["g"], a["beta"],
+                                    ctypes.c_float(a["scale"]), a["A_log"], a["dt_bias"],
+                                    ctypes.c_float(a["lb"]), a["sin"], a["sout"], a["out"], a["N"],
+                                    a["H"], a["K"], a["V"], a["stream"]))
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(K=64), -1), (dict(V=64), -1), (dict(q=None), -2), (dict(sin=None), -2),
+    (dict(sout=None), -2), (dict(out=None), -2), (dict(lb=-6.0), -5),
+    (dict(sin=A16 + 0x804), -7), (dict(q=A16 + 1), -7), (dict(A_log=A16 + 2), -7),
+    (dict(N=-1), -8), (dict(H=0), -8), (dict(scale=float("nan")), -12),
+])
+def test_decode_invalid_arguments_rejected_on_host(L, over, code):
+    assert call_decode(**over) == code
+
+
+def test_decode_empty_and_valid_without_device(L):
+    import torch
+    assert call_decode(N=0, q=None) == 0  # nothing to do
+    if not torch.cuda.is_available():
+        assert call_decode() == -11

@@ -186,3 +186,118 @@ def test_workload_parity(cfg):
     out_g, fin_g = run_gpu(inp)
     r = assert_parity(inp, out_g, fin_g, out_r, fin_r, pairs=pairs, what=f"config {cfg}")
     print(f"config {cfg}: {r}")
+
+
+# ---------------------------------------------------------------------------
+# State variants (kda_fwd_ex): transposed layout, bf16 final state.
+# ---------------------------------------------------------------------------
+def bf16_rne(x: np.ndarray) -> np.ndarray:
+    """fp32 values rounded to bf16 (nearest even), returned as float64."""
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16).double().numpy()
+
+
+@pytest.mark.parametrize("init", ["f32", "bf16"])
+def test_transposed_state_layout_is_the_transpose(init):
+    """S[v][k] in and out gives exactly the transposes of the S[k][v] call, and the same out."""
+    w = ki.Workload("vk", B=2, T=200, H=3, init_state=init)
+    inp = ki.make_inputs(w, 21)
+    d = dev(inp)
+    out_kv, fin_kv = kda.kda_fwd(**d)
+    d_vk = dict(d, initial_state=d["initial_state"].transpose(-1, -2).contiguous())
+    out_vk, fin_vk = kda.kda_fwd_ex(**d_vk, state_layout="vk")
+    torch.cuda.synchronize()
+    assert kda.kda_device_status(reset=True) == 0
+    assert torch.equal(out_vk, out_kv)
+    assert torch.equal(fin_vk, fin_kv.transpose(-1, -2))
+    out_r, fin_r = oracle.forward_inputs(inp)
+    assert_parity(inp, out_vk.float().cpu().numpy().astype(np.float64),
+                  fin_vk.transpose(-1, -2).cpu().numpy().astype(np.float64), out_r, fin_r,
+                  what=f"VK layout init={init}")
+
+
+@pytest.mark.parametrize("layout", ["kv", "vk"])
+def test_bf16_final_state(layout):
+    """The bf16 final state is the fp32 one rounded to nearest even (bit for bit), and
+    within the fp32 bar plus one bf16 half-ulp (2^-9 relative) of the oracle."""
+    inp = small(T=333, H=2, init="f32", seed=8)
+    d = dev(inp)
+    if layout == "vk":
+        d["initial_state"] = d["initial_state"].transpose(-1, -2).contiguous()
+    out32, fin32 = kda.kda_fwd_ex(**d, state_layout=layout)
+    out16, fin16 = kda.kda_fwd_ex(**d, state_layout=layout, final_state_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert kda.kda_device_status(reset=True) == 0
+    assert fin16.dtype == torch.bfloat16 and torch.equal(out16, out32)
+    assert torch.equal(fin16, fin32.to(torch.bfloat16))
+    _, fin_r = oracle.forward_inputs(inp)
+    f = fin16.double().cpu().numpy()
+    if layout == "vk":
+        f = np.swapaxes(f, -1, -2)
+    assert rel(f, fin_r) <= FIN_REL + 2.0 ** -9
+
+
+def test_zero_tokens_state_variants():
+    """T = 0: the final state is the initial one, converted (both states in the same
+    layout, so no transpose)."""
+    inp = small(T=0, init="f32")
+    d = dev(inp)
+    _, fin = kda.kda_fwd_ex(**d, state_layout="vk", final_state_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert torch.equal(fin.cpu(), inp.initial_state.to(torch.bfloat16))
+
+
+# ---------------------------------------------------------------------------
+# Decode step (kda_decode): one token per sequence, state in HBM.
+# ---------------------------------------------------------------------------
+def decode_inputs(N, H, seed, g_std=1.0):
+    w = ki.Workload("decode", B=N, T=1, H=H, init_state="f32", g_std=g_std)
+    return ki.make_inputs(w, seed)
+
+
+def run_decode(inp, in_place=True):
+    d = dev(inp)
+    sq = lambda t: t[:, 0].contiguous()  # [N,1,H,D] -> [N,H,D]
+    state = d["initial_state"].clone()
+    out, st = kda.kda_decode(sq(d["q"]), sq(d["k"]), sq(d["v"]), sq(d["g"]), d["beta"][:, 0].contiguous(),
+                             d["scale"], d["A_log"], d["dt_bias"], d["lower_bound"], state,
+                             state_out=None if in_place else torch.empty_like(state))
+    torch.cuda.synchronize()
+    return out, st
+
+
+@pytest.mark.parametrize("N,H,g_std", [(1, 1, 1.0), (5, 3, 1.0), (64, 32, 2.0)])
+def test_decode_matches_oracle(N, H, g_std):
+    inp = decode_inputs(N, H, seed=N + H, g_std=g_std)
+    out, st = run_decode(inp)
+    out_r, fin_r = oracle.forward_inputs(inp)
+    og = out.float().cpu().numpy().astype(np.float64)[:, None]
+    assert_parity(inp, og, st.cpu().numpy().astype(np.float64), out_r, fin_r, what=f"decode N={N}")
+
+
+def test_decode_in_place_equals_out_of_place():
+    inp = decode_inputs(7, 4, seed=3)
+    a = run_decode(inp, in_place=True)
+    b = run_decode(inp, in_place=False)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_prefill_then_decode_equals_longer_prefill():
+    """kda_fwd over T tokens, then kda_decode of token T+1, matches kda_fwd over T+1."""
+    full = small(T=130, H=3, init="f32", seed=12)
+    d = dev(full)
+    out_full, fin_full = kda.kda_fwd(**d)
+    part = {n: d[n][:, :129].contiguous() for n in ("q", "k", "v", "g", "beta")}
+    _, fin_129 = kda.kda_fwd(**dict(d, **part))
+    last = lambda t: t[:, 129].contiguous()
+    out_dec, st = kda.kda_decode(last(d["q"]), last(d["k"]), last(d["v"]), last(d["g"]),
+                                 d["beta"][:, 129].contiguous(), d["scale"], d["A_log"],
+                                 d["dt_bias"], d["lower_bound"], fin_129)
+    torch.cuda.synchronize()
+    # each path against the oracle under the stated bars, and the two GPU paths against
+    # each other under the same bars (each differs from the oracle by less)
+    out_r, fin_r = oracle.forward_inputs(full)
+    od = out_dec.float().cpu().numpy().astype(np.float64)
+    assert np.abs(od - out_r[:, 129]).max() <= OUT_MAXABS and rel(od, out_r[:, 129]) <= OUT_REL
+    assert rel(st.cpu().numpy().astype(np.float64), fin_r) <= FIN_REL
+    assert rel(od, out_full[:, 129].float().cpu().numpy()) <= OUT_REL
+    assert rel(st.cpu().numpy(), fin_full.cpu().numpy()) <= FIN_REL
