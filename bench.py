@@ -67,6 +67,8 @@ def parse():
     # the decode step (one token per sequence, state in HBM) instead of the prefill
     ap.add_argument("--op", default="prefill", choices=["prefill", "decode"])
     ap.add_argument("--decode-seqs", type=int, default=256)
+    # time one of the five parity workloads (kda_inputs recipe) instead of the headline
+    ap.add_argument("--config-id", type=int, default=None, choices=[0, 1, 2, 3, 4])
     a = ap.parse_args()
     if a.batch:
         WORKLOAD["B"] = a.batch
@@ -323,9 +325,66 @@ def run_decode_bench(args, world, rank, local):
     return 0
 
 
+def run_config_bench(args, world, rank, local):
+    """Throughput of kda_fwd on one of the five parity workloads (same seeded inputs as
+    the tests), device-resident inputs, CUDA-event timing."""
+    import kda_inputs as ki
+    import linear_attention_09_b200 as kda
+    from linear_attention_09_b200 import build as kbuild
+    kbuild.build()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    wl = ki.WORKLOADS[args.config_id]
+    inp = ki.make_inputs(args.config_id)
+    d = lambda t: None if t is None else t.to(device)
+    call = dict(q=d(inp.q), k=d(inp.k), v=d(inp.v), g=d(inp.g), beta=d(inp.beta), scale=inp.scale,
+                A_log=d(inp.A_log), dt_bias=d(inp.dt_bias), lower_bound=inp.lower_bound,
+                initial_state=d(inp.initial_state), cu_seqlens=d(inp.cu_seqlens))
+    out = torch.empty_like(call["v"])
+    N, H = inp.num_seqs, inp.H
+    fin = torch.empty((N, H, 128, 128), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    step = lambda: kda.kda_fwd(**call, out=out, final_state=fin, stream=stream)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world)
+    tokens = inp.tokens
+    init_bytes = 0 if inp.initial_state is None else inp.initial_state.element_size() * 128 * 128
+    bytes_launch = tokens * H * BYTES_PER_TOKEN_HEAD + N * H * (STATE_BYTES + init_bytes) + H * 516
+    peak, peak_src = peaks()
+    achieved = bytes_launch / (ms / args.steps / 1e3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": f"KDA fwd prefill tokens/s, workload {wl.name}", "value": tokens * world * args.steps / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
+            "config": {"workload": wl.name, "tokens": tokens, "sequences": N, "heads": H, "ctas": N * H},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
+                         "alg_bytes_per_launch": bytes_launch, "kernel": KERNEL},
+            "clocks": clk.summary(), "gpu_launches": args.steps}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args.gpus)
+    if args.config_id is not None and args.impl == "ours":
+        rc = run_config_bench(args, world, rank, local)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return rc
     if args.op == "decode" and args.impl == "ours":
         rc = run_decode_bench(args, world, rank, local)
         if world > 1:
