@@ -160,6 +160,8 @@ struct Bars {
                           // state role's second product of a chunk of parity b)
     uint64_t u_free;   // u^T read out of TMEM                 (128 arrivals)
     uint64_t u_ready;  // u^T of the chunk in TMEM             (commit)
+    uint64_t nrm;      // norms and beta of the next chunk written by the state role
+                       // (one arrival per state warp)
     uint64_t ops;      // operands of the next in-chunk product written (one arrival per
                        // in-chunk warp); the issue warp waits on it
 };
@@ -170,7 +172,8 @@ struct TMaps {
 
 struct Ctx {
     uint8_t *sm;
-    float *rkq_s /* [64][2] */, *b_s, *gam_s /* [2][128] */, *osum /* [8][128] */, *dtb_s /* [128] */;
+    float *rkq_s /* [2][64][2] */, *b_s /* [2][64] */, *gam_s /* [2][128] */, *osum /* [8][128] */,
+        *dtb_s /* [128] */;  // [2] = by chunk parity
     Bars *bars;
     uint32_t tb;  // TMEM base
     int64_t h, H, tok0, len, rstride;
@@ -254,7 +257,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
 
     // ---- norms (thread: token tid/4, 16-byte chunks 2 (tid%4), 2 (tid%4) + 1 of both
     //      64-channel boxes; each 8-lane phase then reads 8 distinct bank groups) and beta
-    //      of the chunk whose tiles are in shared memory, of length Lc ----
+    //      of chunk 0 (buffer 0); the state role computes those of later chunks ----
     auto norms = [&](int Lc) {
         const float beta_c = __uint_as_float((uint32_t)beta_bits << 16);
         const int t = tid >> 2, qq = tid & 3;
@@ -314,7 +317,6 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         if (ok) {
             norms(chunk_len(0));
             gate_round(0, chunk_len(0), G0);
-            load_beta(1);
         }
     }
 
@@ -324,6 +326,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         const bool has_next = n + 1 < cx.nchunks;
         const uint32_t par = (uint32_t)n & 1u, ppar = (uint32_t)(n - 1) & 1u;
         const uint32_t skp = par ? SM_KP1 : SM_KP0;  // this chunk's k' buffer
+        const float *rkq_c = cx.rkq_s + par * 128, *b_c = cx.b_s + par * 64;  // norms, beta
 
         // ---- channel pass in two rounds of 64 channels.  Block 0 = tokens 0..31
         //      (reference token 15), block 1 = tokens 32..63 (reference token 47). ----
@@ -341,9 +344,20 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             // buffer and gamma slot (both indexed by chunk parity), is fully consumed.
             bool kok = true;
             if (round == 0 && n >= 2) kok = wait_or_flag(&bars->kp_free[par], (uint32_t)((n >> 1) - 1) & 1u, 8);
+            if (round == 0 && n >= 1) {
+                // the state role's norms of this chunk, and the u products of the previous
+                // chunk (they read T_hi / T_lo, which this round's operands overwrite, and
+                // the v tile, which is refilled below)
+                kok = wait_or_flag(&bars->nrm, (uint32_t)(n - 1) & 1u, 15) && kok;
+                kok = wait_or_flag(&bars->u_ready, ppar, 17) && kok;
+            }
             // octant sums -> chunk prefix sums and the reference values G15, G31, G47, G63
             ok = named_bar_and(BAR_IN, NT_IN, kok);
             if (!ok) break;
+            if (round == 0 && n >= 1 && tid == 0) {  // this chunk's v tile (the previous one is consumed)
+                mbar_arrive_expect_tx(&bars->v, 16384);
+                load_tile(sm + SM_V, &tm.v, &bars->v, h, ctok);
+            }
             float2 os[8];
 #pragma unroll
             for (int o = 0; o < 8; ++o) os[o] = *reinterpret_cast<const float2 *>(cx.osum + o * 128 + c0);
@@ -390,7 +404,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
                 constexpr bool kBlk0 = decltype(blk0_tag)::value;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const float2 rkq = *reinterpret_cast<const float2 *>(cx.rkq_s + 2 * (t0 + j));
+                    const float2 rkq = *reinterpret_cast<const float2 *>(rkq_c + 2 * (t0 + j));
                     const float2 kk = mul2(bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_K + rb + o16[j])),
                                            make_float2(rkq.x, rkq.x));
                     const float2 qv = mul2(bf2x2(*reinterpret_cast<const uint32_t *>(sm + SM_Q + rb + o16[j])),
@@ -465,7 +479,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             }
             const int jb = 32 * hf;
             if (ln < 64) {
-                const float bi = cx.b_s[i];
+                const float bi = b_c[i];
 #pragma unroll
                 for (int j0 = 0; j0 < 32; j0 += 4) {
                     float e4[4];
@@ -624,8 +638,8 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             for (int j0 = 0; j0 < 16; j0 += 8) {
                 const float4 x0 = *reinterpret_cast<const float4 *>(Xr + j0);
                 const float4 x1 = *reinterpret_cast<const float4 *>(Xr + j0 + 4);
-                const float4 b0 = *reinterpret_cast<const float4 *>(cx.b_s + jq + j0);
-                const float4 b1 = *reinterpret_cast<const float4 *>(cx.b_s + jq + j0 + 4);
+                const float4 b0 = *reinterpret_cast<const float4 *>(b_c + jq + j0);
+                const float4 b1 = *reinterpret_cast<const float4 *>(b_c + jq + j0 + 4);
                 const float tv[8] = {x0.x * b0.x, x0.y * b0.y, x0.z * b0.z, x0.w * b0.w,
                                      x1.x * b1.x, x1.y * b1.y, x1.z * b1.z, x1.w * b1.w};
                 uint32_t p16[4], phi[4], plo[4];
@@ -644,24 +658,16 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
                 *reinterpret_cast<uint4 *>(sm + SM_TLO + off) = make_uint4(plo[0], plo[1], plo[2], plo[3]);
             }
         }
-        // hand T to the issue warp (w^T = (k^ e^G)^T T^T, u^T = v^T (T_hi + T_lo)^T); the
-        // barrier keeps b_s of this chunk alive until every warp has written T
+        // hand T to the issue warp (w^T = (k^ e^G)^T T^T, u^T = v^T (T_hi + T_lo)^T)
         fence_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->ops);
-        named_bar(BAR_IN, NT_IN);
 
         // ---- w^T = (k^ e^G)^T T^T (fp16), u^T = v^T (T_hi + T_lo)^T (bf16) run on the issue warp ----
-        // ---- while the w/u products run: the next chunk's norms (its second box was
-        //      requested after this chunk's round 1; b_s and the norms of this chunk are
-        //      no longer read) ----
+        // ---- the next chunk's second box (requested after this chunk's round 1) ----
         bool sok = true;
-        if (has_next) {
-            sok = wait_or_flag(&bars->qkg[1], par ^ 1u, 13);
-            norms(chunk_len(n + 1));
-            load_beta(n + 2);
-        }
+        if (has_next) sok = wait_or_flag(&bars->qkg[1], par ^ 1u, 13);
         {
             // (if the issue warp gave up, this bounded wait runs out)
             const bool mok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 3);
@@ -669,10 +675,6 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         }
         tc_fence_after();
         if (!ok) break;
-        if (tid == 0 && has_next) {  // the v tile is consumed: prefetch the next chunk's
-            mbar_arrive_expect_tx(&bars->v, 16384);
-            load_tile(sm + SM_V, &tm.v, &bars->v, h, ctok + C);
-        }
 
         // ---- w (lanes = channel) -> fp16 rows of [w ; q^ e^G]; thread = (channel ln,
         //      tokens 32 hf .. 32 hf + 31) ----
@@ -733,7 +735,9 @@ __device__ void mma_role(const Ctx &cx)
         for (int st = 0; st < 4; ++st)
             mma_f16_ss(tb + TM_W, desc_sw128(skg + st * 2048, 8192, 1024),
                        desc_sw128(st16 + st * 32, 16, 1024), idw, st > 0);
-        mma_commit(&bars->mma_in);  // the in-chunk role needs only w; u goes to the state role
+        mma_commit(&bars->mma_in);  // the in-chunk role needs only w now; u goes to the state
+                                    // role, and the in-chunk role waits for it before it
+                                    // overwrites T_hi / T_lo or the v tile
 #pragma unroll
         for (int st = 0; st < 4; ++st)
             mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
@@ -823,6 +827,46 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
                 tmem_st16(tb + lq + TM_SS + k0 / 2, r);
             }
             tmem_wait_st();
+        }
+
+        // ---- the next chunk's norms and beta, in this role's idle time (its q, k boxes
+        //      were requested after the in-chunk role's rounds of this chunk; buffer
+        //      (n+1) % 2 was last read by chunk n-1, which is done).  Thread v: token
+        //      v / 2, box v % 2, 16-byte chunks visited from 4 (v % 2) on, so that each
+        //      8-lane phase reads 8 distinct bank groups. ----
+        if (n + 1 < cx.nchunks) {
+            const int m = n + 1;
+            const uint32_t mp = (uint32_t)m & 1u;
+            float beta_m = 0.f;
+            if (v < C && (int64_t)m * C + v < cx.len)
+                beta_m = bf2f(p.beta[(cx.tok0 + (int64_t)m * C + v) * H + h]);
+            ok = wait_or_flag(&bars->qkg[0], mp, 16) && wait_or_flag(&bars->qkg[1], mp, 16);
+            const int64_t rem = cx.len - (int64_t)m * C;
+            const int Lm = (int)(rem < C ? rem : C);
+            const int t = v >> 1, hb = v & 1;
+            float sq = 0.f, sk = 0.f;
+#pragma unroll 2
+            for (int ch = 0; ch < 8; ++ch) {
+                const uint32_t off = (uint32_t)hb * 8192u + sw(t, (uint32_t)((ch + 4 * hb) & 7) * 16u);
+                const uint4 qr = *reinterpret_cast<const uint4 *>(sm + SM_Q + off);
+                const uint4 kr = *reinterpret_cast<const uint4 *>(sm + SM_K + off);
+                const uint32_t qw[4] = {qr.x, qr.y, qr.z, qr.w}, kw[4] = {kr.x, kr.y, kr.z, kr.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 qf = bf2x2(qw[e]), kf = bf2x2(kw[e]);
+                    sq += qf.x * qf.x + qf.y * qf.y;
+                    sk += kf.x * kf.x + kf.y * kf.y;
+                }
+            }
+            sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+            sk += __shfl_xor_sync(0xffffffffu, sk, 1);
+            if (hb == 0)
+                *reinterpret_cast<float2 *>(cx.rkq_s + mp * 128 + 2 * t) =
+                    (t < Lm) ? make_float2(rsqrtf(sk + 1e-6f), rsqrtf(sq + 1e-6f)) : make_float2(0.f, 0.f);
+            if (v < C) cx.b_s[mp * 64 + v] = (v < Lm) ? __fdividef(1.f, 1.f + ex2(-beta_m * kLog2e)) : 0.f;
+            __syncwarp();
+            if ((v & 31) == 0) mbar_arrive(&bars->nrm);
+            if (!ok) break;
         }
 
         // ---- wait for the chunk's operands; MMA1: D1 = S~^T [w ; q^ e^G]^T ----
@@ -973,8 +1017,8 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
     Ctx cx;
     cx.sm = sm;
     cx.rkq_s = reinterpret_cast<float *>(sm + SM_MISC);
-    cx.b_s = cx.rkq_s + 128;
-    cx.gam_s = cx.b_s + 64;     // [2][128]
+    cx.b_s = cx.rkq_s + 256;    // [2][64]
+    cx.gam_s = cx.b_s + 128;    // [2][128]
     cx.osum = cx.gam_s + 256;   // [8][128]
     cx.bars = reinterpret_cast<Bars *>(cx.osum + 1024);
     uint32_t *tbase_s = reinterpret_cast<uint32_t *>(cx.bars + 1);
@@ -1009,6 +1053,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
         mbar_init(&b->u_free, NT_ST);
         mbar_init(&b->ops, NT_IN / 32);
         mbar_init(&b->u_ready, 1);
+        mbar_init(&b->nrm, NT_ST / 32);
         fence_mbar_init();
     }
     if (warp == 0) {
