@@ -159,9 +159,6 @@ struct Bars {
     uint64_t kp_free[2];  // k' buffer b, gamma slot b and P consumed (commit after the
                           // state role's second product of a chunk of parity b)
     uint64_t u_free;   // u^T read out of TMEM                 (128 arrivals)
-    uint64_t u_ready;  // u^T of the chunk in TMEM             (commit)
-    uint64_t nrm;      // norms and beta of the next chunk written by the state role
-                       // (one arrival per state warp)
     uint64_t ops;      // operands of the next in-chunk product written (one arrival per
                        // in-chunk warp); the issue warp waits on it
 };
@@ -257,8 +254,8 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
 
     // ---- norms (thread: token tid/4, 16-byte chunks 2 (tid%4), 2 (tid%4) + 1 of both
     //      64-channel boxes; each 8-lane phase then reads 8 distinct bank groups) and beta
-    //      of chunk 0 (buffer 0); the state role computes those of later chunks ----
-    auto norms = [&](int Lc) {
+    //      of the chunk whose tiles are in shared memory, of length Lc, into buffer buf ----
+    auto norms = [&](int Lc, int buf) {
         const float beta_c = __uint_as_float((uint32_t)beta_bits << 16);
         const int t = tid >> 2, qq = tid & 3;
         float sq = 0.f, sk = 0.f;
@@ -280,9 +277,9 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         sq += __shfl_xor_sync(0xffffffffu, sq, 2);
         sk += __shfl_xor_sync(0xffffffffu, sk, 2);
         if (qq == 0)  // (1/|k|, 1/|q|) per token, zero past the chunk end
-            *reinterpret_cast<float2 *>(cx.rkq_s + 2 * t) =
+            *reinterpret_cast<float2 *>(cx.rkq_s + buf * 128 + 2 * t) =
                 (t < Lc) ? make_float2(rsqrtf(sk + 1e-6f), rsqrtf(sq + 1e-6f)) : make_float2(0.f, 0.f);
-        if (tid < C) cx.b_s[tid] = (tid < Lc) ? __fdividef(1.f, 1.f + ex2(-beta_c * kLog2e)) : 0.f;
+        if (tid < C) cx.b_s[buf * 64 + tid] = (tid < Lc) ? __fdividef(1.f, 1.f + ex2(-beta_c * kLog2e)) : 0.f;
     };
 
     // ---- gate of one 64-channel round: in-octant cumulative log2-decay of the pair
@@ -310,13 +307,15 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
     // Chunk 0's norms and round-0 gate run here.  For chunk n+1, the round-0 gate runs
     // while chunk n's second A/P product is on the tensor cores and the norms while its
     // w/u products are (the octant-sum barrier at the top of the round publishes them).
+    // Norms and beta are double-buffered by chunk parity.
     float2 G0[8];  // round-0 gate of the chunk about to be processed
     if (cx.nchunks > 0) {
         load_beta(0);
         ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->qkg[0], 0, 6) && wait_or_flag(&bars->qkg[1], 0, 13));
         if (ok) {
-            norms(chunk_len(0));
+            norms(chunk_len(0), 0);
             gate_round(0, chunk_len(0), G0);
+            load_beta(1);
         }
     }
 
@@ -344,13 +343,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             // buffer and gamma slot (both indexed by chunk parity), is fully consumed.
             bool kok = true;
             if (round == 0 && n >= 2) kok = wait_or_flag(&bars->kp_free[par], (uint32_t)((n >> 1) - 1) & 1u, 8);
-            if (round == 0 && n >= 1) {
-                // the state role's norms of this chunk, and the u products of the previous
-                // chunk (they read T_hi / T_lo, which this round's operands overwrite, and
-                // the v tile, which is refilled below)
-                kok = wait_or_flag(&bars->nrm, (uint32_t)(n - 1) & 1u, 15) && kok;
-                kok = wait_or_flag(&bars->u_ready, ppar, 17) && kok;
-            }
+
             // octant sums -> chunk prefix sums and the reference values G15, G31, G47, G63
             ok = named_bar_and(BAR_IN, NT_IN, kok);
             if (!ok) break;
@@ -665,9 +658,15 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         if (lane == 0) mbar_arrive(&bars->ops);
 
         // ---- w^T = (k^ e^G)^T T^T (fp16), u^T = v^T (T_hi + T_lo)^T (bf16) run on the issue warp ----
-        // ---- the next chunk's second box (requested after this chunk's round 1) ----
+        // ---- while the w/u products run: the next chunk's norms (its second box was
+        //      requested after this chunk's round 1; they go to the other buffer, since
+        //      this chunk's b may still be read by a warp finishing T) ----
         bool sok = true;
-        if (has_next) sok = wait_or_flag(&bars->qkg[1], par ^ 1u, 13);
+        if (has_next) {
+            sok = wait_or_flag(&bars->qkg[1], par ^ 1u, 13);
+            norms(chunk_len(n + 1), (int)(par ^ 1u));
+            load_beta(n + 2);
+        }
         {
             // (if the issue warp gave up, this bounded wait runs out)
             const bool mok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 3);
@@ -735,9 +734,6 @@ __device__ void mma_role(const Ctx &cx)
         for (int st = 0; st < 4; ++st)
             mma_f16_ss(tb + TM_W, desc_sw128(skg + st * 2048, 8192, 1024),
                        desc_sw128(st16 + st * 32, 16, 1024), idw, st > 0);
-        mma_commit(&bars->mma_in);  // the in-chunk role needs only w now; u goes to the state
-                                    // role, and the in-chunk role waits for it before it
-                                    // overwrites T_hi / T_lo or the v tile
 #pragma unroll
         for (int st = 0; st < 4; ++st)
             mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
@@ -746,7 +742,7 @@ __device__ void mma_role(const Ctx &cx)
         for (int st = 0; st < 4; ++st)
             mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
                        desc_sw128(slo + st * 32, 16, 1024), idu, 1);
-        mma_commit(&bars->u_ready);
+        mma_commit(&bars->mma_in);  // w and u: T, v and k^ e^G are consumed once it completes
     }
 }
 
@@ -829,46 +825,6 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
             tmem_wait_st();
         }
 
-        // ---- the next chunk's norms and beta, in this role's idle time (its q, k boxes
-        //      were requested after the in-chunk role's rounds of this chunk; buffer
-        //      (n+1) % 2 was last read by chunk n-1, which is done).  Thread v: token
-        //      v / 2, box v % 2, 16-byte chunks visited from 4 (v % 2) on, so that each
-        //      8-lane phase reads 8 distinct bank groups. ----
-        if (n + 1 < cx.nchunks) {
-            const int m = n + 1;
-            const uint32_t mp = (uint32_t)m & 1u;
-            float beta_m = 0.f;
-            if (v < C && (int64_t)m * C + v < cx.len)
-                beta_m = bf2f(p.beta[(cx.tok0 + (int64_t)m * C + v) * H + h]);
-            ok = wait_or_flag(&bars->qkg[0], mp, 16) && wait_or_flag(&bars->qkg[1], mp, 16);
-            const int64_t rem = cx.len - (int64_t)m * C;
-            const int Lm = (int)(rem < C ? rem : C);
-            const int t = v >> 1, hb = v & 1;
-            float sq = 0.f, sk = 0.f;
-#pragma unroll 2
-            for (int ch = 0; ch < 8; ++ch) {
-                const uint32_t off = (uint32_t)hb * 8192u + sw(t, (uint32_t)((ch + 4 * hb) & 7) * 16u);
-                const uint4 qr = *reinterpret_cast<const uint4 *>(sm + SM_Q + off);
-                const uint4 kr = *reinterpret_cast<const uint4 *>(sm + SM_K + off);
-                const uint32_t qw[4] = {qr.x, qr.y, qr.z, qr.w}, kw[4] = {kr.x, kr.y, kr.z, kr.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 qf = bf2x2(qw[e]), kf = bf2x2(kw[e]);
-                    sq += qf.x * qf.x + qf.y * qf.y;
-                    sk += kf.x * kf.x + kf.y * kf.y;
-                }
-            }
-            sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-            sk += __shfl_xor_sync(0xffffffffu, sk, 1);
-            if (hb == 0)
-                *reinterpret_cast<float2 *>(cx.rkq_s + mp * 128 + 2 * t) =
-                    (t < Lm) ? make_float2(rsqrtf(sk + 1e-6f), rsqrtf(sq + 1e-6f)) : make_float2(0.f, 0.f);
-            if (v < C) cx.b_s[mp * 64 + v] = (v < Lm) ? __fdividef(1.f, 1.f + ex2(-beta_m * kLog2e)) : 0.f;
-            __syncwarp();
-            if ((v & 31) == 0) mbar_arrive(&bars->nrm);
-            if (!ok) break;
-        }
-
         // ---- wait for the chunk's operands; MMA1: D1 = S~^T [w ; q^ e^G]^T ----
         tc_fence_before();  // the S~ stores above precede MMA1
         ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(&bars->full, par, 10));
@@ -884,12 +840,7 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
             mma_commit(&bars->mma_st);
             mma_commit(&bars->wq_free);
         }
-        {
-            // MMA1 done, and u^T of this chunk (issued after w by the issue warp) is in TMEM
-            const bool m1 = wait_or_flag(&bars->mma_st, (mma_cnt++) & 1u, 4);
-            const bool uo = wait_or_flag(&bars->u_ready, par, 14);
-            ok = named_bar_and(BAR_ST, NT_ST, m1 && uo);
-        }
+        ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(&bars->mma_st, (mma_cnt++) & 1u, 4));
         tc_fence_after();
         if (!ok) break;
 
@@ -1052,8 +1003,6 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
         mbar_init(&b->kp_free[1], 1);
         mbar_init(&b->u_free, NT_ST);
         mbar_init(&b->ops, NT_IN / 32);
-        mbar_init(&b->u_ready, 1);
-        mbar_init(&b->nrm, NT_ST / 32);
         fence_mbar_init();
     }
     if (warp == 0) {
