@@ -89,6 +89,9 @@ typedef struct CUstream_st *kda_stream_t;
  *   of length 0 returns its initial state (or zeros) as final state and writes
  *   no output; tokens outside [cu_seqlens[0], cu_seqlens[num_seqs]) are not
  *   written.
+ * The kernel reads q, k, v, g, beta in tiles of 64 tokens, so the last tile of a
+ *   sequence also reads up to 63 rows after it; those tokens are masked, but the
+ *   rows must hold finite values (rows past the end of the tensors read as zero).
  * stream: the work is enqueued on it; the call does not synchronise.
  * T == 0 is valid: only final_state is written.
  * Returns KDA_OK or a negative code (see above).  Never traps the GPU.
@@ -135,10 +138,14 @@ size_t kda_fwd_host_workspace_size(int64_t B, int64_t T, int64_t H, int64_t K, i
  * Every pointer except workspace is a host pointer (pinned memory gives
  * asynchronous copies; pageable memory works but copies synchronously).  The
  * call copies the inputs into `workspace` (a device buffer of at least
- * kda_fwd_host_workspace_size(...) bytes, owned by the caller), runs kda_fwd on
- * `stream`, copies out (and final_state) back, and synchronises `stream` before
- * returning, so the host buffers are ready on return.  Same return codes as
- * kda_fwd, plus KDA_ERR_WORKSPACE.
+ * kda_fwd_host_workspace_size(...) bytes, owned by the caller), runs the pass and
+ * copies out (and final_state) back, and synchronises `stream` before returning,
+ * so the host buffers are ready on return.  The work is pipelined over up to 8
+ * pieces (batch entries, or consecutive varlen sequences of about equal token
+ * counts): the copies in of one piece (on `stream`), the kernel of another and the
+ * copies out of a third (two library-owned streams per host thread and device)
+ * overlap.  Output rows of tokens outside every sequence are not written.  Same
+ * return codes as kda_fwd, plus KDA_ERR_WORKSPACE.
  */
 int kda_fwd_host(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
                  const kda_bf16 *beta, float scale, const float *A_log, const float *dt_bias,

@@ -239,6 +239,68 @@ extern "C" size_t kda_fwd_host_workspace_size(int64_t B, int64_t T, int64_t H, i
     return host_total(host_sizes(B, T, H, N, initial_state_dtype, want_final_state, varlen));
 }
 
+namespace {
+
+// Pieces of a host-buffer call: contiguous token ranges with their contiguous state
+// ranges (batch entries, or consecutive sequences of a varlen batch of about equal
+// token counts), so that the copies of one piece overlap the kernel of another.
+struct Piece {
+    int64_t tok0, toks;  // rows of the [tokens, H, *] tensors
+    int64_t seq0, seqs;  // states [seq0, seq0 + seqs)
+};
+
+int plan_pieces(int64_t B, int64_t T, const int64_t *cu_host, int64_t num_seqs, Piece *out,
+                int max_pieces)
+{
+    int n = 0;
+    if (!cu_host) {
+        const int64_t per = (B + max_pieces - 1) / max_pieces;
+        for (int64_t b = 0; b < B; b += per) {
+            const int64_t nb = (B - b < per) ? B - b : per;
+            out[n++] = Piece{b * T, nb * T, b, nb};
+        }
+        return n;
+    }
+    const int64_t total = cu_host[num_seqs] - cu_host[0];
+    const int64_t target = (total + max_pieces - 1) / max_pieces;
+    int64_t s0 = 0;
+    while (s0 < num_seqs) {
+        int64_t s1 = s0 + 1;
+        while (s1 < num_seqs && cu_host[s1] - cu_host[s0] < target && n < max_pieces - 1) ++s1;
+        if (n == max_pieces - 1) s1 = num_seqs;
+        out[n++] = Piece{cu_host[s0], cu_host[s1] - cu_host[s0], s0, s1 - s0};
+        s0 = s1;
+    }
+    return n;
+}
+
+// Helper streams and events of the pipelined host path, per host thread and device
+// (created once; a thread's calls on one device are serialised by the final sync).
+struct HostPipe {
+    cudaStream_t comp = nullptr, d2h = nullptr;
+    cudaEvent_t ev[2 * 8 + 1] = {};
+    bool ok = false;
+};
+
+HostPipe *host_pipe()
+{
+    static thread_local HostPipe pipes[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    HostPipe &hp = pipes[dev];
+    if (!hp.ok) {
+        if (cudaStreamCreateWithFlags(&hp.comp, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess)
+            return nullptr;
+        for (auto &e : hp.ev)
+            if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+        hp.ok = true;
+    }
+    return &hp;
+}
+
+}  // namespace
+
 extern "C" int kda_fwd_host(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v,
                             const kda_bf16 *g, const kda_bf16 *beta, float scale,
                             const float *A_log, const float *dt_bias, float lower_bound,
@@ -258,6 +320,8 @@ extern "C" int kda_fwd_host(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16
     if (!workspace || workspace_bytes < host_total(s) || !aligned(workspace, 256))
         return KDA_ERR_WORKSPACE;
     const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    HostPipe *hp = host_pipe();
+    if (!hp) return KDA_ERR_CUDA;
     char *w = static_cast<char *>(workspace);
     auto take = [&](size_t bytes) {
         char *r = w;
@@ -267,26 +331,89 @@ extern "C" int kda_fwd_host(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16
     char *dq = take(s.qk), *dk = take(s.qk), *dg = take(s.qk), *dv = take(s.vv),
          *dout = take(s.vv), *dbeta = take(s.beta), *dalog = take(s.alog), *ddt = take(s.dt),
          *dinit = take(s.init), *dfin = take(s.fin), *dcu = take(s.cu);
-    auto h2d = [&](void *dst, const void *src, size_t n) {
-        return n == 0 || cudaMemcpyAsync(dst, src, n, cudaMemcpyHostToDevice, st) == cudaSuccess;
+    auto copy = [&](void *dst, const void *src, size_t n, cudaMemcpyKind kind, cudaStream_t on) {
+        return n == 0 || cudaMemcpyAsync(dst, src, n, kind, on) == cudaSuccess;
     };
-    if (!h2d(dq, q, s.qk) || !h2d(dk, k, s.qk) || !h2d(dg, g, s.qk) || !h2d(dv, v, s.vv) ||
-        !h2d(dbeta, beta, s.beta) || !h2d(dalog, A_log, s.alog) || !h2d(ddt, dt_bias, s.dt) ||
-        !h2d(dinit, initial_state, s.init) || !h2d(dcu, cu_seqlens, s.cu))
+    const size_t row = (size_t)H * kda::kHead * 2;                 // bytes per token row
+    const size_t st_in = s.init / (size_t)(N > 0 ? N : 1), st_out = s.fin / (size_t)(N > 0 ? N : 1);
+    // parameters first, then the pieces: copy in (stream st) -> kernel (comp) -> copy out (d2h)
+    if (!copy(dalog, A_log, s.alog, cudaMemcpyHostToDevice, st) ||
+        !copy(ddt, dt_bias, s.dt, cudaMemcpyHostToDevice, st) ||
+        !copy(dcu, cu_seqlens, s.cu, cudaMemcpyHostToDevice, st))
         return KDA_ERR_CUDA;
-    rc = kda_fwd(reinterpret_cast<const kda_bf16 *>(dq), reinterpret_cast<const kda_bf16 *>(dk),
-                 reinterpret_cast<const kda_bf16 *>(dv), reinterpret_cast<const kda_bf16 *>(dg),
-                 reinterpret_cast<const kda_bf16 *>(dbeta), scale,
-                 reinterpret_cast<const float *>(dalog), reinterpret_cast<const float *>(ddt),
-                 lower_bound, initial_state ? dinit : nullptr, initial_state_dtype,
-                 final_state ? reinterpret_cast<float *>(dfin) : nullptr,
-                 cu_seqlens ? reinterpret_cast<const int64_t *>(dcu) : nullptr, num_seqs,
-                 reinterpret_cast<kda_bf16 *>(dout), B, T, H, K, V, stream);
-    if (rc != KDA_OK) return rc;
-    if (s.vv && cudaMemcpyAsync(out, dout, s.vv, cudaMemcpyDeviceToHost, st) != cudaSuccess)
-        return KDA_ERR_CUDA;
-    if (s.fin &&
-        cudaMemcpyAsync(final_state, dfin, s.fin, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    Piece pcs[8];
+    const int np = (B * T == 0) ? 0 : plan_pieces(B, T, cu_seqlens, num_seqs, pcs, 8);
+    // A varlen piece's last tile also reads up to 63 rows after it, which belong to the
+    // next piece and may not be copied in yet; the kernel masks those tokens but needs
+    // finite values there, so they start as zeros.
+    if (cu_seqlens) {
+        const int64_t rows = B * T;
+        for (int i = 0; i + 1 < np; ++i) {
+            const int64_t r0 = pcs[i].tok0 + pcs[i].toks;
+            const int64_t nr = (rows - r0 < kda::kHead / 2) ? rows - r0 : kda::kHead / 2;
+            if (nr <= 0) continue;
+            char *bases[4] = {dq, dk, dg, dv};
+            for (char *b : bases)
+                if (cudaMemsetAsync(b + (size_t)r0 * row, 0, (size_t)nr * row, st) != cudaSuccess)
+                    return KDA_ERR_CUDA;
+            if (cudaMemsetAsync(dbeta + (size_t)r0 * H * 2, 0, (size_t)nr * H * 2, st) != cudaSuccess)
+                return KDA_ERR_CUDA;
+        }
+    }
+    int launches = 0;
+    for (int i = 0; i < np; ++i) {
+        const Piece &pc = pcs[i];
+        const size_t o = (size_t)pc.tok0 * row, nb = (size_t)pc.toks * row;
+        const size_t ob = (size_t)pc.tok0 * H * 2, nbb = (size_t)pc.toks * H * 2;
+        if (!copy(dq + o, (const char *)q + o, nb, cudaMemcpyHostToDevice, st) ||
+            !copy(dk + o, (const char *)k + o, nb, cudaMemcpyHostToDevice, st) ||
+            !copy(dg + o, (const char *)g + o, nb, cudaMemcpyHostToDevice, st) ||
+            !copy(dv + o, (const char *)v + o, nb, cudaMemcpyHostToDevice, st) ||
+            !copy(dbeta + ob, (const char *)beta + ob, nbb, cudaMemcpyHostToDevice, st) ||
+            !copy(dinit + pc.seq0 * st_in, (const char *)initial_state + pc.seq0 * st_in,
+                  pc.seqs * st_in, cudaMemcpyHostToDevice, st) ||
+            cudaEventRecord(hp->ev[2 * i], st) != cudaSuccess ||
+            cudaStreamWaitEvent(hp->comp, hp->ev[2 * i], 0) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        // the piece as its own call: a batch slice, or a range of varlen sequences
+        // (cu_seqlens holds absolute token offsets, so only its start moves)
+        const bool varlen = cu_seqlens != nullptr;
+        rc = kda_fwd(reinterpret_cast<const kda_bf16 *>(varlen ? dq : dq + o),
+                     reinterpret_cast<const kda_bf16 *>(varlen ? dk : dk + o),
+                     reinterpret_cast<const kda_bf16 *>(varlen ? dv : dv + o),
+                     reinterpret_cast<const kda_bf16 *>(varlen ? dg : dg + o),
+                     reinterpret_cast<const kda_bf16 *>(varlen ? dbeta : dbeta + ob), scale,
+                     reinterpret_cast<const float *>(dalog), reinterpret_cast<const float *>(ddt),
+                     lower_bound, initial_state ? dinit + pc.seq0 * st_in : nullptr,
+                     initial_state_dtype,
+                     final_state ? reinterpret_cast<float *>(dfin + pc.seq0 * st_out) : nullptr,
+                     varlen ? reinterpret_cast<const int64_t *>(dcu) + pc.seq0 : nullptr,
+                     varlen ? pc.seqs : 0,
+                     reinterpret_cast<kda_bf16 *>(varlen ? dout : dout + o),
+                     varlen ? 1 : pc.seqs, varlen ? B * T : T, H, K, V,
+                     reinterpret_cast<kda_stream_t>(hp->comp));
+        if (rc != KDA_OK) return rc;
+        launches += g_last_launches;
+        if (cudaEventRecord(hp->ev[2 * i + 1], hp->comp) != cudaSuccess ||
+            cudaStreamWaitEvent(hp->d2h, hp->ev[2 * i + 1], 0) != cudaSuccess ||
+            !copy((char *)out + o, dout + o, nb, cudaMemcpyDeviceToHost, hp->d2h) ||
+            !copy((char *)final_state + pc.seq0 * st_out, dfin + pc.seq0 * st_out,
+                  final_state ? pc.seqs * st_out : 0, cudaMemcpyDeviceToHost, hp->d2h))
+            return KDA_ERR_CUDA;
+    }
+    if (np == 0 && final_state) {  // no tokens: the final state is the initial one
+        if (!copy(dinit, initial_state, s.init, cudaMemcpyHostToDevice, st)) return KDA_ERR_CUDA;
+        rc = kda_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, scale, nullptr, nullptr,
+                     lower_bound, initial_state ? dinit : nullptr, initial_state_dtype,
+                     reinterpret_cast<float *>(dfin), nullptr, 0, nullptr, B, 0, H, K, V, stream);
+        if (rc != KDA_OK) return rc;
+        launches = g_last_launches;
+        if (!copy(final_state, dfin, s.fin, cudaMemcpyDeviceToHost, st)) return KDA_ERR_CUDA;
+    }
+    g_last_launches = launches;
+    // the caller's stream waits for the copies out, then everything is complete
+    if (cudaEventRecord(hp->ev[16], hp->d2h) != cudaSuccess ||
+        cudaStreamWaitEvent(st, hp->ev[16], 0) != cudaSuccess)
         return KDA_ERR_CUDA;
     return cudaStreamSynchronize(st) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }

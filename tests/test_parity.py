@@ -301,3 +301,21 @@ def test_prefill_then_decode_equals_longer_prefill():
     assert rel(st.cpu().numpy().astype(np.float64), fin_r) <= FIN_REL
     assert rel(od, out_full[:, 129].float().cpu().numpy()) <= OUT_REL
     assert rel(st.cpu().numpy(), fin_full.cpu().numpy()) <= FIN_REL
+
+
+@pytest.mark.parametrize("case", ["batch3", "varlen"])
+def test_pipelined_host_entry_matches_device_entry(case):
+    """The host entry point splits the call into pieces (batch entries / groups of
+    sequences) with overlapped copies; the result is bit for bit the device call's."""
+    if case == "batch3":
+        inp = ki.make_inputs(ki.Workload("h3", B=3, T=200, H=2, init_state="f32"), 31)
+    else:
+        inp = small(lengths=[70, 0, 1, 130, 64, 257, 3, 90, 33, 200], init="bf16", seed=32)
+    out_d, fin_d = run_gpu(inp)
+    pin = lambda t: None if t is None else t.pin_memory()
+    out_h, fin_h = kda.kda_fwd_host(pin(inp.q), pin(inp.k), pin(inp.v), pin(inp.g), pin(inp.beta),
+                                    inp.scale, inp.A_log, inp.dt_bias, inp.lower_bound,
+                                    initial_state=pin(inp.initial_state), cu_seqlens=inp.cu_seqlens)
+    for (b, t0, nn) in inp.seq_bounds():
+        np.testing.assert_array_equal(out_h[b, t0:t0 + nn].float().numpy(), out_d[b, t0:t0 + nn])
+    np.testing.assert_array_equal(fin_h.numpy(), fin_d)
