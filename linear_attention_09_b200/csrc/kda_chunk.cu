@@ -497,9 +497,10 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         tc_fence_after();
 
         // ---- X = (I + Diag(b) A)^-1 by blocked forward substitution on 16 x 16 blocks.
-        //      Diagonal blocks: thread = (block I, column j), row sums split four ways.
-        if (tid < 64) {
-            const int I = tid >> 4, j = tid & 15, base = 16 * I;
+        //      Diagonal blocks: warp I (one per scheduler) solves block I, lane = column j
+        //      (lanes 16..31 idle), row sums split four ways.
+        if (warp < 4 && lane < 16) {
+            const int I = warp, j = lane, base = 16 * I;
             float x[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -517,9 +518,9 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             }
 #pragma unroll
             for (int i = 0; i < 16; ++i) Xm[(base + i) * LST + base + j] = x[i];
-        } else {
+        } else if (warp >= 4) {
             // zero the blocks above the block diagonal
-            for (int e = tid - 64; e < 6 * 256; e += NT_IN - 64) {
+            for (int e = tid - 128; e < 6 * 256; e += NT_IN - 128) {
                 const int blkid = e >> 8, r = (e >> 4) & 15, cc = e & 15;
                 const int I = blkid < 3 ? 0 : (blkid < 5 ? 1 : 2);
                 const int J = blkid < 3 ? blkid + 1 : (blkid < 5 ? blkid - 1 : 3);
@@ -578,9 +579,10 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             }
             named_bar(BAR_IN, NT_IN);
             {
-                // Zb = L_hl X_ll: thread = (row r = lane, columns 4 warp ..+3); rows m < 4 warp
-                // of X_ll are zero in these columns
-                const int r = lane, c4 = 4 * warp;
+                // Zb = L_hl X_ll: thread = (row r = lane, columns c4 ..+3); rows m < c4 of
+                // X_ll are zero in these columns.  Column groups 0,1,2,3,7,6,5,4 for warps
+                // 0..7, so that the two warps of each scheduler (w, w+4) share 9 quads.
+                const int r = lane, c4 = 4 * (warp < 4 ? warp : 11 - warp);
                 const float *Ar = Lm + (32 + r) * LST;
                 float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
                 for (int m = c4; m < 32; m += 4) {
@@ -599,9 +601,10 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             }
             named_bar(BAR_IN, NT_IN);
             {
-                // X_hl = -X_hh Zb: thread = (rows 4 warp ..+3 of the half, column c = lane);
-                // X_hh is lower triangular, so row r needs m <= r only
-                const int r4 = 4 * warp, c = lane;
+                // X_hl = -X_hh Zb: thread = (rows r4 ..+3 of the half, column c = lane);
+                // X_hh is lower triangular, so row r needs m <= r only (row groups
+                // permuted as the column groups above)
+                const int r4 = 4 * (warp < 4 ? warp : 11 - warp), c = lane;
                 float a[4] = {0.f, 0.f, 0.f, 0.f}, b[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int m = 0; m < r4 + 4; m += 4) {
                     const float z0 = Zb[(m + 0) * ZST + c], z1 = Zb[(m + 1) * ZST + c];
