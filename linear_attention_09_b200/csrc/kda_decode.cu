@@ -8,7 +8,8 @@
 // One pass reads S (the two contractions S'^T k^ and S'^T q^), one pass writes it:
 // every thread keeps its 64 entries of S' in registers in between.  The step is
 // bound by HBM traffic (128 KB of state per token-head), so it runs on the CUDA
-// cores with coalesced row accesses; there is no contraction worth a tensor core.
+// cores with coalesced row accesses (streaming cache hints: the state is touched
+// once per step); there is no contraction worth a tensor core.
 #include "kda.h"
 #include "kda_internal.cuh"
 
@@ -71,7 +72,7 @@ __global__ void __launch_bounds__(DT) decode_kernel(const DecodeParams p)
     const int c0 = half * RH;
     float s[RH];
 #pragma unroll
-    for (int i = 0; i < RH; ++i) s[i] = p.state_in[sbase + (size_t)(c0 + i) * kHead];
+    for (int i = 0; i < RH; ++i) s[i] = __ldcs(p.state_in + sbase + (size_t)(c0 + i) * kHead);
     float dk = 0.f, dq = 0.f;
 #pragma unroll
     for (int i = 0; i < RH; ++i) {
@@ -88,7 +89,7 @@ __global__ void __launch_bounds__(DT) decode_kernel(const DecodeParams p)
     // ---- write pass: S = S' + b k^ r^T ----
     const float br = b * r;
 #pragma unroll
-    for (int i = 0; i < RH; ++i) p.state_out[sbase + (size_t)(c0 + i) * kHead] = s[i] + br * kh_s[c0 + i];
+    for (int i = 0; i < RH; ++i) __stcs(p.state_out + sbase + (size_t)(c0 + i) * kHead, s[i] + br * kh_s[c0 + i]);
 }
 
 }  // namespace
