@@ -1,4 +1,4 @@
-"""CPU fp64 oracle of the KDA forward pass -- TEST INFRASTRUCTURE ONLY.
+"""CPU fp64 oracle of the KDA forward and backward passes -- TEST INFRASTRUCTURE ONLY.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  The product path (the CUDA library and
@@ -48,6 +48,13 @@ def _load():
             lib.kda_oracle_fwd.restype = I
             lib.kda_oracle_core.argtypes = [I64, I64, I64, P, P, P, P, P, D, P, P, P]
             lib.kda_oracle_core.restype = I
+            lib.kda_oracle_fwd_f64.argtypes = [P, P, P, P, P, D, P, P, D, P, P, P, I64, P,
+                                               I64, I64, I64, I64, I64, D]
+            lib.kda_oracle_fwd_f64.restype = I
+            lib.kda_oracle_bwd_f64.argtypes = [P, P, P, P, P, D, P, P, D, P, P, P, P, I64,
+                                               P, P, P, P, P, P, P, P,
+                                               I64, I64, I64, I64, I64, D]
+            lib.kda_oracle_bwd_f64.restype = I
             lib.kda_oracle_threads.argtypes = []
             lib.kda_oracle_threads.restype = I
             _lib = lib
@@ -139,3 +146,69 @@ def forward_inputs(inp, eps=EPS, want_out=True, want_final=True, mask=None):
     return forward(bits(inp.q), bits(inp.k), bits(inp.v), bits(inp.g), bits(inp.beta), inp.scale,
                    inp.A_log.numpy(), inp.dt_bias.numpy(), inp.lower_bound, init, idt, cu, eps,
                    want_out, want_final, mask)
+
+
+def _f64(a):
+    return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+
+
+def forward_f64(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, S0=None, cu_seqlens=None,
+                eps=EPS):
+    """Forward pass on raw fp64 inputs (the twin of ``forward`` that finite differences
+    can be taken of).  Shapes as in ``forward``; S0 fp64 [N,H,K,V] or None.
+    Returns (out [B,T,H,V], final [N,H,K,V]), fp64."""
+    q, k, v, g, beta, A_log, dt_bias, S0 = map(_f64, (q, k, v, g, beta, A_log, dt_bias, S0))
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int64)
+    N = B if cu is None else cu.size - 1
+    out = np.zeros((B, T, H, V), np.float64)
+    fin = np.zeros((N, H, K, V), np.float64)
+    rc = _load().kda_oracle_fwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                                    _ptr(A_log), _ptr(dt_bias), float(lower_bound), _ptr(S0),
+                                    _ptr(fin), _ptr(cu), int(N if cu is not None else 0),
+                                    _ptr(out), B, T, H, K, V, float(eps))
+    if rc != 0:
+        raise RuntimeError(f"kda_oracle_fwd_f64 failed: {rc}")
+    return out, fin
+
+
+def backward(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, dO, S0=None, dS_final=None,
+             cu_seqlens=None, eps=EPS):
+    """Gradients of L = <dO, out> + <dS_final, final> (fp64, token by token in reverse).
+
+    Inputs are raw fp64 values with the shapes of ``forward``; dO [B,T,H,V];
+    dS_final [N,H,K,V] or None (zero).  Returns a dict with dq, dk, dg [B,T,H,K],
+    dv [B,T,H,V], dbeta [B,T,H], dA_log [H], ddt_bias [H,K], dS0 [N,H,K,V].
+    Tokens outside every sequence get zeros."""
+    q, k, v, g, beta, A_log, dt_bias, S0, dO, dSf = map(
+        _f64, (q, k, v, g, beta, A_log, dt_bias, S0, dO, dS_final))
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int64)
+    N = B if cu is None else cu.size - 1
+    r = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v), dg=np.zeros_like(g),
+             dbeta=np.zeros_like(beta), dA_log=np.zeros(H), ddt_bias=np.zeros((H, K)),
+             dS0=np.zeros((N, H, K, V)))
+    rc = _load().kda_oracle_bwd_f64(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(A_log), _ptr(dt_bias),
+        float(lower_bound), _ptr(S0), _ptr(dO), _ptr(dSf), _ptr(cu),
+        int(N if cu is not None else 0), _ptr(r["dq"]), _ptr(r["dk"]), _ptr(r["dv"]), _ptr(r["dg"]),
+        _ptr(r["dbeta"]), _ptr(r["dA_log"]), _ptr(r["ddt_bias"]), _ptr(r["dS0"]),
+        B, T, H, K, V, float(eps))
+    if rc != 0:
+        raise RuntimeError(f"kda_oracle_bwd_f64 failed: {rc}")
+    return r
+
+
+def backward_inputs(inp, dO, dS_final=None, eps=EPS):
+    """``backward`` on a ``kda_inputs.KDAInputs`` (CPU tensors; bf16 values and a bf16
+    or fp32 initial state promoted exactly to fp64); dO and dS_final are CPU tensors
+    (any float dtype, promoted exactly)."""
+    import torch
+
+    d = lambda t: None if t is None else t.detach().to(torch.float64).numpy()
+    cu = None if inp.cu_seqlens is None else inp.cu_seqlens.numpy()
+    return backward(d(inp.q), d(inp.k), d(inp.v), d(inp.g), d(inp.beta), inp.scale,
+                    d(inp.A_log), d(inp.dt_bias), inp.lower_bound, d(dO), d(inp.initial_state),
+                    d(dS_final), cu, eps)
