@@ -65,7 +65,7 @@ def parse():
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--seqlen", type=int, default=None)
     # the decode step (one token per sequence, state in HBM) instead of the prefill
-    ap.add_argument("--op", default="prefill", choices=["prefill", "decode"])
+    ap.add_argument("--op", default="prefill", choices=["prefill", "decode", "backward"])
     ap.add_argument("--decode-seqs", type=int, default=256)
     # time one of the five parity workloads (kda_inputs recipe) instead of the headline
     ap.add_argument("--config-id", type=int, default=None, choices=[0, 1, 2, 3, 4])
@@ -325,6 +325,80 @@ def run_decode_bench(args, world, rank, local):
     return 0
 
 
+# Backward pass: compulsory bytes per token-head (q, k, v, g, dO, beta read as bf16;
+# dq, dk, dv, dg, dbeta written as fp32) and the minimal arithmetic of reverse mode
+# through the token recurrence: one forward step (alpha S, S^T k, rank-1 update: 5 K V
+# FLOP) and the reverse step (12 K V FLOP), FMA = 2 FLOP.
+BWD_BYTES_PER_TOKEN_HEAD = 5 * 256 + 2 + 4 * 512 + 4
+BWD_FLOPS_PER_TOKEN_HEAD = 17 * 128 * 128
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+BWD_KERNEL_SRC = ["linear_attention_09_b200/csrc/kda_backward.cu"]
+
+
+def run_backward_bench(args, world, rank, local):
+    """Backward pass on the headline prefill shape: kda_bwd with dL/dout given and
+    dL/dS_0 returned (no dL/dS_final), device-resident inputs, CUDA-event timing."""
+    import linear_attention_09_b200 as kda
+    from linear_attention_09_b200 import build as kbuild
+    kbuild.build()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = WORKLOAD
+    B, T, H = args.batch or w["B"], args.seqlen or w["T"], w["H"]
+    inp = device_inputs(args.seed + 1000 * rank, device)
+    if (B, T) != (w["B"], w["T"]):
+        for key in ("q", "k", "v", "g", "beta"):
+            inp[key] = inp[key][:B, :T].contiguous()
+    gen = torch.Generator(device=device)
+    gen.manual_seed(args.seed + 7 + 1000 * rank)
+    dO = torch.empty((B, T, H, w["V"]), device=device).normal_(0.0, 1.0, generator=gen)
+    dO = dO.to(torch.bfloat16)
+    ws = torch.empty(kda.kda_bwd_workspace_size(B, T, H), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        kda.kda_bwd(**inp, d_out=dO, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    launches = kda.kda_last_launch_count()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_local = ev0.elapsed_time(ev1)
+    ms = max_over_ranks(ms_local, world)
+    th = B * T * H
+    flops = th * BWD_FLOPS_PER_TOKEN_HEAD
+    achieved = flops / (ms_local / args.steps / 1e3) / 1e12
+    bytes_launch = th * BWD_BYTES_PER_TOKEN_HEAD + B * H * STATE_BYTES
+    if rank == 0:
+        print(json.dumps({
+            "metric": "KDA bwd tokens/s (H=32, K=V=128, T=32K)", "value":
+            B * T * world * args.steps / (ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16-in/fp32", "data": "synthetic",
+            "config": {"workload": f"bwd_B{B}_T{T}_H{H}_g2", "global_batch": B * world,
+                       "seq_len": T, "heads": H,
+                       "l2": f"inputs + gradients {bytes_launch / 1e9:.1f} GB per rank > 126 MB L2"},
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS,
+                         "unit": "TFLOP/s", "frac": achieved / FP32_PEAK_TFLOPS, "traffic": None,
+                         "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
+                         "alg_flops_per_launch": flops, "alg_bytes_per_launch": bytes_launch,
+                         "hbm_gbs_algorithmic": bytes_launch / (ms_local / args.steps / 1e3) / 1e9,
+                         "kernel": "bwd_kernel"},
+            "clocks": clk.summary(), "gpu_launches": launches * args.steps}), flush=True)
+    return 0
+
+
 def run_config_bench(args, world, rank, local):
     """Throughput of kda_fwd on one of the five parity workloads (same seeded inputs as
     the tests), device-resident inputs, CUDA-event timing."""
@@ -385,8 +459,9 @@ def main():
             import torch.distributed as dist
             dist.destroy_process_group()
         return rc
-    if args.op == "decode" and args.impl == "ours":
-        rc = run_decode_bench(args, world, rank, local)
+    if args.op in ("decode", "backward") and args.impl == "ours":
+        rc = (run_decode_bench if args.op == "decode" else run_backward_bench)(args, world, rank,
+                                                                                local)
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()

@@ -173,6 +173,47 @@ int kda_decode(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kd
                float lower_bound, const float *state_in, float *state_out, kda_bf16 *out,
                int64_t N, int64_t H, int64_t K, int64_t V, kda_stream_t stream);
 
+/*
+ * kda_bwd -- backward pass of kda_fwd: the gradients of
+ *   L = sum over tokens of <d_out_t, out_t>  +  <d_final_state, final_state>
+ * with respect to every input (reverse mode through the recurrence of the FlashKDA
+ * pages, 7minutos.es "¿Qué es la atención Kimi Delta...?"; the training step the
+ * FLA integration on github.zuobiaodaohang.com, section "作为 FLA 后端的用法", calls
+ * for).
+ *
+ * Inputs: q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, initial_state /
+ * initial_state_dtype, cu_seqlens / num_seqs, B, T, H, K, V exactly as kda_fwd
+ * (states in the S[k][v] layout), and
+ *   d_out          [B, T, H, V] bf16   dL/dout
+ *   d_final_state  [N, H, K, V] fp32   dL/dS_final, or NULL (zero)
+ * Outputs (fp32, device, written by this call):
+ *   dq, dk, dg     [B, T, H, K]       dv  [B, T, H, V]       dbeta  [B, T, H]
+ *   dA_log         [H]                ddt_bias  [H, K]  (sums over all sequences)
+ *   d_initial_state [N, H, K, V] or NULL (not requested)
+ * Token rows outside every sequence (varlen with cu_seqlens[0] > 0 or
+ * cu_seqlens[N] < T) are not written.  The gradient of the gate clamp
+ * lam = max(lower_bound, z) is taken as zero where z < lower_bound.
+ *
+ * workspace: device memory of at least kda_bwd_workspace_size(...) bytes, 256-byte
+ * aligned, owned by the caller and free for reuse once the call's work on stream
+ * is done.  It holds the state before every 64-token chunk (64 KB per chunk and
+ * head) and per-CTA scratch.
+ * The call is asynchronous on stream.  Returns KDA_OK or the codes of kda_fwd
+ * (d_out takes the place of out in the checks), plus KDA_ERR_NULL for a missing
+ * gradient output, KDA_ERR_ALIGN (16 bytes for dq, dk, dv, dg; 4 for the other fp32
+ * buffers; 256 for the workspace) and KDA_ERR_WORKSPACE.
+ */
+size_t kda_bwd_workspace_size(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                              int64_t num_seqs);
+int kda_bwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
+            const kda_bf16 *beta, float scale, const float *A_log, const float *dt_bias,
+            float lower_bound, const void *initial_state, int initial_state_dtype,
+            const kda_bf16 *d_out, const float *d_final_state, const int64_t *cu_seqlens,
+            int64_t num_seqs, float *dq, float *dk, float *dv, float *dg, float *dbeta,
+            float *dA_log, float *ddt_bias, float *d_initial_state, void *workspace,
+            size_t workspace_bytes, int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+            kda_stream_t stream);
+
 /* Human-readable text of a return code (static storage; never NULL). */
 const char *kda_strerror(int code);
 

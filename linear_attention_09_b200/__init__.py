@@ -1,12 +1,12 @@
-"""Python binding of libkda.so, the B200 (sm_100a) Kimi Delta Attention forward pass.
+"""Python binding of libkda.so, the B200 (sm_100a) Kimi Delta Attention forward and backward passes.
 
 Argument marshalling only: every step of the pass runs in the CUDA kernels of
 ``libkda.so``.  PyTorch provides device memory and streams.  There is no CPU or
 PyTorch fallback: if the library cannot be loaded, the calls raise.
 
 The functions mirror the C ABI in ``include/kda.h``:
-  kda_fwd, kda_fwd_ex, kda_decode, kda_fwd_host, kda_fwd_host_workspace_size, kda_strerror,
-  kda_last_launch_count, kda_device_status.
+  kda_fwd, kda_fwd_ex, kda_decode, kda_bwd, kda_bwd_workspace_size, kda_fwd_host,
+  kda_fwd_host_workspace_size, kda_strerror, kda_last_launch_count, kda_device_status.
 """
 from __future__ import annotations
 
@@ -60,6 +60,11 @@ def lib() -> ctypes.CDLL:
             L.kda_fwd_host.restype = I
             L.kda_fwd_host_workspace_size.argtypes = [I64, I64, I64, I64, I64, I64, I, I]
             L.kda_fwd_host_workspace_size.restype = SZ
+            L.kda_bwd.argtypes = [P, P, P, P, P, F, P, P, F, P, I, P, P, P, I64, P, P, P, P, P,
+                                  P, P, P, P, SZ, I64, I64, I64, I64, I64, P]
+            L.kda_bwd.restype = I
+            L.kda_bwd_workspace_size.argtypes = [I64, I64, I64, I64, I64, I64]
+            L.kda_bwd_workspace_size.restype = SZ
             L.kda_strerror.argtypes = [I]
             L.kda_strerror.restype = ctypes.c_char_p
             L.kda_last_launch_count.argtypes = []
@@ -180,6 +185,48 @@ def kda_decode(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, state, stat
     if rc != 0:
         raise KDAError(rc, "kda_decode")
     return out, state_out
+
+
+def kda_bwd_workspace_size(B, T, H, K=HEAD, V=HEAD, num_seqs=0) -> int:
+    """Workspace bytes of ``kda_bwd`` (0 for an invalid shape)."""
+    return int(lib().kda_bwd_workspace_size(B, T, H, K, V, num_seqs))
+
+
+def kda_bwd(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, d_out, initial_state=None,
+            d_final_state=None, cu_seqlens=None, want_d_initial_state=True, workspace=None,
+            stream=None):
+    """Backward pass on CUDA tensors (the inputs of ``kda_fwd`` plus d_out bf16
+    [B,T,H,V] and d_final_state fp32 [N,H,128,128] or None).
+
+    Returns a dict of fp32 tensors: dq, dk, dg [B,T,H,128], dv [B,T,H,128], dbeta
+    [B,T,H], dA_log [H], ddt_bias [H,128] and dS0 [N,H,128,128] (None unless
+    ``want_d_initial_state``).  ``workspace`` is a CUDA uint8 tensor of at least
+    ``kda_bwd_workspace_size`` bytes (allocated here if None).
+    """
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    N = B if cu_seqlens is None else num_seqs
+    dev = q.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    g_ = dict(dq=torch.empty((B, T, H, K), **f32), dk=torch.empty((B, T, H, K), **f32),
+              dv=torch.empty((B, T, H, V), **f32), dg=torch.empty((B, T, H, K), **f32),
+              dbeta=torch.empty((B, T, H), **f32), dA_log=torch.empty((H,), **f32),
+              ddt_bias=torch.empty((H, K), **f32),
+              dS0=torch.empty((N, H, K, V), **f32) if want_d_initial_state else None)
+    need = kda_bwd_workspace_size(B, T, H, K, V, num_seqs)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    rc = lib().kda_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(A_log),
+                       _ptr(dt_bias), float(lower_bound), _ptr(initial_state),
+                       _state_dtype(initial_state), _ptr(d_out), _ptr(d_final_state),
+                       _ptr(cu_seqlens), num_seqs, _ptr(g_["dq"]), _ptr(g_["dk"]), _ptr(g_["dv"]),
+                       _ptr(g_["dg"]), _ptr(g_["dbeta"]), _ptr(g_["dA_log"]), _ptr(g_["ddt_bias"]),
+                       _ptr(g_["dS0"]), _ptr(workspace), workspace.numel(), B, T, H, K, V,
+                       _stream_handle(stream, dev))
+    if rc != 0:
+        raise KDAError(rc, "kda_bwd")
+    return g_
 
 
 def kda_fwd_raw(*args) -> int:

@@ -229,6 +229,78 @@ extern "C" int kda_decode(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *
     return KDA_OK;
 }
 
+extern "C" size_t kda_bwd_workspace_size(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                                         int64_t num_seqs)
+{
+    if (K != kda::kHead || V != kda::kHead || B < 1 || T < 0 || H < 1) return 0;
+    const int64_t N = num_seqs > 0 ? num_seqs : B;
+    return kda::bwd_layout(B * T, N, H, nullptr);
+}
+
+extern "C" int kda_bwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
+                       const kda_bf16 *beta, float scale, const float *A_log,
+                       const float *dt_bias, float lower_bound, const void *initial_state,
+                       int initial_state_dtype, const kda_bf16 *d_out,
+                       const float *d_final_state, const int64_t *cu_seqlens, int64_t num_seqs,
+                       float *dq, float *dk, float *dv, float *dg, float *dbeta, float *dA_log,
+                       float *ddt_bias, float *d_initial_state, void *workspace,
+                       size_t workspace_bytes, int64_t B, int64_t T, int64_t H, int64_t K,
+                       int64_t V, kda_stream_t stream)
+{
+    int64_t N = 0;
+    int rc = validate(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, initial_state,
+                      initial_state_dtype, nullptr, cu_seqlens, num_seqs, d_out, B, T, H, K, V,
+                      &N);
+    if (rc != KDA_OK) return rc;
+    const bool any_tokens = B * T > 0;
+    if (any_tokens && (!dq || !dk || !dv || !dg || !dbeta)) return KDA_ERR_NULL;
+    if (!dA_log || !ddt_bias || !A_log || !dt_bias) return KDA_ERR_NULL;
+    if (!aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(dg, 16) ||
+        !aligned(dbeta, 4) || !aligned(dA_log, 4) || !aligned(ddt_bias, 4) ||
+        !aligned(d_final_state, 4) || !aligned(d_initial_state, 4))
+        return KDA_ERR_ALIGN;
+    kda::BwdLayout lay{};
+    const size_t need = kda::bwd_layout(B * T, N, H, &lay);
+    if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return KDA_ERR_ALIGN;
+    if ((rc = check_device()) != KDA_OK) return rc;
+    kda::BwdParams p{};
+    p.q = reinterpret_cast<const __nv_bfloat16 *>(q);
+    p.k = reinterpret_cast<const __nv_bfloat16 *>(k);
+    p.v = reinterpret_cast<const __nv_bfloat16 *>(v);
+    p.g = reinterpret_cast<const __nv_bfloat16 *>(g);
+    p.beta = reinterpret_cast<const __nv_bfloat16 *>(beta);
+    p.dout = reinterpret_cast<const __nv_bfloat16 *>(d_out);
+    p.A_log = A_log;
+    p.dt_bias = dt_bias;
+    p.init = initial_state;
+    p.init_dtype = initial_state_dtype;
+    p.dfinal = d_final_state;
+    p.cu = cu_seqlens;
+    p.dq = dq;
+    p.dk = dk;
+    p.dv = dv;
+    p.dg = dg;
+    p.dbeta = dbeta;
+    p.dA_log = dA_log;
+    p.ddt_bias = ddt_bias;
+    p.dinit = d_initial_state;
+    char *ws = static_cast<char *>(workspace);
+    p.ckpt = reinterpret_cast<float *>(ws);
+    p.scratch = reinterpret_cast<float *>(ws + lay.ckpt_bytes);
+    p.part = reinterpret_cast<float *>(ws + lay.ckpt_bytes + lay.scratch_bytes);
+    p.scale = scale;
+    p.lower_bound = lower_bound;
+    p.B = B;
+    p.T = T;
+    p.H = H;
+    p.N = N;
+    const int n = kda::launch_backward(p, lay, reinterpret_cast<cudaStream_t>(stream));
+    if (n < 0) return n;
+    g_last_launches = n;
+    return KDA_OK;
+}
+
 extern "C" size_t kda_fwd_host_workspace_size(int64_t B, int64_t T, int64_t H, int64_t K,
                                               int64_t V, int64_t num_seqs,
                                               int initial_state_dtype, int want_final_state)

@@ -36,6 +36,33 @@ struct DecodeParams {
 
 int launch_decode(const DecodeParams &p, cudaStream_t stream);
 
+// Backward pass: gradients of <dO, out> + <dS_final, S_final>.
+struct BwdParams {
+    const __nv_bfloat16 *q, *k, *v, *g, *beta, *dout;
+    const float *A_log, *dt_bias;
+    const void *init;        // fp32 or bf16 initial state or nullptr
+    int init_dtype;
+    const float *dfinal;     // fp32 [N,H,K,V] or nullptr (zero)
+    const int64_t *cu;
+    float *dq, *dk, *dv, *dg, *dbeta;  // fp32, layouts of q, k, v, g, beta
+    float *dA_log, *ddt_bias;          // fp32 [H], [H,K]
+    float *dinit;                      // fp32 [N,H,K,V] or nullptr
+    float *ckpt, *scratch, *part;      // workspace regions
+    float scale, lower_bound;
+    int64_t B, T, H, N;
+};
+
+constexpr int kBwdMaxCtas = 148;  // persistent grid of the backward kernel
+
+struct BwdLayout {
+    int grid;
+    size_t ckpt_bytes, scratch_bytes, part_bytes;
+};
+
+// Workspace bytes of a backward call (and the split into regions).
+size_t bwd_layout(int64_t total_tokens, int64_t N, int64_t H, BwdLayout *out);
+int launch_backward(const BwdParams &p, const BwdLayout &l, cudaStream_t stream);
+
 // Kernel launcher; returns the number of kernels it enqueued (>= 0) or a negative
 // KDA_ERR_* code.
 int launch_chunked(const FwdParams &p, cudaStream_t stream);

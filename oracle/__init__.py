@@ -52,7 +52,7 @@ def _load():
                                                I64, I64, I64, I64, I64, D]
             lib.kda_oracle_fwd_f64.restype = I
             lib.kda_oracle_bwd_f64.argtypes = [P, P, P, P, P, D, P, P, D, P, P, P, P, I64,
-                                               P, P, P, P, P, P, P, P,
+                                               P, P, P, P, P, P, P, P, P,
                                                I64, I64, I64, I64, I64, D]
             lib.kda_oracle_bwd_f64.restype = I
             lib.kda_oracle_threads.argtypes = []
@@ -174,12 +174,13 @@ def forward_f64(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, S0=None, c
 
 
 def backward(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, dO, S0=None, dS_final=None,
-             cu_seqlens=None, eps=EPS):
+             cu_seqlens=None, eps=EPS, want_dlam=False):
     """Gradients of L = <dO, out> + <dS_final, final> (fp64, token by token in reverse).
 
     Inputs are raw fp64 values with the shapes of ``forward``; dO [B,T,H,V];
     dS_final [N,H,K,V] or None (zero).  Returns a dict with dq, dk, dg [B,T,H,K],
-    dv [B,T,H,V], dbeta [B,T,H], dA_log [H], ddt_bias [H,K], dS0 [N,H,K,V].
+    dv [B,T,H,V], dbeta [B,T,H], dA_log [H], ddt_bias [H,K], dS0 [N,H,K,V], and with
+    ``want_dlam`` dlam [B,T,H,K] = dL/dlam (the gate's log-decay).
     Tokens outside every sequence get zeros."""
     q, k, v, g, beta, A_log, dt_bias, S0, dO, dSf = map(
         _f64, (q, k, v, g, beta, A_log, dt_bias, S0, dO, dS_final))
@@ -189,19 +190,19 @@ def backward(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, dO, S0=None, 
     N = B if cu is None else cu.size - 1
     r = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v), dg=np.zeros_like(g),
              dbeta=np.zeros_like(beta), dA_log=np.zeros(H), ddt_bias=np.zeros((H, K)),
-             dS0=np.zeros((N, H, K, V)))
+             dS0=np.zeros((N, H, K, V)), dlam=np.zeros_like(g) if want_dlam else None)
     rc = _load().kda_oracle_bwd_f64(
         _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale), _ptr(A_log), _ptr(dt_bias),
         float(lower_bound), _ptr(S0), _ptr(dO), _ptr(dSf), _ptr(cu),
         int(N if cu is not None else 0), _ptr(r["dq"]), _ptr(r["dk"]), _ptr(r["dv"]), _ptr(r["dg"]),
         _ptr(r["dbeta"]), _ptr(r["dA_log"]), _ptr(r["ddt_bias"]), _ptr(r["dS0"]),
-        B, T, H, K, V, float(eps))
+        _ptr(r["dlam"]), B, T, H, K, V, float(eps))
     if rc != 0:
         raise RuntimeError(f"kda_oracle_bwd_f64 failed: {rc}")
     return r
 
 
-def backward_inputs(inp, dO, dS_final=None, eps=EPS):
+def backward_inputs(inp, dO, dS_final=None, eps=EPS, want_dlam=False):
     """``backward`` on a ``kda_inputs.KDAInputs`` (CPU tensors; bf16 values and a bf16
     or fp32 initial state promoted exactly to fp64); dO and dS_final are CPU tensors
     (any float dtype, promoted exactly)."""
@@ -211,4 +212,4 @@ def backward_inputs(inp, dO, dS_final=None, eps=EPS):
     cu = None if inp.cu_seqlens is None else inp.cu_seqlens.numpy()
     return backward(d(inp.q), d(inp.k), d(inp.v), d(inp.g), d(inp.beta), inp.scale,
                     d(inp.A_log), d(inp.dt_bias), inp.lower_bound, d(dO), d(inp.initial_state),
-                    d(dS_final), cu, eps)
+                    d(dS_final), cu, eps, want_dlam)

@@ -437,7 +437,9 @@ static void reverse_step(int64_t K, int64_t V, const double *Sprev, double *dS,
  * Backward of kda_oracle_fwd_f64.  Inputs as there, plus dO [B,T,H,V] and
  * dS_final [N,H,K,V] (NULL = zero).  Outputs (fp64, same layouts as the inputs):
  * dq, dk, dg [B,T,H,K], dv [B,T,H,V], dbeta [B,T,H], dA_log [H], ddt_bias [H,K],
- * dS0 [N,H,K,V] (may be NULL).  Tokens outside every sequence are left untouched.
+ * dS0 [N,H,K,V] (may be NULL), and dlam_out [B,T,H,K] = dL/dlam (may be NULL; lets a
+ * test see both sides of the clamp's kink).  Tokens outside every sequence are left
+ * untouched.
  */
 int kda_oracle_bwd_f64(const double *q, const double *k, const double *v, const double *g,
                        const double *beta, double scale, const double *A_log,
@@ -445,7 +447,8 @@ int kda_oracle_bwd_f64(const double *q, const double *k, const double *v, const 
                        const double *dO, const double *dS_final, const int64_t *cu_seqlens,
                        int64_t num_seqs, double *dq, double *dk, double *dv, double *dg,
                        double *dbeta, double *dA_log, double *ddt_bias, double *dS0,
-                       int64_t B, int64_t T, int64_t H, int64_t K, int64_t V, double eps)
+                       double *dlam_out, int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
+                       double eps)
 {
     if (B < 1 || T < 0 || H < 1 || K < 1 || V < 1)
         return -1;
@@ -530,6 +533,8 @@ int kda_oracle_bwd_f64(const double *q, const double *k, const double *v, const 
                         dAp[K] += dlam[c] * a.z[c];
                     }
                     dg[(tok * H + h) * K + c] = dx;
+                    if (dlam_out)
+                        dlam_out[(tok * H + h) * K + c] = dlam[c];
                     dAp[c] += dx;
                 }
                 dbeta[tok * H + h] = db * a.b * (1.0 - a.b);

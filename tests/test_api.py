@@ -154,3 +154,55 @@ def test_decode_empty_and_valid_without_device(L):
     assert call_decode(N=0, q=None) == 0  # nothing to do
     if not torch.cuda.is_available():
         assert call_decode() == -11
+
+
+WS = 0x4000000  # fake 256-byte aligned workspace address
+
+
+def call_bwd(**over):
+    a = dict(q=A16, k=A16 + 0x100, v=A16 + 0x200, g=A16 + 0x300, beta=A16 + 0x400, scale=0.1,
+             A_log=A16 + 0x500, dt_bias=A16 + 0x600, lb=-5.0, init=None, init_dtype=0,
+             dout=A16 + 0x700, dfin=None, cu=None, num_seqs=0, dq=A16 + 0x1000,
+             dk=A16 + 0x1100, dv=A16 + 0x1200, dg=A16 + 0x1300, dbeta=A16 + 0x1400,
+             dA=A16 + 0x1500, ddt=A16 + 0x1600, dinit=None, ws=WS, ws_bytes=None, B=1, T=64,
+             H=2, K=128, V=128, stream=None)
+    a.update(over)
+    if a["ws_bytes"] is None:
+        a["ws_bytes"] = kda.kda_bwd_workspace_size(a["B"], a["T"], a["H"], a["K"], a["V"],
+                                                   a["num_seqs"])
+    return int(kda.lib().kda_bwd(
+        a["q"], a["k"], a["v"], a["g"], a["beta"], ctypes.c_float(a["scale"]), a["A_log"],
+        a["dt_bias"], ctypes.c_float(a["lb"]), a["init"], a["init_dtype"], a["dout"], a["dfin"],
+        a["cu"], a["num_seqs"], a["dq"], a["dk"], a["dv"], a["dg"], a["dbeta"], a["dA"], a["ddt"],
+        a["dinit"], a["ws"], a["ws_bytes"], a["B"], a["T"], a["H"], a["K"], a["V"], a["stream"]))
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(K=64), -1), (dict(q=None), -2), (dict(dout=None), -2), (dict(dq=None), -2),
+    (dict(dbeta=None), -2), (dict(dA=None), -2), (dict(ddt=None), -2),
+    (dict(cu=A16 + 0x800, num_seqs=2, B=2), -3), (dict(cu=A16 + 0x800, num_seqs=0), -4),
+    (dict(lb=1.0), -5), (dict(init=A16 + 0x900, init_dtype=0), -6),
+    (dict(dq=A16 + 4), -7), (dict(dbeta=A16 + 2), -7), (dict(dfin=A16 + 2), -7),
+    (dict(ws=WS + 16), -7), (dict(T=-1), -8), (dict(ws=None), -10), (dict(ws_bytes=1024), -10),
+    (dict(scale=float("inf")), -12),
+])
+def test_bwd_invalid_arguments_rejected_on_host(L, over, code):
+    assert call_bwd(**over) == code
+
+
+def test_bwd_workspace_size():
+    """64 KB per 64-token chunk and head (plus one slot per sequence), per-CTA scratch
+    and the per-(sequence, head) parameter partials."""
+    one = kda.kda_bwd_workspace_size(1, 64, 1)
+    assert one >= 2 * 65536 + 8 * 65536
+    big = kda.kda_bwd_workspace_size(4, 32768, 32)
+    assert big >= (4 * 32768 // 64 + 4) * 32 * 65536
+    assert kda.kda_bwd_workspace_size(1, 64, 1, K=64) == 0
+    assert kda.kda_bwd_workspace_size(1, 1000, 2, num_seqs=3) >= (1000 // 64 + 3) * 2 * 65536
+
+
+def test_bwd_valid_arguments_without_device(L):
+    import torch
+    if not torch.cuda.is_available():
+        assert call_bwd() == -11
+        assert call_bwd(T=0, q=None, dout=None, dq=None) == -11  # T = 0 still writes dA_log

@@ -217,3 +217,18 @@ def test_forward_twin_equals_bf16_forward(varlen):
                                       d(inp.initial_state), cu)
     np.testing.assert_array_equal(out_f, out_b)
     np.testing.assert_array_equal(fin_f, fin_b)
+
+
+def test_dlam_is_the_gate_gradient_before_the_activation():
+    """dg = -dlam exp(A_log) sigmoid(x) where the clamp is open, 0 where it holds
+    (dg itself is pinned by finite differences above)."""
+    rng = np.random.default_rng(12)
+    c = rand_case(rng, B=1, T=6, H=2, K=6, V=3, g_mu=1.0, g_std=3.0)
+    r = oracle.backward(c["q"], c["k"], c["v"], c["g"], c["beta"], 0.5, c["A_log"], c["dt_bias"],
+                        LB, c["dO"], c["S0"], c["dSf"], None, want_dlam=True)
+    x = c["g"] + c["dt_bias"][None, None]
+    ea = np.exp(c["A_log"])[None, None, :, None]
+    z = -ea * np.logaddexp(0, x)
+    want = np.where(z >= LB, -r["dlam"] * ea / (1 + np.exp(-x)), 0.0)
+    np.testing.assert_allclose(r["dg"], want, rtol=1e-12, atol=1e-15)
+    assert np.any(r["dlam"][z < LB] != 0)  # the kink cuts a nonzero gradient
