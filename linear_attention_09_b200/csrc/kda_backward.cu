@@ -15,20 +15,24 @@
 // holds the value at lb, i.e. where -exp(A_log) softplus(x) < lb).
 //
 // Schedule.  One CTA of 512 threads per (sequence, head), persistent over the
-// units.  Thread (v, qr): value column v, rows c = 32 qr + i (i < 32); S and dS live
-// in registers.  The columns of S evolve independently (the reductions over k
-// stay inside one warp: the four row quarters of a column are adjacent lanes).
+// units.  Thread (r8, cg): rows c = 32 g + 4 r8 + j (g, j < 4; 16 rows) of the two
+// value columns 2 cg, 2 cg + 1; S and dS live in registers.  The columns of S evolve
+// independently; the reductions over k of one column stay inside a warp (its eight
+// row groups are adjacent lanes).  Each row's k^ / alpha / q^ values, read from
+// shared memory, serve two columns: a step is bound by the shared-memory-to-register
+// path, so the bytes read per step are what this layout halves.
 //   1. Forward sweep over the sequence; the state before every 64-token chunk is
 //      stored in the workspace.
 //   2. Reverse over the chunks.  For each chunk: re-run it from its checkpoint and
 //      keep the state before each 8-token sub-chunk (workspace, per CTA).  Then,
 //      per sub-chunk in reverse, per token in reverse, re-run the sub-chunk from its
 //      start state up to the token (at most 7 steps) and take the reverse step.
-// Reductions over v (for dq^, dk^, dalpha) run as a reduce-scatter over the 8
-// columns of a warp followed by a sum over the 16 warps in shared memory.  The
-// norms, gate and sigmoid gradients of a sub-chunk are taken once its 8 tokens are
-// done.  Everything is fp32 on the CUDA cores: each step is a matrix-vector
-// product on the state, with no contraction large enough for the tensor cores.
+// Reductions over v (for dq^, dk^, dalpha) sum the thread's two columns, reduce-
+// scatter over the warp's four column groups and then sum over the 16 warps in
+// shared memory.  The norms, gate and sigmoid gradients of a sub-chunk are taken
+// once its 8 tokens are done.  Everything is fp32 on the CUDA cores: each step is a
+// matrix-vector product on the state, with no contraction large enough for the
+// tensor cores.
 #include <cstddef>
 
 #include "kda.h"
@@ -39,25 +43,24 @@ namespace {
 
 constexpr int BT = 512;          // threads per CTA
 constexpr int NW = BT / 32;      // 16 warps
-constexpr int RQ = 32;           // state rows per thread
+constexpr int RR = 16;           // state rows per thread (per column)
+constexpr int NS = 2 * RR;       // state entries per thread
 constexpr int SUB = 8;           // tokens per sub-chunk
 constexpr int CH = 64;           // tokens per checkpoint chunk
 constexpr int NSUB = CH / SUB;   // sub-chunks per chunk
-constexpr int QP = 36;           // padded floats per row quarter (bank-conflict-free float4 reads)
-constexpr int ROWP = 4 * QP;     // floats per token in the padded per-channel layout
 constexpr int STATE = kHead * kHead;
 constexpr unsigned FULL = 0xffffffffu;
 
 struct Smem {
-    float4 ssub[RQ / 4][BT];     // start state of the current sub-chunk, thread-private
-    alignas(16) float kh[SUB][ROWP];
-    alignas(16) float qh[SUB][ROWP];
-    alignas(16) float al[SUB][ROWP];
-    alignas(16) float xs[SUB][ROWP];
-    alignas(16) float zs[SUB][ROWP];
+    float4 ssub[NS / 4][BT];     // start state of the current sub-chunk, thread-private
+    alignas(16) float kh[SUB][kHead];
+    alignas(16) float qh[SUB][kHead];
+    alignas(16) float al[SUB][kHead];
+    alignas(16) float xs[SUB][kHead];
+    alignas(16) float zs[SUB][kHead];
     alignas(16) float vv[SUB][kHead];
     alignas(16) float dO[SUB][kHead];
-    alignas(16) float red[2][NW][3][kHead + 32];  // per-warp row sums of one token (double-buffered)
+    alignas(16) float red[2][NW][3][kHead];  // per-warp row sums of one token (double-buffered)
     alignas(16) float res[SUB][3][kHead];    // dq^ / scale, dk^, dalpha per token of the sub-chunk
     float b[SUB], rq[SUB], rk[SUB];
     float redb[2][NW];
@@ -66,8 +69,16 @@ struct Smem {
     float pacc[SUB][kHead + 1];  // per-epilogue-warp partial ddt_bias and dA_log
 };
 
-// Padded index of channel c: quarter c / 32 at a 36-float stride.
-__device__ __forceinline__ int pidx(int c) { return (c >> 5) * QP + (c & 31); }
+// Thread layout: lane = 8 cgl + r8; column group cg = 4 warp + cgl (columns 2 cg,
+// 2 cg + 1); register entry i = 4 g + j holds row 32 g + 4 r8 + j.
+struct Lane {
+    int r8, cgl, v0;
+};
+
+__device__ __forceinline__ int row_of(const Lane &L, int i) { return 32 * (i >> 2) + 4 * L.r8 + (i & 3); }
+
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float f4(const float4 &a, int j) { return j == 0 ? a.x : j == 1 ? a.y : j == 2 ? a.z : a.w; }
 
 __device__ __forceinline__ float bf2f(const __nv_bfloat16 *p, size_t i) { return __bfloat162float(p[i]); }
 
@@ -88,9 +99,37 @@ __device__ __forceinline__ float warp_sum(float x)
     return x;
 }
 
-// Stage tokens [tok, tok + L) of head h (L <= SUB): activations in the padded
-// per-channel layout, v (and dO when want_dO) per column.  Warps 0..7 take one
-// token's channels each, warps 8..15 its v / dO.
+// Sum over the eight row groups of a column (lane bits 0..2).
+__device__ __forceinline__ float rows_sum(float x)
+{
+    x += __shfl_xor_sync(FULL, x, 1);
+    x += __shfl_xor_sync(FULL, x, 2);
+    x += __shfl_xor_sync(FULL, x, 4);
+    return x;
+}
+
+// Reduce-scatter over the warp's four column groups (lane bits 3, 4) of a 16-row
+// partial delivered in pairs: lo = entry i, hi = entry i + 8 (i < 8).  The first
+// round (partner lane ^ 16) halves the rows; `half` collects them.
+__device__ __forceinline__ float scatter_a(float lo, float hi, int cgl)
+{
+    const bool up = cgl & 2;
+    return (up ? hi : lo) + __shfl_xor_sync(FULL, up ? lo : hi, 16);
+}
+
+// Second round (partner lane ^ 8): entries 4 cgl .. 4 cgl + 3 of the column sums.
+__device__ __forceinline__ float4 scatter_b(const float (&h)[8], int cgl)
+{
+    const bool up = cgl & 1;
+    float o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) o[i] = (up ? h[i + 4] : h[i]) + __shfl_xor_sync(FULL, up ? h[i] : h[i + 4], 8);
+    return make_float4(o[0], o[1], o[2], o[3]);
+}
+
+// Stage tokens [tok, tok + L) of head h (L <= SUB): activations per channel, v (and
+// dO when want_dO) per column.  Warps 0..7 take one token's channels each, warps
+// 8..15 its v / dO.
 __device__ void stage(Smem &sm, const BwdParams &p, int64_t tok, int L, int64_t h, float ea,
                       bool want_dO)
 {
@@ -105,27 +144,23 @@ __device__ void stage(Smem &sm, const BwdParams &p, int64_t tok, int L, int64_t 
         const float sq = warp_sum(q4.x * q4.x + q4.y * q4.y + q4.z * q4.z + q4.w * q4.w);
         const float sk = warp_sum(k4.x * k4.x + k4.y * k4.y + k4.z * k4.z + k4.w * k4.w);
         const float rq = rsqrtf(sq + 1e-6f), rk = rsqrtf(sk + 1e-6f);
-        const float qa[4] = {q4.x, q4.y, q4.z, q4.w}, ka[4] = {k4.x, k4.y, k4.z, k4.w};
-        const float ga[4] = {g4.x, g4.y, g4.z, g4.w};
-        float4 qo, ko, ao, xo, zo;
-        float *qp = &qo.x, *kp = &ko.x, *ap = &ao.x, *xp = &xo.x, *zp = &zo.x;
+        float qo[4], ko[4], ao[4], xo[4], zo[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const float x = ga[j] + sm.dtb[c0 + j];
+            const float x = f4(g4, j) + sm.dtb[c0 + j];
             const float sp = fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));  // softplus
             const float z = -ea * sp;
-            qp[j] = qa[j] * rq;
-            kp[j] = ka[j] * rk;
-            xp[j] = x;
-            zp[j] = z;
-            ap[j] = expf(fmaxf(p.lower_bound, z));
+            qo[j] = f4(q4, j) * rq;
+            ko[j] = f4(k4, j) * rk;
+            xo[j] = x;
+            zo[j] = z;
+            ao[j] = expf(fmaxf(p.lower_bound, z));
         }
-        const int pi = pidx(c0);
-        *reinterpret_cast<float4 *>(&sm.qh[tt][pi]) = qo;
-        *reinterpret_cast<float4 *>(&sm.kh[tt][pi]) = ko;
-        *reinterpret_cast<float4 *>(&sm.al[tt][pi]) = ao;
-        *reinterpret_cast<float4 *>(&sm.xs[tt][pi]) = xo;
-        *reinterpret_cast<float4 *>(&sm.zs[tt][pi]) = zo;
+        *reinterpret_cast<float4 *>(&sm.qh[tt][c0]) = make_float4(qo[0], qo[1], qo[2], qo[3]);
+        *reinterpret_cast<float4 *>(&sm.kh[tt][c0]) = make_float4(ko[0], ko[1], ko[2], ko[3]);
+        *reinterpret_cast<float4 *>(&sm.al[tt][c0]) = make_float4(ao[0], ao[1], ao[2], ao[3]);
+        *reinterpret_cast<float4 *>(&sm.xs[tt][c0]) = make_float4(xo[0], xo[1], xo[2], xo[3]);
+        *reinterpret_cast<float4 *>(&sm.zs[tt][c0]) = make_float4(zo[0], zo[1], zo[2], zo[3]);
         if (lane == 0) {
             sm.rq[tt] = rq;
             sm.rk[tt] = rk;
@@ -137,68 +172,49 @@ __device__ void stage(Smem &sm, const BwdParams &p, int64_t tok, int L, int64_t 
     }
 }
 
-// One token of the recurrence on this thread's 32 rows of column v.
-__device__ __forceinline__ void fwd_step(float (&s)[RQ], const Smem &sm, int tt, int qr, int v)
+// One token of the recurrence on this thread's 16 rows of its two columns.
+// s[i] is column 2 cg, s[RR + i] column 2 cg + 1.
+__device__ __forceinline__ void fwd_step(float (&s)[NS], const Smem &sm, int tt, const Lane &L)
 {
-    const float *kr = &sm.kh[tt][qr * QP], *ar = &sm.al[tt][qr * QP];
-    float pa = 0.f;
+    float pa0 = 0.f, pa1 = 0.f;
 #pragma unroll
-    for (int i = 0; i < RQ; i += 4) {
-        const float4 k4 = *reinterpret_cast<const float4 *>(kr + i);
-        const float4 a4 = *reinterpret_cast<const float4 *>(ar + i);
-        s[i] *= a4.x;
-        s[i + 1] *= a4.y;
-        s[i + 2] *= a4.z;
-        s[i + 3] *= a4.w;
-        pa = fmaf(s[i], k4.x, pa);
-        pa = fmaf(s[i + 1], k4.y, pa);
-        pa = fmaf(s[i + 2], k4.z, pa);
-        pa = fmaf(s[i + 3], k4.w, pa);
+    for (int g = 0; g < 4; ++g) {
+        const float4 k4 = ld4(&sm.kh[tt][32 * g + 4 * L.r8]), a4 = ld4(&sm.al[tt][32 * g + 4 * L.r8]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = 4 * g + j;
+            s[i] *= f4(a4, j);
+            s[RR + i] *= f4(a4, j);
+            pa0 = fmaf(s[i], f4(k4, j), pa0);
+            pa1 = fmaf(s[RR + i], f4(k4, j), pa1);
+        }
     }
-    pa += __shfl_xor_sync(FULL, pa, 1);
-    pa += __shfl_xor_sync(FULL, pa, 2);
-    const float br = sm.b[tt] * (sm.vv[tt][v] - pa);
+    pa0 = rows_sum(pa0);
+    pa1 = rows_sum(pa1);
+    const float2 v2 = *reinterpret_cast<const float2 *>(&sm.vv[tt][L.v0]);
+    const float bt = sm.b[tt];
+    const float br0 = bt * (v2.x - pa0), br1 = bt * (v2.y - pa1);
 #pragma unroll
-    for (int i = 0; i < RQ; i += 4) {
-        const float4 k4 = *reinterpret_cast<const float4 *>(kr + i);
-        s[i] = fmaf(k4.x, br, s[i]);
-        s[i + 1] = fmaf(k4.y, br, s[i + 1]);
-        s[i + 2] = fmaf(k4.z, br, s[i + 2]);
-        s[i + 3] = fmaf(k4.w, br, s[i + 3]);
+    for (int g = 0; g < 4; ++g) {
+        const float4 k4 = ld4(&sm.kh[tt][32 * g + 4 * L.r8]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int i = 4 * g + j;
+            s[i] = fmaf(f4(k4, j), br0, s[i]);
+            s[RR + i] = fmaf(f4(k4, j), br1, s[RR + i]);
+        }
     }
 }
-
-// Reduce-scatter of 8 rows over the 8 columns of a warp (lane bits 2..4, m = lane >> 2):
-// on entry x[i] is this lane's value for row i of a block of 8; returns the warp's sum
-// for row m of the block.
-__device__ __forceinline__ float reduce8(const float (&x)[8], int m)
-{
-    float y[4], z[2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const bool up = m & 4;
-        y[i] = (up ? x[i + 4] : x[i]) + __shfl_xor_sync(FULL, up ? x[i] : x[i + 4], 16);
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const bool up = m & 2;
-        z[i] = (up ? y[i + 2] : y[i]) + __shfl_xor_sync(FULL, up ? y[i] : y[i + 2], 8);
-    }
-    const bool up = m & 1;
-    return (up ? z[1] : z[0]) + __shfl_xor_sync(FULL, up ? z[0] : z[1], 4);
-}
-
-// Position of channel c in the per-warp row sums: 8 floats of padding per quarter, so
-// that the 32 lanes' stores of one block (c = 32 qr + 8 bk + m) hit 32 distinct banks.
-__device__ __forceinline__ int ridx(int c) { return c + 8 * (c >> 5); }
 
 __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
 {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int m = lane >> 2, qr = lane & 3;
-    const int v = 8 * warp + m;
+    Lane L;
+    L.r8 = lane & 7;
+    L.cgl = lane >> 3;
+    L.v0 = 2 * (4 * warp + L.cgl);
     const int64_t units = p.N * p.H;
 
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
@@ -211,141 +227,211 @@ __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
         const size_t ck_stride = (size_t)p.H * STATE;
         float4 *scr = reinterpret_cast<float4 *>(p.scratch + (size_t)blockIdx.x * NSUB * STATE);
         const size_t st_off = (size_t)u * STATE;
+        // entry i of this thread's two columns in a [K][V] state: + row * 128 + v0 (+1)
+        auto at = [&](int i) { return (size_t)row_of(L, i) * kHead + L.v0; };
         __syncthreads();  // the previous unit's last readers of dtb / pacc are done
         if (tid < kHead) sm.dtb[tid] = p.dt_bias[h * kHead + tid];
 
         // ---- 1. forward sweep: checkpoints before every chunk ----
-        float s[RQ];
+        float s[NS];
 #pragma unroll
-        for (int i = 0; i < RQ; ++i) {
-            const size_t e = st_off + (size_t)(32 * qr + i) * kHead + v;
-            s[i] = !p.init ? 0.f
-                 : p.init_dtype == KDA_STATE_BF16 ? bf2f(static_cast<const __nv_bfloat16 *>(p.init), e)
-                                                  : static_cast<const float *>(p.init)[e];
+        for (int i = 0; i < RR; ++i) {
+            float2 x = make_float2(0.f, 0.f);
+            if (p.init && p.init_dtype == KDA_STATE_BF16) {
+                const __nv_bfloat162 b2 =
+                    *reinterpret_cast<const __nv_bfloat162 *>(static_cast<const __nv_bfloat16 *>(p.init) + st_off + at(i));
+                x = __bfloat1622float2(b2);
+            } else if (p.init) {
+                x = *reinterpret_cast<const float2 *>(static_cast<const float *>(p.init) + st_off + at(i));
+            }
+            s[i] = x.x;
+            s[RR + i] = x.y;
         }
         for (int64_t n = 0; n < nch; ++n) {
             float *c = ck + n * ck_stride;
 #pragma unroll
-            for (int i = 0; i < RQ; ++i) c[(32 * qr + i) * kHead + v] = s[i];
+            for (int i = 0; i < RR; ++i) *reinterpret_cast<float2 *>(c + at(i)) = make_float2(s[i], s[RR + i]);
             for (int j = 0; j < NSUB; ++j) {
                 const int64_t t0 = n * CH + j * SUB;
                 if (t0 >= len) break;
-                const int L = (int)(len - t0 < SUB ? len - t0 : SUB);
+                const int Lj = (int)(len - t0 < SUB ? len - t0 : SUB);
                 __syncthreads();
-                stage(sm, p, bos + t0, L, h, ea, false);
+                stage(sm, p, bos + t0, Lj, h, ea, false);
                 __syncthreads();
-                for (int tt = 0; tt < L; ++tt) fwd_step(s, sm, tt, qr, v);
+                for (int tt = 0; tt < Lj; ++tt) fwd_step(s, sm, tt, L);
             }
         }
 
         // ---- 2. reverse sweep ----
-        float ds[RQ];
+        float ds[NS];
 #pragma unroll
-        for (int i = 0; i < RQ; ++i)
-            ds[i] = p.dfinal ? p.dfinal[st_off + (size_t)(32 * qr + i) * kHead + v] : 0.f;
+        for (int i = 0; i < RR; ++i) {
+            float2 x = make_float2(0.f, 0.f);
+            if (p.dfinal) x = *reinterpret_cast<const float2 *>(p.dfinal + st_off + at(i));
+            ds[i] = x.x;
+            ds[RR + i] = x.y;
+        }
         for (int i = tid; i < SUB * (kHead + 1); i += BT) (&sm.pacc[0][0])[i] = 0.f;
 
         for (int64_t n = nch - 1; n >= 0; --n) {
-            const int nsub = (int)((len - n * CH + SUB - 1) / SUB < NSUB ? (len - n * CH + SUB - 1) / SUB : NSUB);
+            const int64_t left = (len - n * CH + SUB - 1) / SUB;
+            const int nsub = (int)(left < NSUB ? left : NSUB);
             // 2a. start states of the chunk's sub-chunks
             {
                 const float *c = ck + n * ck_stride;
 #pragma unroll
-                for (int i = 0; i < RQ; ++i) s[i] = c[(32 * qr + i) * kHead + v];
+                for (int i = 0; i < RR; ++i) {
+                    const float2 x = *reinterpret_cast<const float2 *>(c + at(i));
+                    s[i] = x.x;
+                    s[RR + i] = x.y;
+                }
             }
             for (int j = 0; j < nsub; ++j) {
 #pragma unroll
-                for (int i = 0; i < RQ; i += 4)
-                    scr[((size_t)j * (RQ / 4) + i / 4) * BT + tid] =
+                for (int i = 0; i < NS; i += 4)
+                    scr[((size_t)j * (NS / 4) + i / 4) * BT + tid] =
                         make_float4(s[i], s[i + 1], s[i + 2], s[i + 3]);
                 if (j == nsub - 1) break;
                 __syncthreads();
                 stage(sm, p, bos + n * CH + j * SUB, SUB, h, ea, false);
                 __syncthreads();
-                for (int tt = 0; tt < SUB; ++tt) fwd_step(s, sm, tt, qr, v);
+                for (int tt = 0; tt < SUB; ++tt) fwd_step(s, sm, tt, L);
             }
             // 2b. sub-chunks in reverse
             for (int j = nsub - 1; j >= 0; --j) {
                 const int64_t t0 = n * CH + j * SUB;
-                const int L = (int)(len - t0 < SUB ? len - t0 : SUB);
+                const int Lj = (int)(len - t0 < SUB ? len - t0 : SUB);
                 __syncthreads();
-                stage(sm, p, bos + t0, L, h, ea, true);
+                stage(sm, p, bos + t0, Lj, h, ea, true);
 #pragma unroll
-                for (int i = 0; i < RQ / 4; ++i) sm.ssub[i][tid] = scr[((size_t)j * (RQ / 4) + i) * BT + tid];
+                for (int i = 0; i < NS / 4; ++i) sm.ssub[i][tid] = scr[((size_t)j * (NS / 4) + i) * BT + tid];
                 __syncthreads();
-                for (int tt = L - 1; tt >= 0; --tt) {
+                for (int tt = Lj - 1; tt >= 0; --tt) {
 #pragma unroll
-                    for (int i = 0; i < RQ / 4; ++i) {
+                    for (int i = 0; i < NS / 4; ++i) {
                         const float4 f = sm.ssub[i][tid];
                         s[4 * i] = f.x;
                         s[4 * i + 1] = f.y;
                         s[4 * i + 2] = f.z;
                         s[4 * i + 3] = f.w;
                     }
-                    for (int t2 = 0; t2 < tt; ++t2) fwd_step(s, sm, t2, qr, v);
+                    for (int t2 = 0; t2 < tt; ++t2) fwd_step(s, sm, t2, L);
                     // s = S_{t-1}; ds = dL/dS_t from everything after token t
-                    const float *kr = &sm.kh[tt][qr * QP], *ar = &sm.al[tt][qr * QP];
-                    const float *qp = &sm.qh[tt][qr * QP];
+                    const float *kr = &sm.kh[tt][4 * L.r8], *ar = &sm.al[tt][4 * L.r8];
+                    const float *qp = &sm.qh[tt][4 * L.r8];  // row group g at + 32 g
                     const float bt = sm.b[tt];
-                    float pa = 0.f;
+                    float pa0 = 0.f, pa1 = 0.f;
 #pragma unroll
-                    for (int i = 0; i < RQ; ++i) pa = fmaf(ar[i] * s[i], kr[i], pa);
-                    pa += __shfl_xor_sync(FULL, pa, 1);
-                    pa += __shfl_xor_sync(FULL, pa, 2);
-                    const float r = sm.vv[tt][v] - pa, br = bt * r;
-                    const float dOv = sm.dO[tt][v], dOs = p.scale * dOv;
-                    const int buf = tt & 1;
-                    float e = 0.f;
-                    // dS_t += scale q^ dO^T; dq^ partial S_t dO; e partial dS^T k^
+                    for (int g = 0; g < 4; ++g) {
+                        const float4 k4 = ld4(kr + 32 * g), a4 = ld4(ar + 32 * g);
 #pragma unroll
-                    for (int bk = 0; bk < 4; ++bk) {
-                        float x[8];
-#pragma unroll
-                        for (int i2 = 0; i2 < 8; ++i2) {
-                            const int i = 8 * bk + i2;
-                            const float st = fmaf(kr[i], br, ar[i] * s[i]);
-                            ds[i] = fmaf(qp[i], dOs, ds[i]);
-                            e = fmaf(ds[i], kr[i], e);
-                            x[i2] = st * dOv;
+                        for (int j2 = 0; j2 < 4; ++j2) {
+                            const int i = 4 * g + j2;
+                            pa0 = fmaf(f4(a4, j2) * s[i], f4(k4, j2), pa0);
+                            pa1 = fmaf(f4(a4, j2) * s[RR + i], f4(k4, j2), pa1);
                         }
-                        sm.red[buf][warp][0][ridx(32 * qr + 8 * bk + m)] = reduce8(x, m);
                     }
-                    e += __shfl_xor_sync(FULL, e, 1);
-                    e += __shfl_xor_sync(FULL, e, 2);
-                    const float dr = bt * e;
-                    const float dbw = warp_sum(qr == 0 ? r * e : 0.f);
-                    if (lane == 0) sm.redb[buf][warp] = dbw;
-                    if (qr == 0) p.dv[(bos + t0 + tt) * p.H * kHead + h * kHead + v] = dr;
-                    // dk^ partial: b dS r - S' dr (dS = dL/dS_t)
+                    pa0 = rows_sum(pa0);
+                    pa1 = rows_sum(pa1);
+                    const float2 v2 = *reinterpret_cast<const float2 *>(&sm.vv[tt][L.v0]);
+                    const float2 o2 = *reinterpret_cast<const float2 *>(&sm.dO[tt][L.v0]);
+                    const float r0 = v2.x - pa0, r1 = v2.y - pa1;
+                    const float br0 = bt * r0, br1 = bt * r1;
+                    const float dOs0 = p.scale * o2.x, dOs1 = p.scale * o2.y;
+                    const int buf = tt & 1;
+                    float e0 = 0.f, e1 = 0.f;
+                    // dS_t += scale q^ dO^T; dq^ partial S_t dO; e partial dS^T k^
+                    {
+                        float hf[8];
 #pragma unroll
-                    for (int bk = 0; bk < 4; ++bk) {
-                        float x[8];
+                        for (int g = 0; g < 2; ++g) {
+                            const float4 kl = ld4(kr + 32 * g), kh4 = ld4(kr + 32 * (g + 2));
+                            const float4 al4 = ld4(ar + 32 * g), ah4 = ld4(ar + 32 * (g + 2));
+                            const float4 ql = ld4(qp + 32 * g), qh4 = ld4(qp + 32 * (g + 2));
 #pragma unroll
-                        for (int i2 = 0; i2 < 8; ++i2) {
-                            const int i = 8 * bk + i2;
-                            x[i2] = fmaf(ds[i], br, -(ar[i] * s[i]) * dr);
+                            for (int j2 = 0; j2 < 4; ++j2) {
+                                float x[2];
+#pragma unroll
+                                for (int hh = 0; hh < 2; ++hh) {
+                                    const int i = 4 * g + j2 + 8 * hh;
+                                    const float kk = f4(hh ? kh4 : kl, j2), aa = f4(hh ? ah4 : al4, j2);
+                                    const float qq = f4(hh ? qh4 : ql, j2);
+                                    const float st0 = fmaf(kk, br0, aa * s[i]);
+                                    const float st1 = fmaf(kk, br1, aa * s[RR + i]);
+                                    ds[i] = fmaf(qq, dOs0, ds[i]);
+                                    ds[RR + i] = fmaf(qq, dOs1, ds[RR + i]);
+                                    e0 = fmaf(ds[i], kk, e0);
+                                    e1 = fmaf(ds[RR + i], kk, e1);
+                                    x[hh] = fmaf(st0, o2.x, st1 * o2.y);
+                                }
+                                hf[4 * g + j2] = scatter_a(x[0], x[1], L.cgl);
+                            }
                         }
-                        sm.red[buf][warp][1][ridx(32 * qr + 8 * bk + m)] = reduce8(x, m);
+                        *reinterpret_cast<float4 *>(&sm.red[buf][warp][0][32 * L.cgl + 4 * L.r8]) =
+                            scatter_b(hf, L.cgl);
+                    }
+                    e0 = rows_sum(e0);
+                    e1 = rows_sum(e1);
+                    const float dr0 = bt * e0, dr1 = bt * e1;
+                    const float dbw = warp_sum(L.r8 == 0 ? fmaf(r0, e0, r1 * e1) : 0.f);
+                    if (lane == 0) sm.redb[buf][warp] = dbw;
+                    if (L.r8 == 0)
+                        *reinterpret_cast<float2 *>(p.dv + (bos + t0 + tt) * p.H * kHead + h * kHead + L.v0) =
+                            make_float2(dr0, dr1);
+                    // dk^ partial: b dS r - S' dr (dS = dL/dS_t)
+                    {
+                        float hf[8];
+#pragma unroll
+                        for (int g = 0; g < 2; ++g) {
+                            const float4 al4 = ld4(ar + 32 * g), ah4 = ld4(ar + 32 * (g + 2));
+#pragma unroll
+                            for (int j2 = 0; j2 < 4; ++j2) {
+                                float x[2];
+#pragma unroll
+                                for (int hh = 0; hh < 2; ++hh) {
+                                    const int i = 4 * g + j2 + 8 * hh;
+                                    const float aa = f4(hh ? ah4 : al4, j2);
+                                    x[hh] = fmaf(ds[i], br0, -(aa * s[i]) * dr0) +
+                                            fmaf(ds[RR + i], br1, -(aa * s[RR + i]) * dr1);
+                                }
+                                hf[4 * g + j2] = scatter_a(x[0], x[1], L.cgl);
+                            }
+                        }
+                        *reinterpret_cast<float4 *>(&sm.red[buf][warp][1][32 * L.cgl + 4 * L.r8]) =
+                            scatter_b(hf, L.cgl);
                     }
                     // dS' = dS - k^ dr^T; dalpha partial rowsum(dS' o S_{t-1}); dS_{t-1} = alpha dS'
+                    {
+                        float hf[8];
 #pragma unroll
-                    for (int bk = 0; bk < 4; ++bk) {
-                        float x[8];
+                        for (int g = 0; g < 2; ++g) {
+                            const float4 kl = ld4(kr + 32 * g), kh4 = ld4(kr + 32 * (g + 2));
+                            const float4 al4 = ld4(ar + 32 * g), ah4 = ld4(ar + 32 * (g + 2));
 #pragma unroll
-                        for (int i2 = 0; i2 < 8; ++i2) {
-                            const int i = 8 * bk + i2;
-                            ds[i] = fmaf(-kr[i], dr, ds[i]);
-                            x[i2] = ds[i] * s[i];
-                            ds[i] *= ar[i];
+                            for (int j2 = 0; j2 < 4; ++j2) {
+                                float x[2];
+#pragma unroll
+                                for (int hh = 0; hh < 2; ++hh) {
+                                    const int i = 4 * g + j2 + 8 * hh;
+                                    const float kk = f4(hh ? kh4 : kl, j2), aa = f4(hh ? ah4 : al4, j2);
+                                    ds[i] = fmaf(-kk, dr0, ds[i]);
+                                    ds[RR + i] = fmaf(-kk, dr1, ds[RR + i]);
+                                    x[hh] = fmaf(ds[i], s[i], ds[RR + i] * s[RR + i]);
+                                    ds[i] *= aa;
+                                    ds[RR + i] *= aa;
+                                }
+                                hf[4 * g + j2] = scatter_a(x[0], x[1], L.cgl);
+                            }
                         }
-                        sm.red[buf][warp][2][ridx(32 * qr + 8 * bk + m)] = reduce8(x, m);
+                        *reinterpret_cast<float4 *>(&sm.red[buf][warp][2][32 * L.cgl + 4 * L.r8]) =
+                            scatter_b(hf, L.cgl);
                     }
                     __syncthreads();
                     if (tid < 3 * kHead) {
                         const int arr = tid >> 7, c = tid & (kHead - 1);
                         float acc = 0.f;
 #pragma unroll
-                        for (int w = 0; w < NW; ++w) acc += sm.red[buf][w][arr][ridx(c)];
+                        for (int w = 0; w < NW; ++w) acc += sm.red[buf][w][arr][c];
                         sm.res[tt][arr][c] = acc;
                     } else if (tid == 3 * kHead) {
                         float acc = 0.f;
@@ -356,52 +442,43 @@ __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
                 }
                 __syncthreads();
                 // 2c. gradients through the activations of the sub-chunk's tokens
-                if (warp < L) {
-                    const int tt = warp, c0 = 4 * lane, pi = pidx(c0);
+                if (warp < Lj) {
+                    const int tt = warp, c0 = 4 * lane;
                     const int64_t row = (bos + t0 + tt) * p.H + h;
-                    const float4 q4 = *reinterpret_cast<const float4 *>(&sm.qh[tt][pi]);
-                    const float4 k4 = *reinterpret_cast<const float4 *>(&sm.kh[tt][pi]);
-                    const float4 a4 = *reinterpret_cast<const float4 *>(&sm.al[tt][pi]);
-                    const float4 x4 = *reinterpret_cast<const float4 *>(&sm.xs[tt][pi]);
-                    const float4 z4 = *reinterpret_cast<const float4 *>(&sm.zs[tt][pi]);
-                    const float4 dqh4 = *reinterpret_cast<const float4 *>(&sm.res[tt][0][c0]);
-                    const float4 dkh4 = *reinterpret_cast<const float4 *>(&sm.res[tt][1][c0]);
-                    const float4 da4 = *reinterpret_cast<const float4 *>(&sm.res[tt][2][c0]);
-                    const float qa[4] = {q4.x, q4.y, q4.z, q4.w}, ka[4] = {k4.x, k4.y, k4.z, k4.w};
-                    const float aa[4] = {a4.x, a4.y, a4.z, a4.w}, xa[4] = {x4.x, x4.y, x4.z, x4.w};
-                    const float za[4] = {z4.x, z4.y, z4.z, z4.w};
-                    float dqh[4] = {dqh4.x, dqh4.y, dqh4.z, dqh4.w}, dkh[4] = {dkh4.x, dkh4.y, dkh4.z, dkh4.w};
-                    const float dal[4] = {da4.x, da4.y, da4.z, da4.w};
+                    const float4 q4 = ld4(&sm.qh[tt][c0]), k4 = ld4(&sm.kh[tt][c0]);
+                    const float4 a4 = ld4(&sm.al[tt][c0]), x4 = ld4(&sm.xs[tt][c0]);
+                    const float4 z4 = ld4(&sm.zs[tt][c0]);
+                    const float4 dqh4 = ld4(&sm.res[tt][0][c0]), dkh4 = ld4(&sm.res[tt][1][c0]);
+                    const float4 da4 = ld4(&sm.res[tt][2][c0]);
                     float pq = 0.f, pk = 0.f;
 #pragma unroll
                     for (int j2 = 0; j2 < 4; ++j2) {
-                        dqh[j2] *= p.scale;
-                        pq = fmaf(qa[j2], dqh[j2], pq);
-                        pk = fmaf(ka[j2], dkh[j2], pk);
+                        pq = fmaf(f4(q4, j2), p.scale * f4(dqh4, j2), pq);
+                        pk = fmaf(f4(k4, j2), f4(dkh4, j2), pk);
                     }
                     pq = warp_sum(pq);
                     pk = warp_sum(pk);
                     const float rq = sm.rq[tt], rk = sm.rk[tt];
-                    float4 dq4, dk4, dg4;
-                    float *dqo = &dq4.x, *dko = &dk4.x, *dgo = &dg4.x;
+                    float dqo[4], dko[4], dgo[4];
                     float dA = 0.f;
 #pragma unroll
                     for (int j2 = 0; j2 < 4; ++j2) {
-                        dqo[j2] = rq * (dqh[j2] - qa[j2] * pq);
-                        dko[j2] = rk * (dkh[j2] - ka[j2] * pk);
-                        const float dlam = dal[j2] * aa[j2];
-                        const bool open = za[j2] >= p.lower_bound;  // clamp not holding
-                        const float sig = 1.f / (1.f + expf(-xa[j2]));
+                        dqo[j2] = rq * (p.scale * f4(dqh4, j2) - f4(q4, j2) * pq);
+                        dko[j2] = rk * (f4(dkh4, j2) - f4(k4, j2) * pk);
+                        const float dlam = f4(da4, j2) * f4(a4, j2);
+                        const float z = f4(z4, j2);
+                        const bool open = z >= p.lower_bound;  // clamp not holding
+                        const float sig = 1.f / (1.f + expf(-f4(x4, j2)));
                         const float dx = open ? -dlam * ea * sig : 0.f;
                         dgo[j2] = dx;
                         sm.pacc[tt][c0 + j2] += dx;  // row tt belongs to this warp alone
-                        dA += open ? dlam * za[j2] : 0.f;
+                        dA += open ? dlam * z : 0.f;
                     }
                     dA = warp_sum(dA);
                     if (lane == 0) sm.pacc[tt][kHead] += dA;
-                    *reinterpret_cast<float4 *>(p.dq + row * kHead + c0) = dq4;
-                    *reinterpret_cast<float4 *>(p.dk + row * kHead + c0) = dk4;
-                    *reinterpret_cast<float4 *>(p.dg + row * kHead + c0) = dg4;
+                    *reinterpret_cast<float4 *>(p.dq + row * kHead + c0) = make_float4(dqo[0], dqo[1], dqo[2], dqo[3]);
+                    *reinterpret_cast<float4 *>(p.dk + row * kHead + c0) = make_float4(dko[0], dko[1], dko[2], dko[3]);
+                    *reinterpret_cast<float4 *>(p.dg + row * kHead + c0) = make_float4(dgo[0], dgo[1], dgo[2], dgo[3]);
                     if (lane == 0) {
                         const float bt = sm.b[tt];
                         p.dbeta[row] = sm.resb[tt] * bt * (1.f - bt);
@@ -413,7 +490,8 @@ __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
         // ---- 3. dL/dS_0 and the per-unit parameter partials ----
         if (p.dinit) {
 #pragma unroll
-            for (int i = 0; i < RQ; ++i) p.dinit[st_off + (size_t)(32 * qr + i) * kHead + v] = ds[i];
+            for (int i = 0; i < RR; ++i)
+                *reinterpret_cast<float2 *>(p.dinit + st_off + at(i)) = make_float2(ds[i], ds[RR + i]);
         }
         __syncthreads();
         if (tid <= kHead) {
