@@ -345,11 +345,8 @@ def run_backward_bench(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     w = WORKLOAD
-    B, T, H = args.batch or w["B"], args.seqlen or w["T"], w["H"]
+    B, T, H = w["B"], w["T"], w["H"]  # --batch / --seqlen already applied by parse()
     inp = device_inputs(args.seed + 1000 * rank, device)
-    if (B, T) != (w["B"], w["T"]):
-        for key in ("q", "k", "v", "g", "beta"):
-            inp[key] = inp[key][:B, :T].contiguous()
     gen = torch.Generator(device=device)
     gen.manual_seed(args.seed + 7 + 1000 * rank)
     dO = torch.empty((B, T, H, w["V"]), device=device).normal_(0.0, 1.0, generator=gen)

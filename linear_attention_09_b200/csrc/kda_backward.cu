@@ -233,19 +233,27 @@ __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
         if (tid < kHead) sm.dtb[tid] = p.dt_bias[h * kHead + tid];
 
         // ---- 1. forward sweep: checkpoints before every chunk ----
+        // (dtype tests outside the unrolled loops: the 16 loads are in flight together)
         float s[NS];
+        if (p.init && p.init_dtype == KDA_STATE_BF16) {
+            const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(p.init) + st_off;
 #pragma unroll
-        for (int i = 0; i < RR; ++i) {
-            float2 x = make_float2(0.f, 0.f);
-            if (p.init && p.init_dtype == KDA_STATE_BF16) {
-                const __nv_bfloat162 b2 =
-                    *reinterpret_cast<const __nv_bfloat162 *>(static_cast<const __nv_bfloat16 *>(p.init) + st_off + at(i));
-                x = __bfloat1622float2(b2);
-            } else if (p.init) {
-                x = *reinterpret_cast<const float2 *>(static_cast<const float *>(p.init) + st_off + at(i));
+            for (int i = 0; i < RR; ++i) {
+                const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(src + at(i)));
+                s[i] = x.x;
+                s[RR + i] = x.y;
             }
-            s[i] = x.x;
-            s[RR + i] = x.y;
+        } else if (p.init) {
+            const float *src = static_cast<const float *>(p.init) + st_off;
+#pragma unroll
+            for (int i = 0; i < RR; ++i) {
+                const float2 x = *reinterpret_cast<const float2 *>(src + at(i));
+                s[i] = x.x;
+                s[RR + i] = x.y;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < NS; ++i) s[i] = 0.f;
         }
         for (int64_t n = 0; n < nch; ++n) {
             float *c = ck + n * ck_stride;
@@ -264,12 +272,16 @@ __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
 
         // ---- 2. reverse sweep ----
         float ds[NS];
+        if (p.dfinal) {
 #pragma unroll
-        for (int i = 0; i < RR; ++i) {
-            float2 x = make_float2(0.f, 0.f);
-            if (p.dfinal) x = *reinterpret_cast<const float2 *>(p.dfinal + st_off + at(i));
-            ds[i] = x.x;
-            ds[RR + i] = x.y;
+            for (int i = 0; i < RR; ++i) {
+                const float2 x = *reinterpret_cast<const float2 *>(p.dfinal + st_off + at(i));
+                ds[i] = x.x;
+                ds[RR + i] = x.y;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < NS; ++i) ds[i] = 0.f;
         }
         for (int i = tid; i < SUB * (kHead + 1); i += BT) (&sm.pacc[0][0])[i] = 0.f;
 

@@ -778,20 +778,29 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
         return state_off + (vk ? (size_t)v * kHead + kk : (size_t)kk * kHead + v);
     };
 
-    // initial state (column v) -> TM_S with tau = 1
+    // initial state (column v) -> TM_S with tau = 1.  The dtype test sits outside the
+    // load loops, so that each group's 32 independent loads are in flight together
+    // (four memory round trips per thread instead of one per element).
     float tau = 1.f;
-    for (int k0 = 0; k0 < kHead; k0 += 16) {
-        uint32_t r[16];
+    {
+        const float *i32 = p.init && p.init_dtype == KDA_STATE_F32 ? reinterpret_cast<const float *>(p.init) : nullptr;
+        const __nv_bfloat16 *i16 =
+            p.init && p.init_dtype == KDA_STATE_BF16 ? reinterpret_cast<const __nv_bfloat16 *>(p.init) : nullptr;
+        for (int k0 = 0; k0 < kHead; k0 += 32) {
+            uint32_t r[2][16];
+            if (i32) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            float x = 0.f;
-            if (p.init && p.init_dtype == KDA_STATE_F32)
-                x = reinterpret_cast<const float *>(p.init)[st_idx(k0 + j)];
-            else if (p.init)
-                x = bf2f(reinterpret_cast<const __nv_bfloat16 *>(p.init)[st_idx(k0 + j)]);
-            r[j] = __float_as_uint(x);
+                for (int j = 0; j < 32; ++j) r[j >> 4][j & 15] = __float_as_uint(__ldg(i32 + st_idx(k0 + j)));
+            } else if (i16) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) r[j >> 4][j & 15] = __float_as_uint(bf2f(i16[st_idx(k0 + j)]));
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) r[j >> 4][j & 15] = 0u;
+            }
+            tmem_st16(tb + lq + TM_S + k0, r[0]);
+            tmem_st16(tb + lq + TM_S + k0 + 16, r[1]);
         }
-        tmem_st16(tb + lq + TM_S + k0, r);
     }
     tmem_wait_st();
 
