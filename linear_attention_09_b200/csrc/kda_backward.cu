@@ -551,14 +551,9 @@ int launch_backward(const BwdParams &p, const BwdLayout &l, cudaStream_t stream)
 {
     const int64_t units = p.N * p.H;
     if (units <= 0) return 0;
-    static int smem_set = 0;
+    static int smem_set[64];
     const int smem = (int)sizeof(Smem);
-    if (!smem_set) {
-        if (cudaFuncSetAttribute(bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-            cudaSuccess)
-            return KDA_ERR_CUDA;
-        smem_set = 1;
-    }
+    if (!set_smem_limit_once(bwd_kernel, smem, smem_set)) return KDA_ERR_CUDA;
     bwd_kernel<<<l.grid, BT, smem, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
     param_reduce_kernel<<<(unsigned)p.H, kHead + 1, 0, stream>>>(p.part, p.N, p.H, p.dA_log,

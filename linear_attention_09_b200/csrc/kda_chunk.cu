@@ -1088,13 +1088,8 @@ int launch_chunked(const FwdParams &p, cudaStream_t stream)
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return KDA_ERR_CUDA;
     }
-    static bool attr_set = false;
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SMEM_ALLOC) != cudaSuccess)
-            return KDA_ERR_CUDA;
-        attr_set = true;
-    }
+    static int attr_set[64];
+    if (!set_smem_limit_once(chunk_kernel, SMEM_ALLOC, attr_set)) return KDA_ERR_CUDA;
     chunk_kernel<<<(unsigned)ctas, NT, SMEM_ALLOC, stream>>>(p, tm);
     return cudaGetLastError() == cudaSuccess ? 1 : KDA_ERR_CUDA;
 }

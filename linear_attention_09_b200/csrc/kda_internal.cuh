@@ -63,6 +63,21 @@ struct BwdLayout {
 size_t bwd_layout(int64_t total_tokens, int64_t N, int64_t H, BwdLayout *out);
 int launch_backward(const BwdParams &p, const BwdLayout &l, cudaStream_t stream);
 
+// Raises `kernel`'s dynamic shared-memory limit to `bytes` once per device (the
+// attribute belongs to the device's context); `done` is the caller's per-device flags.
+template <typename Kernel>
+inline bool set_smem_limit_once(Kernel kernel, int bytes, int (&done)[64])
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const bool cached = dev >= 0 && dev < 64;
+    if (cached && done[dev]) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+        return false;
+    if (cached) done[dev] = 1;
+    return true;
+}
+
 // Kernel launcher; returns the number of kernels it enqueued (>= 0) or a negative
 // KDA_ERR_* code.
 int launch_chunked(const FwdParams &p, cudaStream_t stream);
