@@ -1,0 +1,153 @@
+"""Chunked form of the KDA backward pass in NumPy fp64 -- test-side only.
+
+This is NOT the oracle (the oracle differentiates the token recurrence directly).  It
+restates the backward in the per-chunk matrix form a tensor-core kernel would run, so
+that the algebra can be checked against the oracle's gradients before any kernel of
+that shape exists.
+
+Forward of one chunk of L tokens from state S0 (K x V), on activations q^, k^, b,
+lam, with G the inclusive cumulative sum of lam and Gam = exp(G), GL = G[L-1]
+(the chunked form of the recurrence of the FlashKDA pages, 7minutos.es "¿Qué es la
+atención Kimi Delta...?"):
+  A_ij = sum_c k^_i k^_j exp(G_i - G_j)   (j < i),   P_ij = same with q^_i (j <= i)
+  M = I + Diag(b) A,  T = M^-1 Diag(b)
+  Y = v - (k^ Gam) S0,  U = T Y
+  O = scale [(q^ Gam) S0 + P U]
+  S_end = Diag(exp GL) S0 + (k^ exp(GL - G))^T U
+Reverse of the chunk, given dO and dS_end (written as dS):
+  dU = scale P^T dO + K' dS          (K' = k^ exp(GL - G))
+  dY = T^T dU;  dv = dY;  dT = dU Y^T
+  dS0 = scale (q^ Gam)^T dO + Diag(exp GL) dS - (k^ Gam)^T dY
+  d(k^ Gam) = -dY S0^T;  d(q^ Gam) = scale dO S0^T;  dP = scale dO U^T (j <= i)
+  dK' = U dS^T;  d(exp GL) = rowsum(dS o S0)
+  dMinv = dT Diag(b);  db_j += sum_i dT_ij Minv_ij
+  dM = -Minv^T dMinv Minv^T;  dA = Diag(b) dM (j < i);  db_i += sum_j dM_ij A_ij
+then through the decay-weighted products into dq^, dk^ and dG, and dlam is the
+reverse cumulative sum of dG.  The chunks are visited in reverse, dS passing from
+each chunk's dS0 to the chunk before it.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def _gram(x, k, G, strict):
+    """M_ij = sum_c x_i k_j exp(G_i - G_j) on the lower triangle; also E_ijc."""
+    E = np.exp(G[:, None, :] - G[None, :, :])  # [L, L, K]; only the lower part is used
+    L = G.shape[0]
+    mask = np.tril(np.ones((L, L)), -1 if strict else 0)
+    E = E * mask[:, :, None]
+    return np.einsum("ic,jc,ijc->ij", x, k, E), E
+
+
+def chunk_backward(qh, kh, v, b, lam, scale, dO, S0=None, dSf=None, C=64):
+    """Gradients w.r.t. the activations of ONE (sequence, head).
+
+    Returns (dqh, dkh, dv, db, dlam, dS0) in fp64 for L = <dO, out> + <dSf, S_final>.
+    """
+    T_, K = qh.shape
+    V = v.shape[1]
+    S = np.zeros((K, V)) if S0 is None else np.array(S0, dtype=np.float64)
+    starts = []
+    for c0 in range(0, T_, C):  # forward: the state before every chunk
+        starts.append(S.copy())
+        L = min(C, T_ - c0)
+        sl = slice(c0, c0 + L)
+        G = np.cumsum(lam[sl], axis=0)
+        A, _ = _gram(kh[sl], kh[sl], G, True)
+        Tm = np.linalg.solve(np.eye(L) + b[sl, None] * A, np.diag(b[sl]))
+        U = Tm @ (v[sl] - (kh[sl] * np.exp(G)) @ S)
+        S = np.exp(G[L - 1])[:, None] * S + (kh[sl] * np.exp(G[L - 1][None] - G)).T @ U
+    dqh, dkh = np.zeros_like(qh), np.zeros_like(kh)
+    dv, db, dlam = np.zeros_like(v), np.zeros_like(b), np.zeros_like(lam)
+    dS = np.zeros((K, V)) if dSf is None else np.array(dSf, dtype=np.float64)
+    for n in reversed(range(len(starts))):
+        c0 = n * C
+        L = min(C, T_ - c0)
+        sl = slice(c0, c0 + L)
+        q_, k_, v_, b_, S0n, dO_ = qh[sl], kh[sl], v[sl], b[sl], starts[n], dO[sl]
+        G = np.cumsum(lam[sl], axis=0)
+        Gam, GL = np.exp(G), G[L - 1]
+        A, EA = _gram(k_, k_, G, True)
+        P, EP = _gram(q_, k_, G, False)
+        Minv = np.linalg.inv(np.eye(L) + b_[:, None] * A)
+        Tm = Minv * b_[None, :]
+        KG, QG = k_ * Gam, q_ * Gam
+        Kp = k_ * np.exp(GL[None] - G)
+        Y = v_ - KG @ S0n
+        U = Tm @ Y
+        # reverse of the chunk
+        dU = scale * P.T @ dO_ + Kp @ dS
+        dY = Tm.T @ dU
+        dT = np.tril(dU @ Y.T)
+        dS0 = scale * QG.T @ dO_ + np.exp(GL)[:, None] * dS - KG.T @ dY
+        dKG = -dY @ S0n.T
+        dQG = scale * dO_ @ S0n.T
+        dP = np.tril(scale * dO_ @ U.T)
+        dKp = U @ dS.T
+        dGL = (dS * S0n).sum(1) * np.exp(GL)
+        dv[sl] = dY
+        dMinv = dT * b_[None, :]
+        db_ = (dT * Minv).sum(0)
+        dM = -Minv.T @ dMinv @ Minv.T
+        dA = np.tril(b_[:, None] * dM, -1)
+        db_ += (np.tril(dM, -1) * A).sum(1)
+        # decay-weighted products -> dq^, dk^, dG
+        dG = np.zeros_like(G)
+        tA_i = np.einsum("ij,jc,ijc->ic", dA, k_, EA)   # sum_j dA_ij k_j E_ij
+        tA_j = np.einsum("ij,ic,ijc->jc", dA, k_, EA)   # sum_i dA_ij k_i E_ij
+        tP_i = np.einsum("ij,jc,ijc->ic", dP, k_, EP)
+        tP_j = np.einsum("ij,ic,ijc->jc", dP, q_, EP)
+        dk_ = tA_i + tA_j + tP_j + dKG * Gam + dKp * np.exp(GL[None] - G)
+        dq_ = tP_i + dQG * Gam
+        dG += k_ * tA_i - k_ * tA_j + q_ * tP_i - k_ * tP_j
+        dG += dKG * KG + dQG * QG
+        dG -= dKp * Kp
+        dG[L - 1] += (dKp * Kp).sum(0) + dGL
+        dqh[sl], dkh[sl], db[sl] = dq_, dk_, db_
+        dlam[sl] = np.cumsum(dG[::-1], axis=0)[::-1]  # dlam_s = sum_{i >= s} dG_i
+        dS = dS0
+    return dqh, dkh, dv, db, dlam, dS
+
+
+def backward_inputs(inp, dO, dSf=None, C=64, eps=1e-6):
+    """``chunk_backward`` over a ``kda_inputs.KDAInputs``, chained through the norms,
+    the sigmoid and the gate to the raw inputs; returns the dict of ``oracle.backward``
+    (plus dlam)."""
+    q, k, v, g = (t.double().numpy() for t in (inp.q, inp.k, inp.v, inp.g))
+    beta = inp.beta.double().numpy()
+    A_log, dt = inp.A_log.double().numpy(), inp.dt_bias.double().numpy()
+    init = None if inp.initial_state is None else inp.initial_state.double().numpy()
+    dOn = dO.double().numpy()
+    dSn = None if dSf is None else dSf.double().numpy()
+    B, Tt, H, K = q.shape
+    seqs = inp.seq_bounds()
+    r = dict(dq=np.zeros_like(q), dk=np.zeros_like(k), dv=np.zeros_like(v), dg=np.zeros_like(g),
+             dbeta=np.zeros_like(beta), dA_log=np.zeros(H), ddt_bias=np.zeros((H, K)),
+             dS0=np.zeros((len(seqs), H, K, v.shape[3])), dlam=np.zeros_like(g))
+    for s, (bi, t0, n) in enumerate(seqs):
+        sl = slice(t0, t0 + n)
+        for h in range(H):
+            qq, kk, gg = q[bi, sl, h], k[bi, sl, h], g[bi, sl, h]
+            rq = 1 / np.sqrt((qq * qq).sum(-1, keepdims=True) + eps)
+            rk = 1 / np.sqrt((kk * kk).sum(-1, keepdims=True) + eps)
+            qh, kh = qq * rq, kk * rk
+            bb = 1 / (1 + np.exp(-beta[bi, sl, h]))
+            x = gg + dt[h][None]
+            z = -np.exp(A_log[h]) * (np.maximum(x, 0) + np.log1p(np.exp(-np.abs(x))))
+            lam = np.maximum(inp.lower_bound, z)
+            dqh, dkh, dvv, dbb, dlam, dS0 = chunk_backward(
+                qh, kh, v[bi, sl, h], bb, lam, inp.scale, dOn[bi, sl, h],
+                None if init is None else init[s, h], None if dSn is None else dSn[s, h], C)
+            r["dq"][bi, sl, h] = rq * (dqh - qh * (qh * dqh).sum(-1, keepdims=True))
+            r["dk"][bi, sl, h] = rk * (dkh - kh * (kh * dkh).sum(-1, keepdims=True))
+            r["dv"][bi, sl, h] = dvv
+            r["dbeta"][bi, sl, h] = dbb * bb * (1 - bb)
+            openm = z >= inp.lower_bound
+            dx = np.where(openm, -dlam * np.exp(A_log[h]) / (1 + np.exp(-x)), 0.0)
+            r["dg"][bi, sl, h] = dx
+            r["dlam"][bi, sl, h] = dlam
+            r["ddt_bias"][h] += dx.sum(0)
+            r["dA_log"][h] += np.where(openm, dlam * z, 0.0).sum()
+            r["dS0"][s, h] = dS0
+    return r
