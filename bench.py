@@ -169,14 +169,15 @@ class ClockSampler:
                 "samples": len(busy)}
 
 
-def profile_traffic(kernel_source):
-    """Per-launch DRAM bytes from the committed ncu summary, if the kernel is unchanged."""
-    path = os.path.join(ROOT, "profiles", PROFILE)
+def profile_traffic(kernel_source, profile=PROFILE, key="traffic_bytes_per_launch"):
+    """DRAM bytes (``key``: per launch, or per unit) from a committed ncu summary, if the
+    kernel source is unchanged since the capture."""
+    path = os.path.join(ROOT, "profiles", profile)
     try:
         txt = open(path).read()
     except OSError:
         return None, None
-    m = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    m = re.search(key + r":\s*([0-9.eE+]+)", txt)
     h = re.search(r"source_sha256:\s*([0-9a-f]+)", txt)
     if not m or not h or h.group(1) != source_hash(kernel_source):
         return None, None
@@ -266,6 +267,8 @@ def run_reference(args, world, rank):
 
 
 DECODE_BYTES_PER_TOKEN_HEAD = 2 * 128 * 128 * 4 + 4 * 128 * 2 + 2 + 128 * 2  # state r+w, q k v g, beta, out
+DECODE_SRC = ["linear_attention_09_b200/csrc/kda_decode.cu"]
+DECODE_PROFILE = "decode_kernel_N128_H32.md"  # ncu DRAM bytes per token-head + source hash
 
 
 def run_decode_bench(args, world, rank, local):
@@ -309,6 +312,8 @@ def run_decode_bench(args, world, rank, local):
     peak, peak_src = peaks()
     bytes_launch = N * H * DECODE_BYTES_PER_TOKEN_HEAD
     achieved = bytes_launch / (ms_local / args.steps / 1e3) / 1e9
+    per_unit, _ = profile_traffic(DECODE_SRC, DECODE_PROFILE, "traffic_bytes_per_token_head")
+    traffic = None if per_unit is None else per_unit * N * H
     if rank == 0:
         print(json.dumps({
             "metric": "KDA decode step token-heads/s (H=32, K=V=128, fp32 state in HBM)",
@@ -319,7 +324,7 @@ def run_decode_bench(args, world, rank, local):
             "config": {"workload": f"decode_N{N}_H{H}", "sequences": N * world, "heads": H,
                        "l2": f"state {N * H * 64 // 1024} MB per rank > 126 MB L2"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
+                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                          "alg_bytes_per_launch": bytes_launch, "kernel": "decode_kernel"},
             "clocks": clk.summary(), "gpu_launches": args.steps}), flush=True)
     return 0
