@@ -24,13 +24,15 @@
 //   1. Forward sweep over the sequence; the state before every 64-token chunk is
 //      stored in the workspace.
 //   2. Reverse over the chunks.  For each chunk: re-run it from its checkpoint and
-//      keep the state before each 8-token sub-chunk (workspace, per CTA).  Then,
+//      keep the state before each 4-token sub-chunk (workspace, per CTA).  Then,
 //      per sub-chunk in reverse, per token in reverse, re-run the sub-chunk from its
-//      start state up to the token (at most 7 steps) and take the reverse step.
-// Reductions over v (for dq^, dk^, dalpha) sum the thread's two columns, reduce-
-// scatter over the warp's four column groups and then sum over the 16 warps in
-// shared memory.  The norms, gate and sigmoid gradients of a sub-chunk are taken
-// once its 8 tokens are done.  Everything is fp32 on the CUDA cores: each step is a
+//      start state up to the token (at most 3 steps) and take the reverse step.
+// Reductions over v (for dq^, dk^, dalpha) sum the thread's two columns and
+// reduce-scatter over the warp's four column groups; each token's per-warp partials
+// go to their own shared-memory slot, summed over the 16 warps once the sub-chunk's
+// tokens are done (no barrier per token).  The norms, gate and sigmoid gradients of
+// the sub-chunk follow.  While a sub-chunk computes, the rows of the next one are
+// prefetched into L2.  Everything is fp32 on the CUDA cores: each step is a
 // matrix-vector product on the state, with no contraction large enough for the
 // tensor cores.
 #include <cstddef>
@@ -45,7 +47,7 @@ constexpr int BT = 512;          // threads per CTA
 constexpr int NW = BT / 32;      // 16 warps
 constexpr int RR = 16;           // state rows per thread (per column)
 constexpr int NS = 2 * RR;       // state entries per thread
-constexpr int SUB = 8;           // tokens per sub-chunk
+constexpr int SUB = 4;           // tokens per sub-chunk
 constexpr int CH = 64;           // tokens per checkpoint chunk
 constexpr int NSUB = CH / SUB;   // sub-chunks per chunk
 constexpr int STATE = kHead * kHead;
@@ -60,10 +62,10 @@ struct Smem {
     alignas(16) float zs[SUB][kHead];
     alignas(16) float vv[SUB][kHead];
     alignas(16) float dO[SUB][kHead];
-    alignas(16) float red[2][NW][3][kHead];  // per-warp row sums of one token (double-buffered)
+    alignas(16) float red[SUB][NW][3][kHead];  // per-warp row sums of each token of the sub-chunk
     alignas(16) float res[SUB][3][kHead];    // dq^ / scale, dk^, dalpha per token of the sub-chunk
     float b[SUB], rq[SUB], rk[SUB];
-    float redb[2][NW];
+    float redb[SUB][NW];
     float resb[SUB];             // db per token
     float dtb[kHead];
     float pacc[SUB][kHead + 1];  // per-epilogue-warp partial ddt_bias and dA_log
@@ -172,6 +174,24 @@ __device__ void stage(Smem &sm, const BwdParams &p, int64_t tok, int L, int64_t 
     }
 }
 
+// Hint the rows of tokens [tok, tok + L) of head h towards L2, so that the stage() of
+// that sub-chunk waits on L2 rather than DRAM: one 128-byte line per thread (two per
+// 256-byte row of q, k, g, v and, with want_dO, dO), beta by threads 448 and up.
+__device__ __forceinline__ void prefetch_rows(const BwdParams &p, int64_t tok, int L, int64_t h,
+                                              bool want_dO)
+{
+    const int t = threadIdx.x;
+    const int narr = want_dO ? 5 : 4;
+    if (t < narr * 2 * L) {
+        const int a = t / (2 * L), rem = t - a * 2 * L, tt = rem >> 1, half = rem & 1;
+        const __nv_bfloat16 *base = a == 0 ? p.q : a == 1 ? p.k : a == 2 ? p.g : a == 3 ? p.v : p.dout;
+        const __nv_bfloat16 *addr = base + ((tok + tt) * p.H + h) * kHead + 64 * half;
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(addr));
+    } else if (t >= 448 && t < 448 + L) {
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(p.beta + (tok + (t - 448)) * p.H + h));
+    }
+}
+
 // One token of the recurrence on this thread's 16 rows of its two columns.
 // s[i] is column 2 cg, s[RR + i] column 2 cg + 1.
 __device__ __forceinline__ void fwd_step(float (&s)[NS], const Smem &sm, int tt, const Lane &L)
@@ -266,6 +286,8 @@ __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
                 __syncthreads();
                 stage(sm, p, bos + t0, Lj, h, ea, false);
                 __syncthreads();
+                if (t0 + SUB < len)
+                    prefetch_rows(p, bos + t0 + SUB, (int)(len - t0 - SUB < SUB ? len - t0 - SUB : SUB), h, false);
                 for (int tt = 0; tt < Lj; ++tt) fwd_step(s, sm, tt, L);
             }
         }
@@ -307,6 +329,11 @@ __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
                 __syncthreads();
                 stage(sm, p, bos + n * CH + j * SUB, SUB, h, ea, false);
                 __syncthreads();
+                {
+                    // next: sub-chunk j + 1 here, or (the last one) the first of 2b, with dO
+                    const int64_t tn = n * CH + (j + 1) * SUB;
+                    prefetch_rows(p, bos + tn, (int)(len - tn < SUB ? len - tn : SUB), h, j + 1 == nsub - 1);
+                }
                 for (int tt = 0; tt < SUB; ++tt) fwd_step(s, sm, tt, L);
             }
             // 2b. sub-chunks in reverse
@@ -318,6 +345,11 @@ __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
 #pragma unroll
                 for (int i = 0; i < NS / 4; ++i) sm.ssub[i][tid] = scr[((size_t)j * (NS / 4) + i) * BT + tid];
                 __syncthreads();
+                // next: sub-chunk j - 1 (with dO), or the first sub-chunk of chunk n - 1 (2a)
+                if (j > 0)
+                    prefetch_rows(p, bos + t0 - SUB, SUB, h, true);
+                else if (n > 0)
+                    prefetch_rows(p, bos + (n - 1) * CH, SUB, h, false);
                 for (int tt = Lj - 1; tt >= 0; --tt) {
 #pragma unroll
                     for (int i = 0; i < NS / 4; ++i) {
@@ -350,7 +382,6 @@ __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
                     const float r0 = v2.x - pa0, r1 = v2.y - pa1;
                     const float br0 = bt * r0, br1 = bt * r1;
                     const float dOs0 = p.scale * o2.x, dOs1 = p.scale * o2.y;
-                    const int buf = tt & 1;
                     float e0 = 0.f, e1 = 0.f;
                     // dS_t += scale q^ dO^T; dq^ partial S_t dO; e partial dS^T k^
                     {
@@ -379,14 +410,14 @@ __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
                                 hf[4 * g + j2] = scatter_a(x[0], x[1], L.cgl);
                             }
                         }
-                        *reinterpret_cast<float4 *>(&sm.red[buf][warp][0][32 * L.cgl + 4 * L.r8]) =
+                        *reinterpret_cast<float4 *>(&sm.red[tt][warp][0][32 * L.cgl + 4 * L.r8]) =
                             scatter_b(hf, L.cgl);
                     }
                     e0 = rows_sum(e0);
                     e1 = rows_sum(e1);
                     const float dr0 = bt * e0, dr1 = bt * e1;
                     const float dbw = warp_sum(L.r8 == 0 ? fmaf(r0, e0, r1 * e1) : 0.f);
-                    if (lane == 0) sm.redb[buf][warp] = dbw;
+                    if (lane == 0) sm.redb[tt][warp] = dbw;
                     if (L.r8 == 0)
                         *reinterpret_cast<float2 *>(p.dv + (bos + t0 + tt) * p.H * kHead + h * kHead + L.v0) =
                             make_float2(dr0, dr1);
@@ -409,7 +440,7 @@ __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
                                 hf[4 * g + j2] = scatter_a(x[0], x[1], L.cgl);
                             }
                         }
-                        *reinterpret_cast<float4 *>(&sm.red[buf][warp][1][32 * L.cgl + 4 * L.r8]) =
+                        *reinterpret_cast<float4 *>(&sm.red[tt][warp][1][32 * L.cgl + 4 * L.r8]) =
                             scatter_b(hf, L.cgl);
                     }
                     // dS' = dS - k^ dr^T; dalpha partial rowsum(dS' o S_{t-1}); dS_{t-1} = alpha dS'
@@ -435,22 +466,24 @@ __global__ void __launch_bounds__(BT, 1) bwd_kernel(const BwdParams p)
                                 hf[4 * g + j2] = scatter_a(x[0], x[1], L.cgl);
                             }
                         }
-                        *reinterpret_cast<float4 *>(&sm.red[buf][warp][2][32 * L.cgl + 4 * L.r8]) =
+                        *reinterpret_cast<float4 *>(&sm.red[tt][warp][2][32 * L.cgl + 4 * L.r8]) =
                             scatter_b(hf, L.cgl);
                     }
-                    __syncthreads();
-                    if (tid < 3 * kHead) {
-                        const int arr = tid >> 7, c = tid & (kHead - 1);
-                        float acc = 0.f;
+                }
+                // sums over the 16 warps of every token's partials
+                __syncthreads();
+                for (int it = tid; it < Lj * 3 * kHead; it += BT) {
+                    const int tt = it / (3 * kHead), r = it - tt * 3 * kHead, arr = r >> 7, c = r & (kHead - 1);
+                    float acc = 0.f;
 #pragma unroll
-                        for (int w = 0; w < NW; ++w) acc += sm.red[buf][w][arr][c];
-                        sm.res[tt][arr][c] = acc;
-                    } else if (tid == 3 * kHead) {
-                        float acc = 0.f;
+                    for (int w = 0; w < NW; ++w) acc += sm.red[tt][w][arr][c];
+                    sm.res[tt][arr][c] = acc;
+                }
+                if (tid < Lj) {
+                    float acc = 0.f;
 #pragma unroll
-                        for (int w = 0; w < NW; ++w) acc += sm.redb[buf][w];
-                        sm.resb[tt] = acc;
-                    }
+                    for (int w = 0; w < NW; ++w) acc += sm.redb[tid][w];
+                    sm.resb[tid] = acc;
                 }
                 __syncthreads();
                 // 2c. gradients through the activations of the sub-chunk's tokens
