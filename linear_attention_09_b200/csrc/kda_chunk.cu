@@ -57,6 +57,7 @@ constexpr int NT_MMA = 32;   // tensor-core issue warp for the in-chunk products
 constexpr int NT = NT_IN + NT_ST + NT_MMA;
 constexpr uint32_t BAR_IN = 1, BAR_ST = 2;  // named barriers of the two roles
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kLptMax = 128;  // varlen batches up to this many sequences run longest first
 
 // ---- shared memory (byte offsets from a 1024-byte aligned base) ----
 // q, k, g, v tiles arrive by TMA as 2 boxes of [64 tokens][64 channels] bf16 with
@@ -174,6 +175,7 @@ struct Ctx {
     Bars *bars;
     uint32_t tb;  // TMEM base
     int64_t h, H, tok0, len, rstride;
+    int64_t unit;  // (sequence, head) unit = sequence * H + head
     int nchunks;
 };
 
@@ -766,8 +768,7 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
     const uint32_t lq = (uint32_t)((warp & 3) * 32) << 16;
     const bool leader = (v == 0);
     const int64_t H = cx.H, h = cx.h, rstride = cx.rstride;
-    const int64_t sidx = blockIdx.x;  // (sequence, head) unit = sequence * H + head
-    const size_t state_off = (size_t)sidx * kHead * kHead;
+    const size_t state_off = (size_t)cx.unit * kHead * kHead;
     uint32_t mma_cnt = 0;
     bool ok = true;
 
@@ -989,8 +990,28 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
 
     const int tid = threadIdx.x, warp = tid >> 5;
     cx.H = p.H;
-    const int64_t s = blockIdx.x / p.H;
+    int64_t s = blockIdx.x / p.H;
     cx.h = blockIdx.x % p.H;
+    if (p.cu && p.N > 1 && p.N <= kLptMax) {
+        // Longest sequences first: CTA group r takes the sequence of rank r in decreasing
+        // length (ties by index; the ranks are a permutation), so that the end of the grid
+        // holds short sequences rather than a long one started last.  The A/P region is
+        // free until the first chunk.
+        int64_t *lens = reinterpret_cast<int64_t *>(sm + SM_APA);
+        int *pick = reinterpret_cast<int *>(sm + SM_APA + 8 * kLptMax);
+        for (int i = tid; i < p.N; i += NT) lens[i] = p.cu[i + 1] - p.cu[i];
+        __syncthreads();
+        for (int c = tid; c < p.N; c += NT) {
+            const int64_t lc = lens[c];
+            int64_t rank = 0;
+            for (int u = 0; u < p.N; ++u) rank += (lens[u] > lc) || (lens[u] == lc && u < c);
+            if (rank == s) *pick = c;
+        }
+        __syncthreads();
+        s = *pick;
+        __syncthreads();  // every thread has read pick before the region is reused
+    }
+    cx.unit = s * p.H + cx.h;
     if (p.cu) {
         cx.tok0 = p.cu[s];
         cx.len = p.cu[s + 1] - cx.tok0;
