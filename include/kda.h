@@ -52,8 +52,8 @@ typedef struct CUstream_st *kda_stream_t;
 #define KDA_STATE_F32 1
 #define KDA_STATE_BF16 2
 
-/* Return codes.  Every negative code except KDA_ERR_CUDA is detected on the host
- * before anything is launched. */
+/* Return codes.  Every negative code except KDA_ERR_CUDA and KDA_ERR_SEQLENS is
+ * detected on the host before anything is launched. */
 #define KDA_OK 0
 #define KDA_ERR_HEAD_DIM (-1)     /* K != 128 or V != 128 */
 #define KDA_ERR_NULL (-2)         /* a required pointer is NULL */
@@ -70,6 +70,8 @@ typedef struct CUstream_st *kda_stream_t;
 #define KDA_ERR_DEVICE (-11)      /* no usable sm_100 device for this call */
 #define KDA_ERR_SCALE (-12)       /* scale is not finite */
 #define KDA_ERR_LAYOUT (-13)      /* state_layout is not KV / VK */
+#define KDA_ERR_SEQLENS (-14)     /* with checks on (kda_set_checks): cu_seqlens is not
+                                     non-decreasing within [0, B*T]; nothing was run */
 
 /* State layouts (kda_fwd_ex).  The FLA call on the pages passes
  * transpose_state_layout=True, i.e. per (sequence, head) the state stored value-major. */
@@ -213,6 +215,17 @@ int kda_bwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_b
             float *dA_log, float *ddt_bias, float *d_initial_state, void *workspace,
             size_t workspace_bytes, int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
             kda_stream_t stream);
+
+/*
+ * kda_set_checks -- debug checks of device-resident arguments, process-wide; returns
+ * the previous level.  0 (default): none; the kernels trust cu_seqlens.  1: every call
+ * with cu_seqlens (kda_fwd, kda_fwd_ex, kda_bwd) first checks on the device, on its
+ * stream, that 0 <= cu_seqlens[0] <= ... <= cu_seqlens[num_seqs] <= B*T, reads the
+ * result back (a stream synchronisation) and returns KDA_ERR_SEQLENS without
+ * launching anything if it fails.  The [cu_seqlens[0], cu_seqlens[num_seqs]) range
+ * may be any part of the rows (the host entry point passes sub-ranges).
+ */
+int kda_set_checks(int level);
 
 /* Human-readable text of a return code (static storage; never NULL). */
 const char *kda_strerror(int code);

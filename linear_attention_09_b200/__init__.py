@@ -6,7 +6,8 @@ PyTorch fallback: if the library cannot be loaded, the calls raise.
 
 The functions mirror the C ABI in ``include/kda.h``:
   kda_fwd, kda_fwd_ex, kda_decode, kda_bwd, kda_bwd_workspace_size, kda_fwd_host,
-  kda_fwd_host_workspace_size, kda_strerror, kda_last_launch_count, kda_device_status.
+  kda_fwd_host_workspace_size, kda_set_checks, kda_strerror, kda_last_launch_count,
+  kda_device_status.
 """
 from __future__ import annotations
 
@@ -65,6 +66,8 @@ def lib() -> ctypes.CDLL:
             L.kda_bwd.restype = I
             L.kda_bwd_workspace_size.argtypes = [I64, I64, I64, I64, I64, I64]
             L.kda_bwd_workspace_size.restype = SZ
+            L.kda_set_checks.argtypes = [I]
+            L.kda_set_checks.restype = I
             L.kda_strerror.argtypes = [I]
             L.kda_strerror.restype = ctypes.c_char_p
             L.kda_last_launch_count.argtypes = []
@@ -77,6 +80,12 @@ def lib() -> ctypes.CDLL:
 
 def kda_strerror(code: int) -> str:
     return lib().kda_strerror(int(code)).decode()
+
+
+def kda_set_checks(level: int) -> int:
+    """Debug checks of device arguments (1: cu_seqlens checked on the device before each
+    varlen call, synchronously); returns the previous level."""
+    return int(lib().kda_set_checks(int(level)))
 
 
 def kda_last_launch_count() -> int:

@@ -9,6 +9,35 @@
 namespace {
 
 thread_local int g_last_launches = 0;
+int g_checks = 0;  // kda_set_checks level
+
+// cu_seqlens check of the debug level: bad |= 1 unless 0 <= cu[0] <= ... <= cu[n] <= rows.
+__global__ void check_offsets_kernel(const int64_t *cu, int64_t n, int64_t rows, int *bad)
+{
+    for (int64_t i = threadIdx.x; i <= n; i += blockDim.x) {
+        const int64_t c = cu[i];
+        if (c < 0 || c > rows || (i > 0 && cu[i - 1] > c)) atomicOr(bad, 1);
+    }
+}
+
+// Runs the check on `stream` and waits for it; KDA_OK, KDA_ERR_SEQLENS or KDA_ERR_CUDA.
+int check_offsets(const int64_t *cu, int64_t n, int64_t rows, cudaStream_t stream)
+{
+    int *bad = nullptr;
+    if (cudaMallocAsync(reinterpret_cast<void **>(&bad), sizeof(int), stream) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    int host = 0;
+    bool ok = cudaMemsetAsync(bad, 0, sizeof(int), stream) == cudaSuccess;
+    if (ok) {
+        check_offsets_kernel<<<1, 256, 0, stream>>>(cu, n, rows, bad);
+        ok = cudaGetLastError() == cudaSuccess &&
+             cudaMemcpyAsync(&host, bad, sizeof(int), cudaMemcpyDeviceToHost, stream) == cudaSuccess;
+    }
+    ok = (cudaFreeAsync(bad, stream) == cudaSuccess) && ok;
+    ok = ok && cudaStreamSynchronize(stream) == cudaSuccess;
+    if (!ok) return KDA_ERR_CUDA;
+    return host ? KDA_ERR_SEQLENS : KDA_OK;
+}
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -115,11 +144,19 @@ extern "C" const char *kda_strerror(int code)
     case KDA_ERR_DEVICE: return "no usable sm_100 (B200) device";
     case KDA_ERR_SCALE: return "scale must be finite";
     case KDA_ERR_LAYOUT: return "state_layout must be KDA_LAYOUT_KV or KDA_LAYOUT_VK";
+    case KDA_ERR_SEQLENS: return "cu_seqlens must be non-decreasing within [0, B*T] (device check)";
     default: return "unknown kda error code";
     }
 }
 
 extern "C" int kda_last_launch_count(void) { return g_last_launches; }
+
+extern "C" int kda_set_checks(int level)
+{
+    const int old = g_checks;
+    g_checks = level;
+    return old;
+}
 
 extern "C" int kda_device_status(int reset) { return kda::chunked_device_error(reset != 0); }
 
@@ -140,6 +177,9 @@ extern "C" int kda_fwd_ex(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *
     if (final_state && final_state_dtype != KDA_STATE_F32 && final_state_dtype != KDA_STATE_BF16)
         return KDA_ERR_STATE_DTYPE;
     if ((rc = check_device()) != KDA_OK) return rc;
+    if (g_checks && cu_seqlens &&
+        (rc = check_offsets(cu_seqlens, N, B * T, reinterpret_cast<cudaStream_t>(stream))) != KDA_OK)
+        return rc;
     kda::FwdParams p{};
     p.q = reinterpret_cast<const __nv_bfloat16 *>(q);
     p.k = reinterpret_cast<const __nv_bfloat16 *>(k);
@@ -264,6 +304,9 @@ extern "C" int kda_bwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, 
     if (!workspace || workspace_bytes < need) return KDA_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return KDA_ERR_ALIGN;
     if ((rc = check_device()) != KDA_OK) return rc;
+    if (g_checks && cu_seqlens &&
+        (rc = check_offsets(cu_seqlens, N, B * T, reinterpret_cast<cudaStream_t>(stream))) != KDA_OK)
+        return rc;
     kda::BwdParams p{};
     p.q = reinterpret_cast<const __nv_bfloat16 *>(q);
     p.k = reinterpret_cast<const __nv_bfloat16 *>(k);

@@ -206,3 +206,13 @@ def test_bwd_valid_arguments_without_device(L):
     if not torch.cuda.is_available():
         assert call_bwd() == -11
         assert call_bwd(T=0, q=None, dout=None, dq=None) == -11  # T = 0 still writes dA_log
+
+
+def test_checks_level_and_message(L):
+    old = kda.kda_set_checks(1)
+    try:
+        assert kda.kda_set_checks(1) == 1
+    finally:
+        kda.kda_set_checks(old)
+    assert kda.kda_set_checks(old) == old
+    assert "cu_seqlens" in kda.kda_strerror(-14)

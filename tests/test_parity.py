@@ -319,3 +319,34 @@ def test_pipelined_host_entry_matches_device_entry(case):
     for (b, t0, nn) in inp.seq_bounds():
         np.testing.assert_array_equal(out_h[b, t0:t0 + nn].float().numpy(), out_d[b, t0:t0 + nn])
     np.testing.assert_array_equal(fin_h.numpy(), fin_d)
+
+
+@pytest.mark.gpu
+def test_device_offset_check_rejects_bad_cu_seqlens():
+    """With checks on, a varlen call whose cu_seqlens is not non-decreasing within
+    [0, B*T] returns KDA_ERR_SEQLENS before any kernel runs (outputs untouched); a valid
+    one gives the same bits as with checks off."""
+    inp = small(lengths=[5, 10, 20], init="f32", seed=41)
+    d = lambda t: None if t is None else t.cuda()
+    args = (d(inp.q), d(inp.k), d(inp.v), d(inp.g), d(inp.beta), inp.scale, d(inp.A_log),
+            d(inp.dt_bias), inp.lower_bound)
+    ref, ref_fin = kda.kda_fwd(*args, initial_state=d(inp.initial_state), cu_seqlens=d(inp.cu_seqlens))
+    old = kda.kda_set_checks(1)
+    try:
+        out, fin = kda.kda_fwd(*args, initial_state=d(inp.initial_state), cu_seqlens=d(inp.cu_seqlens))
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref) and torch.equal(fin, ref_fin)
+        for bad in ([0, 10, 5, 35], [0, 5, 15, 36], [-1, 5, 15, 35]):
+            cu = torch.tensor(bad, dtype=torch.int64, device="cuda")
+            sentinel = torch.full_like(ref, 7.0)
+            with pytest.raises(kda.KDAError) as e:
+                kda.kda_fwd(*args, initial_state=d(inp.initial_state), cu_seqlens=cu, out=sentinel)
+            assert e.value.code == -14
+            dO = torch.zeros_like(ref)
+            with pytest.raises(kda.KDAError) as e:
+                kda.kda_bwd(*args, dO, initial_state=d(inp.initial_state), cu_seqlens=cu)
+            assert e.value.code == -14
+            torch.cuda.synchronize()
+            assert bool((sentinel == 7.0).all())
+    finally:
+        kda.kda_set_checks(old)
