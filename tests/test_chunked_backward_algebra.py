@@ -39,3 +39,48 @@ def test_varlen_with_empty_and_boundary_lengths():
 
 def test_strong_decay_without_state_gradient():
     run(T=200, g_std=2.0, init=None, dfinal=False, seed=3)
+
+
+# Precision plan for a tensor-core backward, emulated on the CPU (chunked_bwd_ref's
+# tiled form with operand rounding): A and P in tf32 (as the forward kernel), their
+# adjoints in fp32, every other product operand fp16 with a power-of-two scale per row
+# or column (along the non-contracted dimension), T fp16, the solve adjoint tf32.
+BWD_PLAN = {"APf": "tf32", "APb": "f32", "F": "f16", "T": "f16", "dM": "tf32", "Minv": "f32"}
+BARS = ("dq", "dk", "dv", "dg", "dbeta", "dA_log", "ddt_bias", "dS0")
+
+
+def _case(g_std, init, seed):
+    inp = ki.make_inputs(ki.Workload("cbp", B=1, T=200, H=2, init_state=init, g_std=g_std), seed)
+    gen = torch.Generator().manual_seed(2)
+    dO = torch.randn(inp.v.shape, generator=gen).to(torch.bfloat16)
+    dSf = torch.randn((1, 2, 128, 128), generator=gen) * 0.1
+    return inp, dO, dSf, oracle.backward_inputs(inp, dO, dSf, want_dlam=True)
+
+
+def _rel(a, b):
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+def test_tiled_form_equals_the_oracle():
+    """Sub-blocks with mid-block reference tokens (no rounding) change nothing."""
+    inp, dO, dSf, ref = _case(2.0, "f32", 5)
+    got = cb.backward_inputs(inp, dO, dSf, tiled=True)
+    for n in BARS:
+        assert _rel(got[n], ref[n]) <= 1e-11, n
+
+
+@pytest.mark.parametrize("g_std,init,seed", [(2.0, "f32", 5), (1.0, None, 6)])
+def test_backward_precision_plan_meets_the_bars(g_std, init, seed):
+    inp, dO, dSf, ref = _case(g_std, init, seed)
+    got = cb.backward_inputs(inp, dO, dSf, prec=BWD_PLAN)
+    for n in BARS:
+        assert _rel(got[n], ref[n]) <= 1e-3, (n, _rel(got[n], ref[n]))
+
+
+def test_tf32_adjoints_of_the_decay_weighted_products_break_the_gate_gradients():
+    """Why the plan keeps those products in fp32: with their operands in tf32 the gate
+    gradients (sums over the chunk of nearly cancelling terms) miss the bar tenfold."""
+    inp, dO, dSf, ref = _case(2.0, "f32", 5)
+    got = cb.backward_inputs(inp, dO, dSf, prec=dict(BWD_PLAN, APb="tf32"))
+    assert _rel(got["ddt_bias"], ref["ddt_bias"]) > 1e-2
+    assert _rel(got["dv"], ref["dv"]) <= 1e-3  # the rest is unaffected
