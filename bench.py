@@ -214,6 +214,38 @@ def cpu_baseline(min_seconds=10.0, max_passes=8):
                       f"(out and final state), {dt:.1f} s"}
 
 
+def cpu_config_baseline(config_id, min_seconds=10.0):
+    """The fp64 oracle on a bounded sample of parity workload ``config_id``: all heads of
+    the first m sequences, m doubling until one pass takes at least a second, then
+    repeated until ``min_seconds`` of CPU work.  tokens/s counts a token once for its H
+    heads (the sampled token-heads divided by H)."""
+    import kda_inputs as ki
+    import numpy as np
+    import oracle
+    inp = ki.make_inputs(config_id)
+    seqs, H = inp.seq_bounds(), inp.H
+    m = 1
+    while True:
+        mask = np.zeros(len(seqs) * H, np.uint8)
+        mask[: m * H] = 1
+        t0 = time.perf_counter()
+        oracle.forward_inputs(inp, want_final=True, mask=mask)
+        dt = time.perf_counter() - t0
+        if dt >= 1.0 or m >= len(seqs):
+            break
+        m = min(len(seqs), 2 * m)
+    passes = 1
+    while dt < min_seconds and passes < 64:
+        t0 = time.perf_counter()
+        oracle.forward_inputs(inp, want_final=True, mask=mask)
+        dt += time.perf_counter() - t0
+        passes += 1
+    tokens = sum(n for _, _, n in seqs[:m]) * passes
+    return {"value": tokens / dt, "unit": UNIT, "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{passes} pass(es) over {m} of {len(seqs)} sequence(s) x {H} heads of "
+                      f"workload {ki.WORKLOADS[config_id].name} (out and final state), {dt:.1f} s"}
+
+
 def dist_setup(n):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -245,6 +277,19 @@ def max_over_ranks(x, world):
 
 def run_reference(args, world, rank):
     if rank != 0:
+        return 0
+    if args.config_id is not None:
+        import kda_inputs as ki
+        base = cpu_config_baseline(args.config_id)
+        name = ki.WORKLOADS[args.config_id].name
+        print(json.dumps({
+            "impl": "reference", "metric": f"KDA fwd prefill tokens/s, workload {name}",
+            "value": base["value"], "unit": UNIT, "n_gpus": args.gpus, "steps": 1, "warmup": 0,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": name, "parallelism": "cpu"},
+            "cpu_baseline": base,
+            "e2e": {"value": base["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
         return 0
     for _ in range(args.warmup):
         pass  # the oracle has no warm-up state; steps below are timed one by one

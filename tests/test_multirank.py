@@ -68,3 +68,14 @@ def test_reference_arm_two_ranks_prints_once():
     assert d["value"] > 0 and d["unit"] == "tokens/s"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_on_a_parity_workload():
+    """--impl reference --config-id N times the oracle on a bounded sample of workload N."""
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--config-id", "0"]
+    res = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stderr[-2000:]
+    d = json.loads([l for l in res.stdout.splitlines() if l.startswith("{")][0])
+    assert d["impl"] == "reference" and "tiny_B1_T512_H4" in d["metric"]
+    assert d["value"] > 0 and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0
