@@ -191,7 +191,8 @@ def chunk_backward_tiled(qh, kh, v, b, lam, scale, dO, S0=None, dSf=None, C=64, 
     """``chunk_backward`` with the decay-weighted products in sub-blocks and the
     tensor-core operands rounded per ``prec``.  Operand groups:
       "APf"  factors of the decay-weighted products A and P,
-      "APb"  operands of their adjoints (dA, dP and the k^ / q^ factors),
+      "APb"  operands of their adjoints (dA, dP and the k^ / q^ factors); "tf32x3"
+             emulates the three-product split of each operand into tf32 halves,
       "Minv" the solve result, "dM" the solve adjoint products,
       "T"    T as a product operand, "F"  the other fp16 operands (k^Gam, q^Gam, K',
       P, S0, dS, dO, U, Y, dU, dY with per-slice scales).
@@ -215,6 +216,15 @@ def chunk_backward_tiled(qh, kh, v, b, lam, scale, dO, S0=None, dSf=None, C=64, 
                 M[I0:I1, J0:J1] = R("APf", x[I0:I1] * rho) @ R("APf", k[J0:J1] * sig).T
         return np.tril(M, -1 if strict else 0)
 
+    def mm(a, b_):
+        """Product of the adjoint operands: rounded per "APb", or with "tf32x3" the
+        three-term split a_hi b_hi + a_hi b_lo + a_lo b_hi of tf32 halves."""
+        if prec.get("APb") == "tf32x3":
+            ah, bh = round_to(a, "tf32"), round_to(b_, "tf32")
+            al, bl = round_to(a - ah, "tf32"), round_to(b_ - bh, "tf32")
+            return ah @ bh + ah @ bl + al @ bh
+        return R("APb", a) @ R("APb", b_)
+
     def gram_adjoint(dM, x, k, G):
         """(sum_j dM_ij k_j e^{G_i-G_j}, sum_i dM_ij x_i e^{G_i-G_j}) per channel."""
         L = G.shape[0]
@@ -225,9 +235,9 @@ def chunk_backward_tiled(qh, kh, v, b, lam, scale, dO, S0=None, dSf=None, C=64, 
                 if J0 >= I1:
                     continue
                 sig = np.exp(G[r] - G[J0:J1])
-                blk = R("APb", dM[I0:I1, J0:J1])
-                ti[I0:I1] += rho * (blk @ R("APb", k[J0:J1] * sig))
-                tj[J0:J1] += sig * (blk.T @ R("APb", x[I0:I1] * rho))
+                blk, ks, xr = dM[I0:I1, J0:J1], k[J0:J1] * sig, x[I0:I1] * rho
+                ti[I0:I1] += rho * mm(blk, ks)
+                tj[J0:J1] += sig * mm(blk.T, xr)
         return ti, tj
 
     def solve(A, b_):

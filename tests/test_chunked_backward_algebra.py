@@ -84,3 +84,12 @@ def test_tf32_adjoints_of_the_decay_weighted_products_break_the_gate_gradients()
     got = cb.backward_inputs(inp, dO, dSf, prec=dict(BWD_PLAN, APb="tf32"))
     assert _rel(got["ddt_bias"], ref["ddt_bias"]) > 1e-2
     assert _rel(got["dv"], ref["dv"]) <= 1e-3  # the rest is unaffected
+
+
+def test_three_tf32_products_recover_the_adjoints():
+    """The fp32-grade adjoint products the plan needs, made of tf32 tensor-core products:
+    a b ~ a_hi b_hi + a_hi b_lo + a_lo b_hi (halves rounded to tf32) meets the bars."""
+    inp, dO, dSf, ref = _case(2.0, "f32", 5)
+    got = cb.backward_inputs(inp, dO, dSf, prec=dict(BWD_PLAN, APb="tf32x3"))
+    for n in BARS:
+        assert _rel(got[n], ref[n]) <= 1e-3, (n, _rel(got[n], ref[n]))
