@@ -364,3 +364,41 @@ def test_workload_inputs_are_deterministic():
     # the varlen recipe's lengths are the first draws of the seeded stream
     lens = ki.draw_lengths(np.random.Generator(np.random.PCG64(2)), 16, 256, 4096, 32768)
     assert lens.sum() == 32768 and lens.min() >= 256 and lens.max() <= 4096 and len(lens) == 16
+
+
+# ---------------------------------------------------------------------------
+# Reduction to Gated DeltaNet: KDA refines it with per-channel decay, so with a gate
+# that is the same on every channel the decay is a scalar per token.
+# ---------------------------------------------------------------------------
+def test_channel_constant_gate_reduces_to_scalar_decay_delta_rule():
+    """g and dt_bias constant across channels: the full public path must equal a
+    scalar-decay delta rule written independently here, S <- a (S - b k (k^T S))
+    + b k v^T (Diag(a) = a I commutes with the erase), out = scale S^T q."""
+    rng = np.random.default_rng(21)
+    B, T, H, K, V = 1, 40, 2, 8, 6
+    q = torch.randn((B, T, H, K), generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    k = torch.randn((B, T, H, K), generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
+    v = torch.randn((B, T, H, V), generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    gt = torch.randn((B, T, H, 1), generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    g = gt.expand(B, T, H, K).contiguous()                 # the same gate on every channel
+    beta = torch.randn((B, T, H), generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    A_log = np.log(rng.uniform(1, 16, H)).astype(np.float32)
+    dtb = np.repeat(rng.normal(0, 0.1, (H, 1)), K, axis=1).astype(np.float32)
+    S0 = (rng.standard_normal((B, H, K, V)) * 0.3).astype(np.float32)
+    scale, lb = 0.3, -5.0
+    b16 = lambda t: t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    out, fin = oracle.forward(b16(q), b16(k), b16(v), b16(g), b16(beta), scale, A_log, dtb, lb,
+                              S0, oracle.STATE_F32)
+    for h in range(H):
+        S = S0[0, h].astype(np.float64)
+        for t in range(T):
+            qq, kk = q[0, t, h].double().numpy(), k[0, t, h].double().numpy()
+            qh = qq / math.sqrt(qq @ qq + oracle.EPS)
+            kh = kk / math.sqrt(kk @ kk + oracle.EPS)
+            x = float(gt[0, t, h, 0]) + float(dtb[h, 0])
+            lam = max(lb, -math.exp(float(A_log[h])) * (max(x, 0) + math.log1p(math.exp(-abs(x)))))
+            a = math.exp(lam)
+            bb = 1 / (1 + math.exp(-float(beta[0, t, h])))
+            S = a * (S - bb * np.outer(kh, kh @ S)) + bb * np.outer(kh, v[0, t, h].double().numpy())
+            np.testing.assert_allclose(out[0, t, h], scale * S.T @ qh, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(fin[0, h], S, rtol=1e-12, atol=1e-13)
