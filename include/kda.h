@@ -70,8 +70,10 @@ typedef struct CUstream_st *kda_stream_t;
 #define KDA_ERR_DEVICE (-11)      /* no usable sm_100 device for this call */
 #define KDA_ERR_SCALE (-12)       /* scale is not finite */
 #define KDA_ERR_LAYOUT (-13)      /* state_layout is not KV / VK */
-#define KDA_ERR_SEQLENS (-14)     /* with checks on (kda_set_checks): cu_seqlens is not
-                                     non-decreasing within [0, B*T]; nothing was run */
+#define KDA_ERR_SEQLENS (-14)     /* cu_seqlens is not non-decreasing within [0, B*T]:
+                                     always checked by kda_fwd_host (host offsets), by the
+                                     device entry points with checks on (kda_set_checks);
+                                     nothing was run */
 
 /* State layouts (kda_fwd_ex).  The FLA call on the pages passes
  * transpose_state_layout=True, i.e. per (sequence, head) the state stored value-major. */
@@ -146,8 +148,10 @@ size_t kda_fwd_host_workspace_size(int64_t B, int64_t T, int64_t H, int64_t K, i
  * pieces (batch entries, or consecutive varlen sequences of about equal token
  * counts): the copies in of one piece (on `stream`), the kernel of another and the
  * copies out of a third (two library-owned streams per host thread and device)
- * overlap.  Output rows of tokens outside every sequence are not written.  Same
- * return codes as kda_fwd, plus KDA_ERR_WORKSPACE.
+ * overlap.  Output rows of tokens outside every sequence are not written.
+ * cu_seqlens is a host pointer here and is checked before anything is copied: offsets
+ * that are not non-decreasing within [0, B*T] give KDA_ERR_SEQLENS.  Same return codes
+ * as kda_fwd, plus KDA_ERR_WORKSPACE.
  */
 int kda_fwd_host(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
                  const kda_bf16 *beta, float scale, const float *A_log, const float *dt_bias,

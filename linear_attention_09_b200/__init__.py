@@ -123,6 +123,70 @@ def _stream_handle(stream, device) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _check_form(t, name, dtypes, shape):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor, got {type(t).__name__}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected "
+                        + " or ".join(str(d) for d in dtypes))
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major, no strides)")
+
+
+def _check_place(t, name, device, host):
+    if host:
+        if t.device.type != "cpu":
+            raise ValueError(f"{name} must be a host (CPU) tensor, got {t.device}")
+    elif t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor, got {t.device}")
+    elif device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device} (the device of q)")
+
+
+def _check_all(specs, device=None, host=False):
+    """Reject tensors the library cannot take: wrong shape, dtype or memory layout
+    (checked for every tensor first), then wrong device.  Nothing is launched on a bad
+    argument: a host pointer handed to a kernel would fault the GPU, and a strided view
+    or another dtype would be read as something else.  ``specs``: (tensor or None,
+    name, allowed dtypes, shape or None); None tensors are optional and skipped."""
+    specs = [sp for sp in specs if sp[0] is not None]
+    for t, name, dtypes, shape in specs:
+        _check_form(t, name, dtypes, shape)
+    for t, name, _, _ in specs:
+        _check_place(t, name, device, host)
+
+
+_BF16, _F32, _I64, _U8 = (torch.bfloat16,), (torch.float32,), (torch.int64,), (torch.uint8,)
+_STATE = (torch.float32, torch.bfloat16)
+
+
+def _check_call(q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens, extra=(),
+                host=False, state_shape=None):
+    """Shapes, dtypes, layouts and devices of the common arguments and of ``extra``
+    specs (q decides B, T, H, K and the device).  Returns (B, T, H, K, V, N)."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 4:
+        raise ValueError("q must be a 4-D tensor [B, T, H, K]")
+    if not isinstance(v, torch.Tensor) or v.dim() != 4:
+        raise ValueError("v must be a 4-D tensor [B, T, H, V]")
+    if cu_seqlens is not None and (not isinstance(cu_seqlens, torch.Tensor)
+                                   or cu_seqlens.dim() != 1):
+        raise ValueError("cu_seqlens must be a 1-D tensor [num_seqs + 1]")
+    B, T, H, K = q.shape
+    V = v.shape[3]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    dims = dict(B=B, T=T, H=H, K=K, V=V, N=N)
+    specs = [(q, "q", _BF16, (B, T, H, K)), (k, "k", _BF16, (B, T, H, K)),
+             (g, "g", _BF16, (B, T, H, K)), (v, "v", _BF16, (B, T, H, V)),
+             (beta, "beta", _BF16, (B, T, H)), (A_log, "A_log", _F32, (H,)),
+             (dt_bias, "dt_bias", _F32, (H, K)), (cu_seqlens, "cu_seqlens", _I64, None),
+             (initial_state, "initial_state", _STATE, state_shape or (N, H, K, V))]
+    specs += [(t, n, d, (sh(dims) if callable(sh) else sh)) for t, n, d, sh in extra]
+    _check_all(specs, None if host else q.device, host)
+    return B, T, H, K, V, N
+
+
 def kda_fwd(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, initial_state=None,
             final_state=None, cu_seqlens=None, out=None, output_final_state=True, stream=None):
     """Run the KDA forward pass on CUDA tensors; returns (out, final_state or None).
@@ -133,10 +197,11 @@ def kda_fwd(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, initial_state=
     given (then they are written), else they are allocated on q's device.  The
     call is asynchronous on ``stream`` (default: the current stream).
     """
-    B, T, H, K = q.shape
-    V = v.shape[3]
-    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
-    N = B if cu_seqlens is None else num_seqs
+    B, T, H, K, V, N = _check_call(
+        q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens,
+        extra=[(out, "out", _BF16, lambda d: (d["B"], d["T"], d["H"], d["V"])),
+               (final_state, "final_state", _F32, lambda d: (d["N"], d["H"], d["K"], d["V"]))])
+    num_seqs = 0 if cu_seqlens is None else N
     if out is None:
         out = torch.empty((B, T, H, V), dtype=torch.bfloat16, device=q.device)
     if final_state is None and output_final_state:
@@ -156,11 +221,14 @@ def kda_fwd_ex(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, initial_sta
     """``kda_fwd`` with the state variants: ``state_layout`` "kv" (S[k][v]) or "vk"
     (S[v][k], the transposed layout) for both states, and a bf16 or fp32 final state
     (``final_state_dtype``, or the dtype of a given ``final_state``)."""
-    B, T, H, K = q.shape
-    V = v.shape[3]
-    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
-    N = B if cu_seqlens is None else num_seqs
     layout = _LAYOUTS.get(state_layout, -1) if isinstance(state_layout, str) else int(state_layout)
+    vk = layout == KDA_LAYOUT_VK
+    B, T, H, K, V, N = _check_call(
+        q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens,
+        extra=[(out, "out", _BF16, lambda d: (d["B"], d["T"], d["H"], d["V"])),
+               (final_state, "final_state", _STATE,
+                lambda d: (d["N"], d["H"]) + ((d["V"], d["K"]) if vk else (d["K"], d["V"])))])
+    num_seqs = 0 if cu_seqlens is None else N
     if out is None:
         out = torch.empty((B, T, H, V), dtype=torch.bfloat16, device=q.device)
     if final_state is None and output_final_state:
@@ -182,8 +250,18 @@ def kda_decode(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, state, stat
     """One decode step on CUDA tensors: q, k, g bf16 [N,H,128], v bf16 [N,H,128], beta
     bf16 [N,H]; ``state`` fp32 [N,H,128,128] (S[k][v]) is updated in place unless
     ``state_out`` is given.  Returns (out [N,H,128] bf16, new state)."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 3 or not isinstance(v, torch.Tensor) \
+            or v.dim() != 3:
+        raise ValueError("q and v must be 3-D tensors [N, H, K] / [N, H, V]")
     N, H, K = q.shape
     V = v.shape[2]
+    if state is None:
+        raise ValueError("state is required")
+    _check_all([(q, "q", _BF16, (N, H, K)), (k, "k", _BF16, (N, H, K)), (g, "g", _BF16, (N, H, K)),
+                (v, "v", _BF16, (N, H, V)), (beta, "beta", _BF16, (N, H)),
+                (A_log, "A_log", _F32, (H,)), (dt_bias, "dt_bias", _F32, (H, K)),
+                (state, "state", _F32, (N, H, K, V)), (state_out, "state_out", _F32, (N, H, K, V)),
+                (out, "out", _BF16, (N, H, V))], q.device)
     if state_out is None:
         state_out = state
     if out is None:
@@ -212,10 +290,14 @@ def kda_bwd(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, d_out, initial
     ``want_d_initial_state``).  ``workspace`` is a CUDA uint8 tensor of at least
     ``kda_bwd_workspace_size`` bytes (allocated here if None).
     """
-    B, T, H, K = q.shape
-    V = v.shape[3]
-    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
-    N = B if cu_seqlens is None else num_seqs
+    if d_out is None:
+        raise ValueError("d_out is required")
+    B, T, H, K, V, N = _check_call(
+        q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens,
+        extra=[(d_out, "d_out", _BF16, lambda d: (d["B"], d["T"], d["H"], d["V"])),
+               (d_final_state, "d_final_state", _F32, lambda d: (d["N"], d["H"], d["K"], d["V"])),
+               (workspace, "workspace", _U8, None)])
+    num_seqs = 0 if cu_seqlens is None else N
     dev = q.device
     f32 = dict(dtype=torch.float32, device=dev)
     g_ = dict(dq=torch.empty((B, T, H, K), **f32), dk=torch.empty((B, T, H, K), **f32),
@@ -252,10 +334,13 @@ def kda_fwd_host(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, initial_s
     bytes (allocated here if None).  Returns (out, final_state or None); both are
     ready when the call returns.
     """
-    B, T, H, K = q.shape
-    V = v.shape[3]
-    num_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
-    N = B if cu_seqlens is None else num_seqs
+    B, T, H, K, V, N = _check_call(
+        q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens, host=True,
+        extra=[(out, "out", _BF16, lambda d: (d["B"], d["T"], d["H"], d["V"])),
+               (final_state, "final_state", _F32, lambda d: (d["N"], d["H"], d["K"], d["V"]))])
+    num_seqs = 0 if cu_seqlens is None else N
+    if workspace is not None:
+        _check_all([(workspace, "workspace", _U8, None)])
     if out is None:
         out = torch.empty((B, T, H, V), dtype=torch.bfloat16)
     if final_state is None and output_final_state:

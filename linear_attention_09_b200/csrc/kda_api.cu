@@ -429,6 +429,15 @@ extern "C" int kda_fwd_host(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16
                       initial_state_dtype, final_state, cu_seqlens, num_seqs, out, B, T, H, K, V,
                       &N);
     if (rc != KDA_OK) return rc;
+    // cu_seqlens is in host memory here, so it is checked before anything uses it: the
+    // piece plan and the copy offsets come from it
+    if (cu_seqlens) {
+        const int64_t rows = B * T;
+        for (int64_t i = 0; i <= num_seqs; ++i) {
+            const int64_t c = cu_seqlens[i];
+            if (c < 0 || c > rows || (i > 0 && cu_seqlens[i - 1] > c)) return KDA_ERR_SEQLENS;
+        }
+    }
     if ((rc = check_device()) != KDA_OK) return rc;
     const HostSizes s = host_sizes(B, T, H, N, initial_state_dtype, final_state != nullptr,
                                    cu_seqlens != nullptr);
@@ -459,11 +468,11 @@ extern "C" int kda_fwd_host(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16
     Piece pcs[8];
     const int np = (B * T == 0) ? 0 : plan_pieces(B, T, cu_seqlens, num_seqs, pcs, 8);
     // A varlen piece's last tile also reads up to 63 rows after it, which belong to the
-    // next piece and may not be copied in yet; the kernel masks those tokens but needs
-    // finite values there, so they start as zeros.
+    // next piece (not copied in yet) or to no sequence at all (after the last one); the
+    // kernel masks those tokens but needs finite values there, so they start as zeros.
     if (cu_seqlens) {
         const int64_t rows = B * T;
-        for (int i = 0; i + 1 < np; ++i) {
+        for (int i = 0; i < np; ++i) {
             const int64_t r0 = pcs[i].tok0 + pcs[i].toks;
             const int64_t nr = (rows - r0 < kda::kHead / 2) ? rows - r0 : kda::kHead / 2;
             if (nr <= 0) continue;
@@ -520,7 +529,9 @@ extern "C" int kda_fwd_host(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16
         if (!copy(dinit, initial_state, s.init, cudaMemcpyHostToDevice, st)) return KDA_ERR_CUDA;
         rc = kda_fwd(nullptr, nullptr, nullptr, nullptr, nullptr, scale, nullptr, nullptr,
                      lower_bound, initial_state ? dinit : nullptr, initial_state_dtype,
-                     reinterpret_cast<float *>(dfin), nullptr, 0, nullptr, B, 0, H, K, V, stream);
+                     reinterpret_cast<float *>(dfin),
+                     cu_seqlens ? reinterpret_cast<const int64_t *>(dcu) : nullptr,
+                     cu_seqlens ? num_seqs : 0, nullptr, B, T, H, K, V, stream);
         if (rc != KDA_OK) return rc;
         launches = g_last_launches;
         if (!copy(final_state, dfin, s.fin, cudaMemcpyDeviceToHost, st)) return KDA_ERR_CUDA;

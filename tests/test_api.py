@@ -216,3 +216,22 @@ def test_checks_level_and_message(L):
         kda.kda_set_checks(old)
     assert kda.kda_set_checks(old) == old
     assert "cu_seqlens" in kda.kda_strerror(-14)
+
+
+def test_host_entry_checks_host_offsets_before_copying(L):
+    """kda_fwd_host reads cu_seqlens on the host (it plans the copies from it), so bad
+    offsets are refused with KDA_ERR_SEQLENS before any device work."""
+    import numpy as np
+    T, H = 100, 2
+    hb = lambda *shape: np.zeros(shape, np.uint16)
+    q, k, v, g = (hb(1, T, H, 128) for _ in range(4))
+    beta = hb(1, T, H)
+    A_log, dt = np.zeros(H, np.float32), np.zeros((H, 128), np.float32)
+    out = hb(1, T, H, 128)
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    for bad in ([0, 60, 50, 100], [0, 40, 101], [-1, 50, 100]):
+        cu = np.asarray(bad, np.int64)
+        rc = L.kda_fwd_host(p(q), p(k), p(v), p(g), p(beta), ctypes.c_float(0.1), p(A_log), p(dt),
+                            ctypes.c_float(-5.0), None, 0, None, p(cu), len(bad) - 1, p(out), 1, T,
+                            H, 128, 128, ctypes.c_void_p(A16), 1 << 30, None)
+        assert rc == -14, bad
