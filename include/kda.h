@@ -221,6 +221,40 @@ int kda_bwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_b
             kda_stream_t stream);
 
 /*
+ * kda_bwd_noalloc -- kda_bwd for callers that cannot allocate device memory: code
+ * running inside a memory pool or allocator that must not be re-entered, a plugin
+ * that is handed tensors but no allocator, or a process whose device memory budget
+ * is fixed before the first call.  The FlashKDA pages have no counterpart of it; it
+ * is a deployment convenience of this library.
+ *
+ * Arguments, results and return codes are those of kda_bwd without the workspace
+ * pair.  The workspace is instead a fixed array in the library's own device memory,
+ * KDA_BWD_NOALLOC_MAX_BYTES (64 MiB) long, which every GPU that loads the library
+ * holds until the process exits.  The call allocates nothing (no cudaMalloc, no
+ * cudaMallocAsync, no library allocator) and frees nothing.
+ *   - A call whose workspace need (kda_bwd_workspace_size of the same shape) exceeds
+ *     KDA_BWD_NOALLOC_MAX_BYTES returns KDA_ERR_WORKSPACE and launches nothing.
+ *   - The first call on a device looks up the array's device address there (once
+ *     per device, with that device current); make that first call before any stream
+ *     capture.
+ *   - All calls share the one array, and its contents persist from call to call
+ *     (the kernels write every part they read, so no clearing is needed).  Calls
+ *     whose work overlaps on the GPU (other streams, other host threads) race on
+ *     it: serialise them.
+ *   - The optional device check of cu_seqlens (kda_set_checks) is not run here, as
+ *     its result would need device memory; cu_seqlens is trusted as in kda_bwd with
+ *     the checks off.
+ */
+#define KDA_BWD_NOALLOC_MAX_BYTES ((size_t)64 << 20)
+int kda_bwd_noalloc(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
+                    const kda_bf16 *beta, float scale, const float *A_log, const float *dt_bias,
+                    float lower_bound, const void *initial_state, int initial_state_dtype,
+                    const kda_bf16 *d_out, const float *d_final_state, const int64_t *cu_seqlens,
+                    int64_t num_seqs, float *dq, float *dk, float *dv, float *dg, float *dbeta,
+                    float *dA_log, float *ddt_bias, float *d_initial_state, int64_t B, int64_t T,
+                    int64_t H, int64_t K, int64_t V, kda_stream_t stream);
+
+/*
  * kda_set_checks -- debug checks of device-resident arguments, process-wide; returns
  * the previous level.  0 (default): none; the kernels trust cu_seqlens.  1: every call
  * with cu_seqlens (kda_fwd, kda_fwd_ex, kda_bwd) first checks on the device, on its

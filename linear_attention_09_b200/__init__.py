@@ -5,7 +5,8 @@ Argument marshalling only: every step of the pass runs in the CUDA kernels of
 PyTorch fallback: if the library cannot be loaded, the calls raise.
 
 The functions mirror the C ABI in ``include/kda.h``:
-  kda_fwd, kda_fwd_ex, kda_decode, kda_bwd, kda_bwd_workspace_size, kda_fwd_host,
+  kda_fwd, kda_fwd_ex, kda_decode, kda_bwd, kda_bwd_noalloc, kda_bwd_workspace_size,
+  kda_fwd_host,
   kda_fwd_host_workspace_size, kda_set_checks, kda_strerror, kda_last_launch_count,
   kda_device_status.
 """
@@ -64,6 +65,9 @@ def lib() -> ctypes.CDLL:
             L.kda_bwd.argtypes = [P, P, P, P, P, F, P, P, F, P, I, P, P, P, I64, P, P, P, P, P,
                                   P, P, P, P, SZ, I64, I64, I64, I64, I64, P]
             L.kda_bwd.restype = I
+            L.kda_bwd_noalloc.argtypes = [P, P, P, P, P, F, P, P, F, P, I, P, P, P, I64, P, P, P,
+                                          P, P, P, P, P, I64, I64, I64, I64, I64, P]
+            L.kda_bwd_noalloc.restype = I
             L.kda_bwd_workspace_size.argtypes = [I64, I64, I64, I64, I64, I64]
             L.kda_bwd_workspace_size.restype = SZ
             L.kda_set_checks.argtypes = [I]
@@ -318,6 +322,58 @@ def kda_bwd(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, d_out, initial
     if rc != 0:
         raise KDAError(rc, "kda_bwd")
     return g_
+
+
+KDA_BWD_NOALLOC_MAX_BYTES = 64 << 20
+
+
+def kda_bwd_noalloc(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, d_out,
+                    initial_state=None, d_final_state=None, cu_seqlens=None,
+                    want_d_initial_state=True, grads=None, stream=None):
+    """``kda_bwd`` through the entry point that allocates no device memory: its
+    workspace is the library's own fixed 64 MiB device array (shapes that need more
+    are rejected with KDA_ERR_WORKSPACE).  For callers that cannot allocate, pass
+    ``grads``, a dict of preallocated fp32 outputs with the keys and shapes ``kda_bwd``
+    returns; otherwise they are allocated here.  Calls that overlap on the GPU share
+    the array and race."""
+    if d_out is None:
+        raise ValueError("d_out is required")
+    gr = grads or {}
+    if grads is not None and any(grads.get(n) is None for n in
+                                 ("dq", "dk", "dv", "dg", "dbeta", "dA_log", "ddt_bias")):
+        raise ValueError("grads must hold dq, dk, dv, dg, dbeta, dA_log and ddt_bias")
+    shp = lambda *ks: (lambda d: tuple(d[x] for x in ks))
+    B, T, H, K, V, N = _check_call(
+        q, k, v, g, beta, A_log, dt_bias, initial_state, cu_seqlens,
+        extra=[(d_out, "d_out", _BF16, shp("B", "T", "H", "V")),
+               (d_final_state, "d_final_state", _F32, shp("N", "H", "K", "V")),
+               (gr.get("dq"), "dq", _F32, shp("B", "T", "H", "K")),
+               (gr.get("dk"), "dk", _F32, shp("B", "T", "H", "K")),
+               (gr.get("dv"), "dv", _F32, shp("B", "T", "H", "V")),
+               (gr.get("dg"), "dg", _F32, shp("B", "T", "H", "K")),
+               (gr.get("dbeta"), "dbeta", _F32, shp("B", "T", "H")),
+               (gr.get("dA_log"), "dA_log", _F32, shp("H")),
+               (gr.get("ddt_bias"), "ddt_bias", _F32, shp("H", "K")),
+               (gr.get("dS0"), "dS0", _F32, shp("N", "H", "K", "V"))])
+    num_seqs = 0 if cu_seqlens is None else N
+    if grads is None:
+        f32 = dict(dtype=torch.float32, device=q.device)
+        grads = dict(dq=torch.empty((B, T, H, K), **f32), dk=torch.empty((B, T, H, K), **f32),
+                     dv=torch.empty((B, T, H, V), **f32), dg=torch.empty((B, T, H, K), **f32),
+                     dbeta=torch.empty((B, T, H), **f32), dA_log=torch.empty((H,), **f32),
+                     ddt_bias=torch.empty((H, K), **f32),
+                     dS0=torch.empty((N, H, K, V), **f32) if want_d_initial_state else None)
+    rc = lib().kda_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                               _ptr(A_log), _ptr(dt_bias), float(lower_bound), _ptr(initial_state),
+                               _state_dtype(initial_state), _ptr(d_out), _ptr(d_final_state),
+                               _ptr(cu_seqlens), num_seqs, _ptr(grads["dq"]), _ptr(grads["dk"]),
+                               _ptr(grads["dv"]), _ptr(grads["dg"]), _ptr(grads["dbeta"]),
+                               _ptr(grads["dA_log"]), _ptr(grads["ddt_bias"]),
+                               _ptr(grads.get("dS0")), B, T, H, K, V,
+                               _stream_handle(stream, q.device))
+    if rc != 0:
+        raise KDAError(rc, "kda_bwd_noalloc")
+    return grads
 
 
 def kda_fwd_raw(*args) -> int:

@@ -127,6 +127,21 @@ size_t host_total(const HostSizes &s)
 
 }  // namespace
 
+// The validation and device check above, for the other host files of the library.
+namespace kda {
+int validate_args(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                  float scale, const float *A_log, const float *dt_bias, float lower_bound,
+                  const void *init, int init_dtype, const void *final_state, const int64_t *cu,
+                  int64_t num_seqs, const void *out, int64_t B, int64_t T, int64_t H, int64_t K,
+                  int64_t V, int64_t *N_out)
+{
+    return validate(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, init, init_dtype,
+                    final_state, cu, num_seqs, out, B, T, H, K, V, N_out);
+}
+
+int device_supported() { return check_device(); }
+}  // namespace kda
+
 extern "C" const char *kda_strerror(int code)
 {
     switch (code) {

@@ -78,6 +78,16 @@ inline bool set_smem_limit_once(Kernel kernel, int bytes, int (&done)[64])
     return true;
 }
 
+// Host-side argument validation of the forward/backward calls (KDA_OK or a negative
+// code; *N_out = number of sequences) and the sm_100 device check, shared by the
+// entry points of the library's host files.
+int validate_args(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                  float scale, const float *A_log, const float *dt_bias, float lower_bound,
+                  const void *init, int init_dtype, const void *final_state, const int64_t *cu,
+                  int64_t num_seqs, const void *out, int64_t B, int64_t T, int64_t H, int64_t K,
+                  int64_t V, int64_t *N_out);
+int device_supported();
+
 // Kernel launcher; returns the number of kernels it enqueued (>= 0) or a negative
 // KDA_ERR_* code.
 int launch_chunked(const FwdParams &p, cudaStream_t stream);

@@ -61,6 +61,8 @@ def test_ex_decode_and_backward_reject_bad_tensors():
                        torch.zeros(H, K), -5.0, torch.zeros(4, H, K, K, dtype=torch.float64))
     with pytest.raises(TypeError, match="d_out has dtype"):
         kda.kda_bwd(**args(), d_out=torch.zeros(B, T, H, K))
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        kda.kda_bwd_noalloc(**args(), d_out=torch.zeros(B, T, H, K, dtype=torch.bfloat16))
 
 
 def test_host_entry_point_wants_contiguous_host_tensors():
