@@ -291,8 +291,6 @@ def run_reference(args, world, rank):
             "e2e": {"value": base["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}), flush=True)
         return 0
-    for _ in range(args.warmup):
-        pass  # the oracle has no warm-up state; steps below are timed one by one
     times = []
     base = None
     for _ in range(max(1, min(args.steps, 3))):

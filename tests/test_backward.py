@@ -2,8 +2,10 @@
 
 Every gradient the call returns is compared element by element with the oracle on
 the same seeded bf16 inputs, random bf16 dL/dout and (optionally) fp32 dL/dS_final.
-Bars (derived in the design doc from the fp32 arithmetic of the token recurrence): per
-gradient tensor rel-L2 <= 1e-3 and max-abs <= 1e-2 of the tensor's largest entry.
+Bars: per gradient tensor rel-L2 <= 1e-3 and max-abs <= 1e-2 of the tensor's largest
+entry.  They follow from the kernel's arithmetic: fp32 sums of at most 128 terms per
+token and a reverse recurrence whose factors alpha are <= 1, so the expected error is
+about 1e-6 relative; the bars leave three orders of magnitude of margin.
 
 The gate clamp lam = max(lb, z) is a kink: where z = -exp(A_log) softplus(x) sits
 within 5e-5 of lb (fp32 evaluates z to within ~3e-6), the kernel (fp32) and the oracle
