@@ -495,6 +495,58 @@ def run_config_bench(args, world, rank, local):
     return 0
 
 
+def strong_scaling(args, world, rank, device):
+    """One fixed global batch (the headline shape) split across the ranks by heads
+    (``partition.plan_heads``): each rank runs kda_fwd on its heads, then the outputs are
+    all-gathered (NCCL) so that every rank holds the global out.  Device time, max over
+    ranks, both without and with the gather (tensor-parallel attention keeps the output
+    head-sharded, so the first is the operator's own cost)."""
+    import torch.distributed as dist
+    import linear_attention_09_b200 as kda
+    from linear_attention_09_b200 import partition
+    w = WORKLOAD
+    B, T, H = w["B"], w["T"], w["H"]
+    plan = partition.plan_heads(H, world)[rank]
+    Hr = plan.heads[1] - plan.heads[0]
+    saved = WORKLOAD["H"]
+    WORKLOAD["H"] = Hr
+    try:
+        inp = device_inputs(args.seed + 7 * rank, device)  # this rank's heads of the batch
+    finally:
+        WORKLOAD["H"] = saved
+    out = torch.empty((B, T, Hr, w["V"]), dtype=torch.bfloat16, device=device)
+    fin = torch.empty((B, Hr, w["K"], w["V"]), dtype=torch.float32, device=device)
+    Hmax = max(p.heads[1] - p.heads[0] for p in partition.plan_heads(H, world))
+    send = torch.zeros((Hmax, B, T, w["V"]), dtype=torch.bfloat16, device=device)
+    recv = [torch.empty_like(send) for _ in range(world)]
+    stream = torch.cuda.current_stream(device)
+
+    def step(gather):
+        kda.kda_fwd(**inp, out=out, final_state=fin, stream=stream)
+        if gather:
+            send[:Hr].copy_(out.permute(2, 0, 1, 3))
+            dist.all_gather(recv, send)
+
+    res = {}
+    for gather in (False, True):
+        for _ in range(args.warmup):
+            step(gather)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            step(gather)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+        res["with_gather" if gather else "kernel"] = {"ms_per_step": ms,
+                                                       "value": B * T / (ms / 1e3)}
+    return {"scaling": "strong", "plan": "heads", "global_batch": B, "seq_len": T, "heads": H,
+            "unit": UNIT, "value": res["kernel"]["value"], "ms_per_step": res["kernel"]["ms_per_step"],
+            "with_all_gather": res["with_gather"]}
+
+
 def main():
     args = parse()
     world, rank, local = dist_setup(args.gpus)
@@ -588,6 +640,8 @@ def main():
     d2h = out_h.numel() * 2 + fin_h.numel() * 4
     del ws
 
+    strong = strong_scaling(args, world, rank, device) if world > 1 else None
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline()
@@ -612,6 +666,8 @@ def main():
             "gpu_launches": launches_per_step * args.steps,
             "cpu_baseline": cpu,
         }
+        if strong is not None:
+            line["strong"] = strong
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -268,26 +268,5 @@ namespace sm100 {
 // slower).
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return make_float2(a.x * b.x, a.y * b.y); }
 
-// fp32 -> tf32 (round to nearest, ties away), as a 32-bit pattern.
-__device__ __forceinline__ uint32_t cvt_tf32(float x)
-{
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return r;
-}
-
-// Warp-level D (16x8 fp32) += A (16x8 tf32, row) * B (8x8 tf32, col).
-// Fragments: g = lane / 4, t = lane % 4; a = {(g,t), (g+8,t), (g,t+4), (g+8,t+4)},
-// b = {(k=t, n=g), (k=t+4, n=g)}, d = {(g,2t), (g,2t+1), (g+8,2t), (g+8,2t+1)}.
-__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], const uint32_t (&a)[4],
-                                                const uint32_t (&b)[2])
-{
-    asm volatile(
-        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-
 }  // namespace sm100
 }  // namespace kda

@@ -79,3 +79,65 @@ def test_reference_arm_on_a_parity_workload():
     assert d["impl"] == "reference" and "tiny_B1_T512_H4" in d["metric"]
     assert d["value"] > 0 and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _strong_main(rank, world, port, outdir):
+    """bench.strong_scaling over gloo on the CPU, with the kernel and the CUDA timing
+    calls replaced by host stand-ins (the collective and the head plan are the real ones)."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      LOCAL_RANK=str(rank), WORLD_SIZE=str(world))
+    sys.path.insert(0, ROOT)
+    import time
+    import types
+
+    import torch
+    import bench
+    import linear_attention_09_b200 as kda
+    import torch.distributed as dist
+
+    class Ev:
+        def __init__(self, **_):
+            self.t = 0.0
+
+        def record(self, *_):
+            self.t = time.perf_counter()
+
+        def elapsed_time(self, other):
+            return (other.t - self.t) * 1e3
+
+    calls = []
+
+    def fake_fwd(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, out=None,
+                 final_state=None, stream=None, **_):
+        calls.append(q.shape)
+        out.fill_(float(rank + 1))
+        final_state.zero_()
+        return out, final_state
+
+    torch.cuda.Event = Ev
+    torch.cuda.synchronize = lambda *a, **k: None
+    torch.cuda.current_stream = lambda *a, **k: None
+    kda.kda_fwd = fake_fwd
+    w, r, _ = bench.dist_setup(world)
+    bench.WORKLOAD.update(B=1, T=64, H=5)
+    args = types.SimpleNamespace(seed=3, warmup=1, steps=2)
+    res = bench.strong_scaling(args, w, r, torch.device("cpu"))
+    with open(os.path.join(outdir, f"s{rank}.txt"), "w") as f:
+        f.write(repr((res["heads"], res["global_batch"], res["value"] > 0,
+                      res["with_all_gather"]["value"] > 0, sorted(set(tuple(c) for c in calls)))))
+    dist.destroy_process_group()
+
+
+def test_strong_scaling_line_two_gloo_ranks(tmp_path):
+    ctx = mp.get_context("spawn")
+    port = free_port()
+    procs = [ctx.Process(target=_strong_main, args=(r, 2, port, str(tmp_path))) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+        assert p.exitcode == 0
+    got = [eval((tmp_path / f"s{r}.txt").read_text()) for r in range(2)]
+    # H = 5 over two ranks: heads 0..2 and 3..4; every step ran the forward on its heads
+    assert got[0][0] == 5 and got[0][2] and got[0][3]
+    assert got[0][4] == [(1, 64, 3, 128)] and got[1][4] == [(1, 64, 2, 128)]
