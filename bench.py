@@ -466,6 +466,7 @@ def run_config_bench(args, world, rank, local):
     step = lambda: kda.kda_fwd(**call, out=out, final_state=fin, stream=stream)
     for _ in range(args.warmup):
         step()
+    launches = kda.kda_last_launch_count()
     torch.cuda.synchronize()
     barrier(world)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -491,7 +492,7 @@ def run_config_bench(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
                          "alg_bytes_per_launch": bytes_launch, "kernel": KERNEL},
-            "clocks": clk.summary(), "gpu_launches": args.steps}), flush=True)
+            "clocks": clk.summary(), "gpu_launches": launches * args.steps}), flush=True)
     return 0
 
 

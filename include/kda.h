@@ -74,6 +74,7 @@ typedef struct CUstream_st *kda_stream_t;
                                      always checked by kda_fwd_host (host offsets), by the
                                      device entry points with checks on (kda_set_checks);
                                      nothing was run */
+#define KDA_ERR_ARG (-15)         /* an argument outside its documented range */
 
 /* State layouts (kda_fwd_ex).  The FLA call on the pages passes
  * transpose_state_layout=True, i.e. per (sequence, head) the state stored value-major. */
@@ -94,8 +95,9 @@ typedef struct CUstream_st *kda_stream_t;
  *   no output; tokens outside [cu_seqlens[0], cu_seqlens[num_seqs]) are not
  *   written.
  * The kernel reads q, k, v, g, beta in tiles of 64 tokens, so the last tile of a
- *   sequence also reads up to 63 rows after it; those tokens are masked, but the
- *   rows must hold finite values (rows past the end of the tensors read as zero).
+ *   sequence also reads up to 63 rows after it (the next sequence's, or rows that
+ *   belong to no sequence).  Those rows are cleared on chip before any use, so
+ *   their bits (NaN and Inf included) never reach a result.
  * stream: the work is enqueued on it; the call does not synchronise.
  * T == 0 is valid: only final_state is written.
  * Returns KDA_OK or a negative code (see above).  Never traps the GPU.
@@ -178,6 +180,26 @@ int kda_decode(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kd
                const kda_bf16 *beta, float scale, const float *A_log, const float *dt_bias,
                float lower_bound, const float *state_in, float *state_out, kda_bf16 *out,
                int64_t N, int64_t H, int64_t K, int64_t V, kda_stream_t stream);
+
+/*
+ * kda_decode_ex -- kda_decode with the state variants of kda_fwd_ex, so that a prefill
+ * in either layout or element type hands its final state straight to decode (initial
+ * and final states bf16 or fp32: FlashKDA de código abierto de Moonshot AI,
+ * 7minutos.es, "Debajo del capó"; the transposed layout is the chunk_kda call's
+ * transpose_state_layout on github.zuobiaodaohang.com, "作为 FLA 后端的用法").
+ *
+ * state_in_dtype / state_out_dtype: KDA_STATE_F32 or KDA_STATE_BF16 (a bf16 state is
+ *   promoted exactly; a bf16 result is the fp32 state rounded to nearest even).
+ * state_layout: KDA_LAYOUT_KV ([N,H,K,V], S[k][v]) or KDA_LAYOUT_VK ([N,H,V,K]).
+ * state_out may equal state_in (update in place) only when the two dtypes are equal,
+ *   else KDA_ERR_STATE_DTYPE.  Everything else as kda_decode; kda_decode(...) ==
+ *   kda_decode_ex(..., KDA_STATE_F32, ..., KDA_STATE_F32, KDA_LAYOUT_KV, ...).
+ */
+int kda_decode_ex(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, const kda_bf16 *g,
+                  const kda_bf16 *beta, float scale, const float *A_log, const float *dt_bias,
+                  float lower_bound, const void *state_in, int state_in_dtype, void *state_out,
+                  int state_out_dtype, int state_layout, kda_bf16 *out, int64_t N, int64_t H,
+                  int64_t K, int64_t V, kda_stream_t stream);
 
 /*
  * kda_bwd -- backward pass of kda_fwd: the gradients of
@@ -276,6 +298,15 @@ int kda_last_launch_count(void);
  * gave up (0 = none; the kernel then skipped the rest of its work and returned
  * without trapping).  Synchronous (reads device memory); reset != 0 clears it. */
 int kda_device_status(int reset);
+
+/* Testing hook for the failure path (no counterpart on the pages): the next forward
+ * launch (kda_fwd, kda_fwd_ex, kda_fwd_host) starts as if one of its CTAs had
+ * already given up a bounded wait with `code` (1..255).  Every CTA of that launch
+ * then returns at its start without writing out or the final state, exactly as
+ * the CTAs that start after a real failure do, and kda_device_status reports
+ * `code`.  Process-wide, consumed by the next launch; code 0 cancels a pending
+ * one.  KDA_OK, or KDA_ERR_ARG for a code outside 0..255. */
+int kda_inject_error(int code);
 
 #ifdef __cplusplus
 }

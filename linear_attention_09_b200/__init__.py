@@ -5,10 +5,11 @@ Argument marshalling only: every step of the pass runs in the CUDA kernels of
 PyTorch fallback: if the library cannot be loaded, the calls raise.
 
 The functions mirror the C ABI in ``include/kda.h``:
-  kda_fwd, kda_fwd_ex, kda_decode, kda_bwd, kda_bwd_noalloc, kda_bwd_workspace_size,
+  kda_fwd, kda_fwd_ex, kda_decode, kda_decode_ex, kda_bwd, kda_bwd_noalloc,
+  kda_bwd_workspace_size,
   kda_fwd_host,
   kda_fwd_host_workspace_size, kda_set_checks, kda_strerror, kda_last_launch_count,
-  kda_device_status.
+  kda_device_status, kda_inject_error.
 """
 from __future__ import annotations
 
@@ -57,6 +58,9 @@ def lib() -> ctypes.CDLL:
             L.kda_fwd_ex.restype = I
             L.kda_decode.argtypes = [P, P, P, P, P, F, P, P, F, P, P, P, I64, I64, I64, I64, P]
             L.kda_decode.restype = I
+            L.kda_decode_ex.argtypes = [P, P, P, P, P, F, P, P, F, P, I, P, I, I, P, I64, I64, I64,
+                                        I64, P]
+            L.kda_decode_ex.restype = I
             L.kda_fwd_host.argtypes = [P, P, P, P, P, F, P, P, F, P, I, P, P, I64, P, I64, I64,
                                        I64, I64, I64, P, SZ, P]
             L.kda_fwd_host.restype = I
@@ -78,6 +82,8 @@ def lib() -> ctypes.CDLL:
             L.kda_last_launch_count.restype = I
             L.kda_device_status.argtypes = [I]
             L.kda_device_status.restype = I
+            L.kda_inject_error.argtypes = [I]
+            L.kda_inject_error.restype = I
             _lib = L
     return _lib
 
@@ -99,6 +105,15 @@ def kda_last_launch_count() -> int:
 def kda_device_status(reset: bool = False) -> int:
     """Error word of the last kernels (0 = every bounded wait completed)."""
     return int(lib().kda_device_status(int(bool(reset))))
+
+
+def kda_inject_error(code: int) -> None:
+    """Testing hook: the next forward launch starts as if one of its CTAs had given up
+    with ``code`` (1..255); its CTAs return at once and kda_device_status reports it.
+    Code 0 cancels a pending injection."""
+    rc = lib().kda_inject_error(int(code))
+    if rc != 0:
+        raise KDAError(rc, "kda_inject_error")
 
 
 def kda_fwd_host_workspace_size(B, T, H, K=HEAD, V=HEAD, num_seqs=0,
@@ -275,6 +290,41 @@ def kda_decode(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, state, stat
                           _ptr(state_out), _ptr(out), N, H, K, V, _stream_handle(stream, q.device))
     if rc != 0:
         raise KDAError(rc, "kda_decode")
+    return out, state_out
+
+
+def kda_decode_ex(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, state, state_out=None,
+                  out=None, state_layout="kv", state_out_dtype=None, stream=None):
+    """``kda_decode`` with the state variants of ``kda_fwd_ex``: ``state`` fp32 or bf16 in
+    the "kv" (S[k][v], [N,H,K,V]) or "vk" (S[v][k], [N,H,V,K]) layout; the new state goes
+    to ``state_out`` (default: in place, which needs ``state_out_dtype`` equal to the
+    input's) with ``state_out_dtype`` (default: the input's, or that of a given
+    ``state_out``).  Returns (out [N,H,128] bf16, new state)."""
+    if not isinstance(q, torch.Tensor) or q.dim() != 3 or not isinstance(v, torch.Tensor) \
+            or v.dim() != 3:
+        raise ValueError("q and v must be 3-D tensors [N, H, K] / [N, H, V]")
+    N, H, K = q.shape
+    V = v.shape[2]
+    layout = _LAYOUTS.get(state_layout, -1) if isinstance(state_layout, str) else int(state_layout)
+    shp = (N, H, V, K) if layout == KDA_LAYOUT_VK else (N, H, K, V)
+    if state is None:
+        raise ValueError("state is required")
+    if state_out is None:
+        want = state.dtype if state_out_dtype is None else state_out_dtype
+        state_out = state if want == state.dtype else torch.empty(shp, dtype=want, device=q.device)
+    _check_all([(q, "q", _BF16, (N, H, K)), (k, "k", _BF16, (N, H, K)), (g, "g", _BF16, (N, H, K)),
+                (v, "v", _BF16, (N, H, V)), (beta, "beta", _BF16, (N, H)),
+                (A_log, "A_log", _F32, (H,)), (dt_bias, "dt_bias", _F32, (H, K)),
+                (state, "state", _STATE, shp), (state_out, "state_out", _STATE, shp),
+                (out, "out", _BF16, (N, H, V))], q.device)
+    if out is None:
+        out = torch.empty((N, H, V), dtype=torch.bfloat16, device=q.device)
+    rc = lib().kda_decode_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), float(scale),
+                             _ptr(A_log), _ptr(dt_bias), float(lower_bound), _ptr(state),
+                             _state_dtype(state), _ptr(state_out), _state_dtype(state_out), layout,
+                             _ptr(out), N, H, K, V, _stream_handle(stream, q.device))
+    if rc != 0:
+        raise KDAError(rc, "kda_decode_ex")
     return out, state_out
 
 

@@ -160,6 +160,7 @@ extern "C" const char *kda_strerror(int code)
     case KDA_ERR_SCALE: return "scale must be finite";
     case KDA_ERR_LAYOUT: return "state_layout must be KDA_LAYOUT_KV or KDA_LAYOUT_VK";
     case KDA_ERR_SEQLENS: return "cu_seqlens must be non-decreasing within [0, B*T] (device check)";
+    case KDA_ERR_ARG: return "argument outside its documented range";
     default: return "unknown kda error code";
     }
 }
@@ -174,6 +175,8 @@ extern "C" int kda_set_checks(int level)
 }
 
 extern "C" int kda_device_status(int reset) { return kda::chunked_device_error(reset != 0); }
+
+extern "C" int kda_inject_error(int code) { return kda::chunked_inject_error(code); }
 
 extern "C" int kda_fwd_ex(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v,
                           const kda_bf16 *g, const kda_bf16 *beta, float scale,
@@ -240,17 +243,23 @@ extern "C" int kda_fwd(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v, 
                       num_seqs, out, B, T, H, K, V, stream);
 }
 
-extern "C" int kda_decode(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v,
-                          const kda_bf16 *g, const kda_bf16 *beta, float scale,
-                          const float *A_log, const float *dt_bias, float lower_bound,
-                          const float *state_in, float *state_out, kda_bf16 *out, int64_t N,
-                          int64_t H, int64_t K, int64_t V, kda_stream_t stream)
+extern "C" int kda_decode_ex(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v,
+                             const kda_bf16 *g, const kda_bf16 *beta, float scale,
+                             const float *A_log, const float *dt_bias, float lower_bound,
+                             const void *state_in, int state_in_dtype, void *state_out,
+                             int state_out_dtype, int state_layout, kda_bf16 *out, int64_t N,
+                             int64_t H, int64_t K, int64_t V, kda_stream_t stream)
 {
     if (K != kda::kHead || V != kda::kHead) return KDA_ERR_HEAD_DIM;
     if (N < 0 || H < 1 || N > (int64_t(1) << 40) / H || N * H > (int64_t(1) << 31) - 1)
         return KDA_ERR_SHAPE;
     if (!(lower_bound >= -5.0f && lower_bound <= 0.0f)) return KDA_ERR_LOWER_BOUND;
     if (!std::isfinite(scale)) return KDA_ERR_SCALE;
+    if (state_layout != KDA_LAYOUT_KV && state_layout != KDA_LAYOUT_VK) return KDA_ERR_LAYOUT;
+    const auto dtype_ok = [](int d) { return d == KDA_STATE_F32 || d == KDA_STATE_BF16; };
+    if (!dtype_ok(state_in_dtype) || !dtype_ok(state_out_dtype)) return KDA_ERR_STATE_DTYPE;
+    // an update in place needs one element type
+    if (state_in == state_out && state_in_dtype != state_out_dtype) return KDA_ERR_STATE_DTYPE;
     if (N == 0) {
         g_last_launches = 0;
         return KDA_OK;
@@ -273,6 +282,9 @@ extern "C" int kda_decode(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *
     p.dt_bias = dt_bias;
     p.state_in = state_in;
     p.state_out = state_out;
+    p.in_dtype = state_in_dtype;
+    p.out_dtype = state_out_dtype;
+    p.state_layout = state_layout;
     p.out = reinterpret_cast<__nv_bfloat16 *>(out);
     p.scale = scale;
     p.lower_bound = lower_bound;
@@ -282,6 +294,17 @@ extern "C" int kda_decode(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *
     if (n < 0) return n;
     g_last_launches = n;
     return KDA_OK;
+}
+
+extern "C" int kda_decode(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v,
+                          const kda_bf16 *g, const kda_bf16 *beta, float scale,
+                          const float *A_log, const float *dt_bias, float lower_bound,
+                          const float *state_in, float *state_out, kda_bf16 *out, int64_t N,
+                          int64_t H, int64_t K, int64_t V, kda_stream_t stream)
+{
+    return kda_decode_ex(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, state_in,
+                         KDA_STATE_F32, state_out, KDA_STATE_F32, KDA_LAYOUT_KV, out, N, H, K, V,
+                         stream);
 }
 
 extern "C" size_t kda_bwd_workspace_size(int64_t B, int64_t T, int64_t H, int64_t K, int64_t V,
@@ -482,23 +505,6 @@ extern "C" int kda_fwd_host(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16
         return KDA_ERR_CUDA;
     Piece pcs[8];
     const int np = (B * T == 0) ? 0 : plan_pieces(B, T, cu_seqlens, num_seqs, pcs, 8);
-    // A varlen piece's last tile also reads up to 63 rows after it, which belong to the
-    // next piece (not copied in yet) or to no sequence at all (after the last one); the
-    // kernel masks those tokens but needs finite values there, so they start as zeros.
-    if (cu_seqlens) {
-        const int64_t rows = B * T;
-        for (int i = 0; i < np; ++i) {
-            const int64_t r0 = pcs[i].tok0 + pcs[i].toks;
-            const int64_t nr = (rows - r0 < kda::kHead / 2) ? rows - r0 : kda::kHead / 2;
-            if (nr <= 0) continue;
-            char *bases[4] = {dq, dk, dg, dv};
-            for (char *b : bases)
-                if (cudaMemsetAsync(b + (size_t)r0 * row, 0, (size_t)nr * row, st) != cudaSuccess)
-                    return KDA_ERR_CUDA;
-            if (cudaMemsetAsync(dbeta + (size_t)r0 * H * 2, 0, (size_t)nr * H * 2, st) != cudaSuccess)
-                return KDA_ERR_CUDA;
-        }
-    }
     int launches = 0;
     for (int i = 0; i < np; ++i) {
         const Piece &pc = pcs[i];

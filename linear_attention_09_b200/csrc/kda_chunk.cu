@@ -34,6 +34,7 @@
 // Orientation: the inter-chunk products are computed transposed (M = value
 // column v on the 128 TMEM lanes), so S^T and U^T are tensor-core A operands
 // read straight from TMEM, and thread v owns value column v.
+#include <atomic>
 #include <cuda.h>
 
 #include <type_traits>
@@ -44,7 +45,13 @@
 
 namespace kda {
 
-__device__ int g_chunk_error;  // set to a non-zero code when a bounded wait gives up
+// Error word: (launch epoch << 8) | code of the first bounded wait that gave up (0 = none).
+// A CTA that starts after another CTA of its launch gave up sees its own epoch there and
+// returns at once, so a failure that hits every CTA ends after one wave of them; a stale
+// word of an earlier launch carries another epoch and is ignored.
+__device__ int g_chunk_error;
+__shared__ uint32_t s_epoch;  // this launch's epoch (the high bits of its error word)
+__shared__ int s_abort;       // set by thread 0: this launch has already failed
 
 namespace {
 
@@ -179,10 +186,14 @@ struct Ctx {
     int nchunks;
 };
 
+// Bounded wait (about 1 s at 1965 MHz); one that gives up records (epoch << 8) | code
+// unless an earlier failure of the launch is already recorded.  The spin itself stays
+// minimal: extra work in this inlined loop, which sits at every hand-off, measurably
+// slowed the kernel.
 __device__ __forceinline__ bool wait_or_flag(uint64_t *bar, uint32_t parity, int code)
 {
-    if (mbar_wait(bar, parity)) return true;
-    atomicExch(&g_chunk_error, code);
+    if (mbar_wait(bar, parity, 2000000000LL)) return true;
+    atomicCAS(&g_chunk_error, 0, (int)(s_epoch << 8) | code);
     return false;
 }
 
@@ -256,10 +267,22 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
 
     // ---- norms (thread: token tid/4, 16-byte chunks 2 (tid%4), 2 (tid%4) + 1 of both
     //      64-channel boxes; each 8-lane phase then reads 8 distinct bank groups) and beta
-    //      of the chunk whose tiles are in shared memory, of length Lc, into buffer buf ----
+    //      of the chunk whose tiles are in shared memory, of length Lc, into buffer buf.
+    //      A partial chunk's tiles also hold the rows after the sequence (the next
+    //      sequence's tokens, or whatever follows the batch); those tokens must add
+    //      exactly zero whatever their bits (0 * NaN is NaN), so the threads that own
+    //      their q and k chunks here overwrite them with zeros before any other read. ----
     auto norms = [&](int Lc, int buf) {
         const float beta_c = __uint_as_float((uint32_t)beta_bits << 16);
         const int t = tid >> 2, qq = tid & 3;
+        if (t >= Lc) {  // a row after the sequence end: cleared, whatever its bits
+#pragma unroll
+            for (int ch = 0; ch < 4; ++ch) {
+                const uint32_t off = (uint32_t)(ch >> 1) * 8192u + sw(t, (2 * qq + (ch & 1)) * 16);
+                *reinterpret_cast<uint4 *>(sm + SM_Q + off) = make_uint4(0u, 0u, 0u, 0u);
+                *reinterpret_cast<uint4 *>(sm + SM_K + off) = make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
         float sq = 0.f, sk = 0.f;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -656,6 +679,19 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
                 *reinterpret_cast<uint4 *>(sm + SM_TLO + off) = make_uint4(plo[0], plo[1], plo[2], plo[3]);
             }
         }
+        // a partial chunk's v rows after the sequence are cleared before u = T v reads
+        // them (16-byte chunks, every in-chunk thread; the v tile arrived long before)
+        bool vok = true;
+        if (L < C) {
+            vok = wait_or_flag(&bars->v, par, 15);
+            if (vok) {
+                for (int e = tid; e < (C - L) * 16; e += NT_IN) {
+                    const int r = L + (e >> 4);
+                    *reinterpret_cast<uint4 *>(sm + SM_V + (uint32_t)(e & 8) * 1024u + (uint32_t)(r * 128 + (e & 7) * 16)) =
+                        make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+        }
         // hand T to the issue warp (w^T = (k^ e^G)^T T^T, u^T = v^T (T_hi + T_lo)^T)
         fence_async_smem();
         tc_fence_before();
@@ -675,7 +711,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         {
             // (if the issue warp gave up, this bounded wait runs out)
             const bool mok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 3);
-            ok = named_bar_and(BAR_IN, NT_IN, sok && mok);
+            ok = named_bar_and(BAR_IN, NT_IN, sok && mok && vok);
         }
         tc_fence_after();
         if (!ok) break;
@@ -1024,6 +1060,9 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
     cx.nchunks = (int)((cx.len + C - 1) / C);
 
     if (tid == 0) {
+        s_epoch = p.epoch;
+        const int e = *reinterpret_cast<volatile int *>(&g_chunk_error);
+        s_abort = e != 0 && ((uint32_t)e >> 8) == p.epoch;
         Bars *b = cx.bars;
         mbar_init(&b->qkg[0], 1);
         mbar_init(&b->qkg[1], 1);
@@ -1047,6 +1086,10 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
     __syncthreads();
     tc_fence_after();
     cx.tb = *tbase_s;
+    if (s_abort) {  // another CTA of this launch gave up before this one started
+        if (warp == 0) tmem_dealloc(cx.tb, 512);
+        return;
+    }
     if (tid == 0 && cx.nchunks > 0) {  // first chunk's tiles
         load_qkg_box(sm, tm, &cx.bars->qkg[0], cx.h, cx.tok0, 0);
         load_qkg_box(sm, tm, &cx.bars->qkg[1], cx.h, cx.tok0, 1);
@@ -1062,6 +1105,9 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
     __syncthreads();
     if (warp == 0) tmem_dealloc(cx.tb, 512);
 }
+
+// Error code the next launch starts with (0 = none); see chunked_inject_error.
+std::atomic<int> g_inject{0};
 
 // Driver entry point for cuTensorMapEncodeTiled, resolved once through the runtime.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -1111,8 +1157,26 @@ int launch_chunked(const FwdParams &p, cudaStream_t stream)
     }
     static int attr_set[64];
     if (!set_smem_limit_once(chunk_kernel, SMEM_ALLOC, attr_set)) return KDA_ERR_CUDA;
-    chunk_kernel<<<(unsigned)ctas, NT, SMEM_ALLOC, stream>>>(p, tm);
+    // the launch's epoch: 24 bits, never 0 (an error word of 0 means no error)
+    static std::atomic<uint32_t> epochs{0};
+    FwdParams pe = p;
+    pe.epoch = (epochs.fetch_add(1u) % 0xFFFFFFu) + 1u;
+    const int inject = g_inject.exchange(0);
+    if (inject) {  // the launch starts as if one of its CTAs had given up with this code
+        const int word = (int)(pe.epoch << 8) | inject;
+        if (cudaMemcpyToSymbolAsync(g_chunk_error, &word, sizeof(int), 0, cudaMemcpyHostToDevice,
+                                    stream) != cudaSuccess)
+            return KDA_ERR_CUDA;
+    }
+    chunk_kernel<<<(unsigned)ctas, NT, SMEM_ALLOC, stream>>>(pe, tm);
     return cudaGetLastError() == cudaSuccess ? 1 : KDA_ERR_CUDA;
+}
+
+int chunked_inject_error(int code)
+{
+    if (code < 0 || code > 255) return KDA_ERR_ARG;  // 0 cancels a pending injection
+    g_inject.store(code);
+    return KDA_OK;
 }
 
 int chunked_device_error(bool reset)
@@ -1123,7 +1187,7 @@ int chunked_device_error(bool reset)
         const int z = 0;
         cudaMemcpyToSymbol(g_chunk_error, &z, sizeof(int));
     }
-    return v;
+    return v & 0xFF;  // the code of the wait that gave up
 }
 
 }  // namespace kda

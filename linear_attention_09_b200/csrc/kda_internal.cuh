@@ -21,14 +21,17 @@ struct FwdParams {
     __nv_bfloat16 *out;
     float scale, lower_bound;
     int64_t B, T, H, N;      // N = number of sequences
+    uint32_t epoch;          // set by the launcher: tags the launch's error word
 };
 
 // One decode step: one token per (sequence, head), state updated in HBM.
 struct DecodeParams {
     const __nv_bfloat16 *q, *k, *v, *g, *beta;  // [N,H,K], [N,H,K], [N,H,V], [N,H,K], [N,H]
     const float *A_log, *dt_bias;
-    const float *state_in;   // fp32 [N,H,K,V] (S[k][v])
-    float *state_out;        // fp32 [N,H,K,V]; may equal state_in
+    const void *state_in;    // [N,H,K,V] (S[k][v]) or [N,H,V,K] (S[v][k]), fp32 or bf16
+    void *state_out;         // same layout, fp32 or bf16; may equal state_in (same dtype)
+    int in_dtype, out_dtype; // KDA_STATE_F32 / KDA_STATE_BF16
+    int state_layout;        // KDA_LAYOUT_KV / KDA_LAYOUT_VK
     __nv_bfloat16 *out;      // [N,H,V]
     float scale, lower_bound;
     int64_t N, H;
@@ -93,5 +96,6 @@ int device_supported();
 int launch_chunked(const FwdParams &p, cudaStream_t stream);
 // Error word the chunked kernel sets when a bounded wait gives up (0 = none).
 int chunked_device_error(bool reset);
+int chunked_inject_error(int code);  // the next launch starts failed with `code`
 
 }  // namespace kda

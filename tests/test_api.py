@@ -156,6 +156,36 @@ def test_decode_empty_and_valid_without_device(L):
         assert call_decode() == -11
 
 
+def call_decode_ex(**over):
+    a = dict(q=A16, k=A16 + 0x100, v=A16 + 0x200, g=A16 + 0x300, beta=A16 + 0x400, scale=0.1,
+             A_log=A16 + 0x500, dt_bias=A16 + 0x600, lb=-5.0, sin=A16 + 0x800, sind=1,
+             sout=A16 + 0x900, soutd=2, layout=1, out=A16 + 0x700, N=4, H=2, K=128, V=128,
+             stream=None)
+    a.update(over)
+    return int(kda.lib().kda_decode_ex(a["q"], a["k"], a["v"], a["g"], a["beta"],
+                                       ctypes.c_float(a["scale"]), a["A_log"], a["dt_bias"],
+                                       ctypes.c_float(a["lb"]), a["sin"], a["sind"], a["sout"],
+                                       a["soutd"], a["layout"], a["out"], a["N"], a["H"], a["K"],
+                                       a["V"], a["stream"]))
+
+
+@pytest.mark.parametrize("over,code", [
+    (dict(layout=2), -13), (dict(sind=0), -6), (dict(soutd=3), -6),
+    (dict(sout=A16 + 0x800), -6),  # in place with two element types
+    (dict(K=64), -1), (dict(sin=None), -2), (dict(sout=A16 + 0x908), -7),
+])
+def test_decode_ex_invalid_arguments_rejected_on_host(L, over, code):
+    assert call_decode_ex(**over) == code
+
+
+def test_decode_ex_valid_without_device(L):
+    import torch
+    assert call_decode_ex(N=0, q=None) == 0
+    if not torch.cuda.is_available():
+        assert call_decode_ex() == -11
+        assert call_decode_ex(sout=A16 + 0x800, soutd=1) == -11  # in place, one dtype
+
+
 WS = 0x4000000  # fake 256-byte aligned workspace address
 
 

@@ -108,6 +108,94 @@ def test_varlen_edges(lengths):
             np.testing.assert_array_equal(fin_g[s], inp.initial_state[s].numpy())
 
 
+@pytest.mark.parametrize("fill", [0x7FC0, 0x7F80, 0xFF80, 0x7F7F])  # NaN, +Inf, -Inf, bf16 max
+def test_rows_after_the_last_sequence_do_not_matter(fill):
+    """A varlen batch may end before its buffer does (cu_seqlens[N] < rows).  The last
+    sequence's final 64-token tile then also covers rows that belong to no sequence.
+    Whatever those rows hold (here NaN, Inf or the largest bf16 in every input), every
+    result must be bit-identical to the run with zero rows there, and the rows
+    themselves must not be written."""
+    lengths, pad = [70, 33, 129], 40
+    inp = small(lengths=lengths, init="f32", seed=9)
+    rows = int(inp.cu_seqlens[-1])
+    d = dev(inp)
+
+    def padded(t, bits):
+        extra = torch.full((1, pad) + tuple(t.shape[2:]), bits, dtype=torch.int16,
+                           device=t.device).view(torch.bfloat16)
+        return torch.cat([t, extra], dim=1).contiguous()
+
+    runs = []
+    for bits in (0, fill - 0x10000 if fill >= 0x8000 else fill):
+        call = dict(d)
+        for name in ("q", "k", "v", "g", "beta"):
+            call[name] = padded(d[name], bits)
+        out = torch.full((1, rows + pad, inp.H, 128), 7.0, dtype=torch.bfloat16, device="cuda")
+        o, f = kda.kda_fwd(**call, out=out)
+        torch.cuda.synchronize()
+        assert kda.kda_device_status(reset=True) == 0
+        runs.append((o.cpu(), f.cpu()))
+    (o0, f0), (o1, f1) = runs
+    assert torch.equal(o0.view(torch.int16), o1.view(torch.int16))
+    assert torch.equal(f0, f1)
+    assert torch.all(o1[:, rows:] == 7.0), "rows outside every sequence were written"
+    out_r, fin_r = oracle.forward_inputs(inp)
+    assert_parity(inp, o1[:, :rows].float().numpy().astype(np.float64),
+                  f1.numpy().astype(np.float64), out_r, fin_r, what=f"pad fill {fill:#x}")
+
+
+
+@pytest.mark.parametrize("fill", [0x7FC0, 0xFF80])  # NaN, -Inf
+def test_a_sequence_ignores_the_bits_of_the_next_one(fill):
+    """Each sequence's last 64-token tile also covers the first rows of the sequence after
+    it.  With every input of sequence 1 set to NaN or -Inf, sequences 0 and 2 must give
+    bit-identical out and final states to the run where sequence 1 is clean."""
+    lengths = [70, 45, 100]
+    inp = small(lengths=lengths, init="f32", seed=21)
+    d = dev(inp)
+    t0, t1 = lengths[0], lengths[0] + lengths[1]
+    bad = dict(d)
+    bits = fill - 0x10000 if fill >= 0x8000 else fill
+    for name in ("q", "k", "v", "g", "beta"):
+        t = d[name].clone()
+        t.view(torch.int16)[:, t0:t1] = bits
+        bad[name] = t
+    runs = []
+    for call in (d, bad):
+        o, f = kda.kda_fwd(**call)
+        torch.cuda.synchronize()
+        assert kda.kda_device_status(reset=True) == 0
+        runs.append((o.cpu(), f.cpu()))
+    (o0, f0), (o1, f1) = runs
+    keep = torch.cat([torch.arange(0, t0), torch.arange(t1, sum(lengths))])
+    assert torch.equal(o0[:, keep].view(torch.int16), o1[:, keep].view(torch.int16))
+    assert torch.equal(f0[[0, 2]], f1[[0, 2]])
+
+
+def test_many_short_sequences_with_empty_ones():
+    """More (sequence, head) units than SMs, most of them a chunk or two long and a
+    quarter of them empty: the work is dealt to a persistent grid in decreasing length
+    (every unit is compared; empty sequences return their initial state)."""
+    rng = np.random.default_rng(77)
+    lengths = [int(x) if rng.random() > 0.25 else 0 for x in rng.integers(1, 150, size=400)]
+    inp = small(lengths=lengths, H=2, init="bf16", seed=78)
+    out_r, fin_r = oracle.forward_inputs(inp)
+    out_g, fin_g = run_gpu(inp)
+    assert_parity(inp, out_g, fin_g, out_r, fin_r, what="400 short sequences")
+    for s_, n in enumerate(lengths):
+        if n == 0:
+            np.testing.assert_array_equal(fin_g[s_], inp.initial_state[s_].float().numpy())
+
+
+def test_fixed_length_more_units_than_sms():
+    """B * H = 200 units of one length (> 148 SMs): a persistent grid takes two units on
+    some CTAs, chaining the second unit's start behind the first one's drain."""
+    w = ki.Workload("b5h40", B=5, T=130, H=40, init_state="f32", g_std=1.0)
+    inp = ki.make_inputs(w, 5)
+    out_r, fin_r = oracle.forward_inputs(inp)
+    out_g, fin_g = run_gpu(inp)
+    assert_parity(inp, out_g, fin_g, out_r, fin_r, what="B=5 H=40")
+
 def test_zero_tokens_returns_initial_state():
     inp = small(T=0, init="bf16")
     out_g, fin_g = run_gpu(inp)
@@ -165,9 +253,9 @@ def test_host_entry_point_matches_device_entry_point():
 # ---------------------------------------------------------------------------
 SAMPLES = {
     0: None,  # every pair
-    1: [(0, 0), (0, 7), (0, 13), (0, 31)],
-    2: "ends",  # shortest and longest sequences, several heads
-    3: [(0, 0), (1, 9), (2, 22), (3, 31)],
+    1: [(0, h) for h in range(32)],  # the one sequence, every head
+    2: "ends",  # every head of the longest sequence; shortest and median, several heads
+    3: [(b, h) for b in range(4) for h in range(b, 32, 4)],  # every entry x 8 heads (32 pairs)
     4: "ends",
 }
 
@@ -178,9 +266,10 @@ def test_workload_parity(cfg):
     pairs = SAMPLES[cfg]
     if pairs == "ends":
         lens = [n for (_, _, n) in inp.seq_bounds()]
-        order = np.argsort(lens)
-        seqs = [int(order[0]), int(order[1]), int(order[-1]), int(order[len(order) // 2])]
+        order = np.argsort(lens, kind="stable")
+        seqs = [int(order[0]), int(order[1]), int(order[len(order) // 2])]
         pairs = [(s, h) for i, s in enumerate(seqs) for h in (i % inp.H, (5 * i + 3) % inp.H)]
+        pairs += [(int(order[-1]), h) for h in range(inp.H)]
     mask = None if pairs is None else mask_for(inp, pairs)
     out_r, fin_r = oracle.forward_inputs(inp, mask=mask)
     out_g, fin_g = run_gpu(inp)
@@ -279,6 +368,54 @@ def test_decode_in_place_equals_out_of_place():
     a = run_decode(inp, in_place=True)
     b = run_decode(inp, in_place=False)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("layout,in_dt,out_dt", [("vk", torch.float32, torch.float32),
+                                                  ("kv", torch.bfloat16, torch.float32),
+                                                  ("vk", torch.bfloat16, torch.bfloat16)])
+def test_decode_state_variants(layout, in_dt, out_dt):
+    """kda_decode_ex on the state variants equals kda_decode on the fp32 S[k][v] copy of the
+    same state: bit for bit with fp32 in and out, the bf16 result being that fp32 state
+    rounded to nearest even."""
+    inp = decode_inputs(9, 4, seed=31)
+    d = dev(inp)
+    sq = lambda t: t[:, 0].contiguous()
+    args = (sq(d["q"]), sq(d["k"]), sq(d["v"]), sq(d["g"]), d["beta"][:, 0].contiguous(),
+            d["scale"], d["A_log"], d["dt_bias"], d["lower_bound"])
+    s_kv = d["initial_state"].to(in_dt).float()  # the values the variant call sees
+    o_ref, st_ref = kda.kda_decode(*args, s_kv.clone())
+    s_in = d["initial_state"].to(in_dt)
+    if layout == "vk":
+        s_in = s_in.transpose(-1, -2).contiguous()
+    o, st = kda.kda_decode_ex(*args, s_in, state_layout=layout, state_out_dtype=out_dt)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref)
+    st_kv = st.transpose(-1, -2) if layout == "vk" else st
+    assert torch.equal(st_kv, st_ref.to(out_dt))
+
+
+def test_vk_prefill_chains_into_vk_decode():
+    """A prefill in the transposed layout with a bf16 final state hands it to decode in the
+    same layout; the result matches the oracle over T + 1 tokens under the bars."""
+    full = small(T=130, H=3, init="f32", seed=14)
+    d = dev(full)
+    part = {n: d[n][:, :129].contiguous() for n in ("q", "k", "v", "g", "beta")}
+    init_vk = d["initial_state"].transpose(-1, -2).contiguous()
+    _, fin_vk = kda.kda_fwd_ex(**dict(d, **part, initial_state=init_vk), state_layout="vk",
+                               final_state_dtype=torch.bfloat16)
+    last = lambda t: t[:, 129].contiguous()
+    out_dec, st = kda.kda_decode_ex(last(d["q"]), last(d["k"]), last(d["v"]), last(d["g"]),
+                                    d["beta"][:, 129].contiguous(), d["scale"], d["A_log"],
+                                    d["dt_bias"], d["lower_bound"], fin_vk, state_layout="vk",
+                                    state_out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    out_r, fin_r = oracle.forward_inputs(full)
+    od = out_dec.float().cpu().numpy().astype(np.float64)
+    assert np.abs(od - out_r[:, 129]).max() <= OUT_MAXABS and rel(od, out_r[:, 129]) <= OUT_REL
+    fs = st.transpose(-1, -2).cpu().numpy().astype(np.float64)
+    # the handed-over state was rounded to bf16 (about 2^-9 relative), so the final state
+    # carries that rounding on top of the kernel's own error
+    assert rel(fs, fin_r) <= 4e-3
 
 
 def test_prefill_then_decode_equals_longer_prefill():
