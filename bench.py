@@ -69,6 +69,8 @@ def parse():
     ap.add_argument("--decode-seqs", type=int, default=256)
     # time one of the five parity workloads (kda_inputs recipe) instead of the headline
     ap.add_argument("--config-id", type=int, default=None, choices=[0, 1, 2, 3, 4])
+    ap.add_argument("--schedule", default="auto", choices=["auto", "fused", "split"],
+                    help="forward kernel schedule (kda_set_schedule); auto picks per launch")
     a = ap.parse_args()
     if a.batch:
         WORKLOAD["B"] = a.batch
@@ -454,6 +456,7 @@ def run_config_bench(args, world, rank, local):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     wl = ki.WORKLOADS[args.config_id]
+    kda.kda_set_schedule(args.schedule)
     inp = ki.make_inputs(args.config_id)
     d = lambda t: None if t is None else t.to(device)
     call = dict(q=d(inp.q), k=d(inp.k), v=d(inp.v), g=d(inp.g), beta=d(inp.beta), scale=inp.scale,
@@ -488,7 +491,8 @@ def run_config_bench(args, world, rank, local):
             "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
-            "config": {"workload": wl.name, "tokens": tokens, "sequences": N, "heads": H, "ctas": N * H},
+            "config": {"workload": wl.name, "tokens": tokens, "sequences": N, "heads": H,
+                       "schedule": args.schedule},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
                          "alg_bytes_per_launch": bytes_launch, "kernel": KERNEL},
@@ -576,6 +580,7 @@ def main():
     kbuild.build()
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
+    kda.kda_set_schedule(args.schedule)
     w = WORKLOAD
     inp = device_inputs(args.seed + 1000 * rank, device)
     B, T, H = w["B"], w["T"], w["H"]

@@ -299,6 +299,20 @@ int kda_last_launch_count(void);
  * without trapping).  Synchronous (reads device memory); reset != 0 clears it. */
 int kda_device_status(int reset);
 
+/* Schedule of the forward kernel, process-wide (returns the previous one, or
+ * KDA_ERR_ARG):
+ *   KDA_SCHEDULE_AUTO  (default) split when every unit fits the device as a cluster
+ *                      and units average at least 4 chunks (256 tokens), else fused;
+ *   KDA_SCHEDULE_FUSED one CTA per (sequence, head) runs both roles;
+ *   KDA_SCHEDULE_SPLIT a cluster of 4 CTAs per (sequence, head) whenever all units
+ *                      fit the device at once (else fused): 3 CTAs prepare every
+ *                      third chunk each and one runs the state pass.
+ * Both schedules run the same arithmetic in the same order: results are identical. */
+#define KDA_SCHEDULE_AUTO 0
+#define KDA_SCHEDULE_FUSED 1
+#define KDA_SCHEDULE_SPLIT 2
+int kda_set_schedule(int mode);
+
 /* Testing hook for the failure path (no counterpart on the pages): the next forward
  * launch (kda_fwd, kda_fwd_ex, kda_fwd_host) starts as if one of its CTAs had
  * already given up a bounded wait with `code` (1..255).  Every CTA of that launch

@@ -9,7 +9,7 @@ The functions mirror the C ABI in ``include/kda.h``:
   kda_bwd_workspace_size,
   kda_fwd_host,
   kda_fwd_host_workspace_size, kda_set_checks, kda_strerror, kda_last_launch_count,
-  kda_device_status, kda_inject_error.
+  kda_device_status, kda_inject_error, kda_set_schedule.
 """
 from __future__ import annotations
 
@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
             L.kda_device_status.restype = I
             L.kda_inject_error.argtypes = [I]
             L.kda_inject_error.restype = I
+            L.kda_set_schedule.argtypes = [I]
+            L.kda_set_schedule.restype = I
             _lib = L
     return _lib
 
@@ -105,6 +107,20 @@ def kda_last_launch_count() -> int:
 def kda_device_status(reset: bool = False) -> int:
     """Error word of the last kernels (0 = every bounded wait completed)."""
     return int(lib().kda_device_status(int(bool(reset))))
+
+
+KDA_SCHEDULE_AUTO, KDA_SCHEDULE_FUSED, KDA_SCHEDULE_SPLIT = 0, 1, 2
+_SCHEDULES = {"auto": KDA_SCHEDULE_AUTO, "fused": KDA_SCHEDULE_FUSED, "split": KDA_SCHEDULE_SPLIT}
+
+
+def kda_set_schedule(mode) -> str:
+    """Forward kernel schedule, process-wide: "auto" (default), "fused" (one CTA per
+    (sequence, head)) or "split" (a 4-CTA cluster per unit whenever all units fit the
+    device); returns the previous one.  Results are identical under every schedule."""
+    rc = lib().kda_set_schedule(_SCHEDULES[mode] if isinstance(mode, str) else int(mode))
+    if rc < 0:
+        raise KDAError(rc, "kda_set_schedule")
+    return {v: k for k, v in _SCHEDULES.items()}[rc]
 
 
 def kda_inject_error(code: int) -> None:

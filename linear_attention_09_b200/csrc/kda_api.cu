@@ -178,6 +178,8 @@ extern "C" int kda_device_status(int reset) { return kda::chunked_device_error(r
 
 extern "C" int kda_inject_error(int code) { return kda::chunked_inject_error(code); }
 
+extern "C" int kda_set_schedule(int mode) { return kda::chunked_set_schedule(mode); }
+
 extern "C" int kda_fwd_ex(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v,
                           const kda_bf16 *g, const kda_bf16 *beta, float scale,
                           const float *A_log, const float *dt_bias, float lower_bound,

@@ -34,6 +34,12 @@
 // Orientation: the inter-chunk products are computed transposed (M = value
 // column v on the 128 TMEM lanes), so S^T and U^T are tensor-core A operands
 // read straight from TMEM, and thread v owns value column v.
+//
+// Split schedule (few units, many idle SMs): a cluster of 4 CTAs per (sequence,
+// head).  CTAs 1..3 each run the in-chunk work for every third chunk and send its
+// results ([w ; q^ e^G], k', P, gamma by a bulk copy, u^T by stores) into one of two
+// slots in CTA 0's shared memory; CTA 0 runs only the state pass, consuming the
+// chunks in order and handing each slot back to the CTA that fills it next.
 #include <atomic>
 #include <cuda.h>
 
@@ -104,6 +110,23 @@ constexpr uint32_t TM_D3 = 384;  // (P U~)^T per lane v (64)
 constexpr uint32_t TM_SS = 384;  // S~^T fp16 pairs (A operand), 64 cols      (aliases D3)
 constexpr uint32_t TM_U = 448;   // u^T: lanes = v, cols = token (64)         (in-chunk -> state)
 
+// ---- schedules: every role runs in the fused kernel (one CTA per unit) or on one side
+//      of the split kernel (in-chunk work on CTAs 1..3, the state pass on CTA 0) ----
+enum Mode { kFused = 0, kProducer = 1, kConsumer = 2 };
+constexpr int kSplitCta = 4;       // CTAs per unit in the split kernel
+constexpr int kProducers = kSplitCta - 1;
+// CTA 0's two slots (byte offsets within a slot of SLOT_BYTES, 1024-aligned parts first)
+constexpr uint32_t SL_WQ = 0;              // 32 KB [w ; q^ e^G] fp16, as SM_WQ
+constexpr uint32_t SL_KP = 32 * 1024;      // 16 KB k' fp16, as SM_KP0
+constexpr uint32_t SL_P = 48 * 1024;       // 8 KB  P fp16, as SM_P
+constexpr uint32_t SL_U = 56 * 1024;       // u^T fp32, row v at SL_U + v * SL_UROW
+constexpr uint32_t SL_UROW = 272;          // 64 floats + 16 bytes: rows start in rotating banks
+constexpr uint32_t SL_GAM = SL_U + 128 * SL_UROW;  // 512 B gamma
+constexpr uint32_t SLOT_BYTES = ((SL_GAM + 512 + 1023) / 1024) * 1024;
+constexpr uint32_t SL_BARS = 2 * SLOT_BYTES;       // consumer barriers
+constexpr uint32_t kSendBytes = 32768 + 16384 + 8192 + 512;  // bulk bytes per chunk
+static_assert(SL_BARS + 256 <= 224 * 1024, "two slots fit the shared memory");
+
 __device__ __forceinline__ uint32_t sw(uint32_t row, uint32_t colbyte) { return sw128_offset(row, colbyte); }
 
 __device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -169,6 +192,16 @@ struct Bars {
     uint64_t u_free;   // u^T read out of TMEM                 (128 arrivals)
     uint64_t ops;      // operands of the next in-chunk product written (one arrival per
                        // in-chunk warp); the issue warp waits on it
+    // split kernel, CTAs 1..3:
+    uint64_t u_rdy;     // u^T of the chunk complete in TMEM              (commit)
+    uint64_t slot_free; // CTA 0 released the slot this CTA fills next    (1 remote arrival)
+};
+
+// Split kernel, CTA 0: slot s holds a chunk once its bulk bytes, its 128 u^T rows and
+// CTA 0's own re-arming arrival (which sets the expected bytes) are all in.
+struct SlotBars {
+    uint64_t full[2];
+    uint64_t mma_st;
 };
 
 struct TMaps {
@@ -184,7 +217,14 @@ struct Ctx {
     int64_t h, H, tok0, len, rstride;
     int64_t unit;  // (sequence, head) unit = sequence * H + head
     int nchunks;
+    // split kernel: this CTA's chunks are first, first + kProducers, ... (CTAs 1..3);
+    // CTA 0's slot base and slot barriers as shared::cluster addresses
+    int first;
+    uint32_t c_slots, c_full;
 };
+
+// The same for a barrier completed by other CTAs of the cluster (acquire at cluster scope).
+__device__ __forceinline__ bool wait_or_flag_cluster(uint64_t *bar, uint32_t parity, int code);
 
 // Bounded wait (about 1 s at 1965 MHz); one that gives up records (epoch << 8) | code
 // unless an earlier failure of the launch is already recorded.  The spin itself stays
@@ -193,6 +233,13 @@ struct Ctx {
 __device__ __forceinline__ bool wait_or_flag(uint64_t *bar, uint32_t parity, int code)
 {
     if (mbar_wait(bar, parity, 2000000000LL)) return true;
+    atomicCAS(&g_chunk_error, 0, (int)(s_epoch << 8) | code);
+    return false;
+}
+
+__device__ __forceinline__ bool wait_or_flag_cluster(uint64_t *bar, uint32_t parity, int code)
+{
+    if (mbar_wait_cluster(bar, parity, 2000000000LL)) return true;
     atomicCAS(&g_chunk_error, 0, (int)(s_epoch << 8) | code);
     return false;
 }
@@ -220,6 +267,7 @@ __device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *tm, u
 // decay-weighted products A and P (tf32), the triangular solve for T, and the
 // products w = T (k^ e^G), u = T v; hands [w ; q^ e^G], k', P, u^T and gamma over.
 // =====================================================================================
+template <Mode M>
 __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx)
 {
     uint8_t *sm = cx.sm;
@@ -236,6 +284,14 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
     const float a2 = aexp * kLog2e, lb2 = p.lower_bound * kLog2e;
     uint32_t mma_cnt = 0;  // completed phases of bars->mma_in waited on so far
     bool ok = true;
+    // The role's own chunks: all of the unit's (fused), or every kProducers-th from
+    // cx.first (split kernel); n counts own chunks (the phases of the local barriers),
+    // uc(n) is the chunk of the unit.
+    constexpr int S = (M == kProducer) ? kProducers : 1;
+    const int f = (M == kProducer) ? cx.first : 0;
+    auto uc = [&](int n) { return f + S * n; };
+    const int nown = cx.nchunks > f ? (cx.nchunks - f + S - 1) / S : 0;
+    bool sent_ok = true;  // split kernel, thread 0: the last hand-off's slot wait
 
     // Channel-pass thread mapping: channel pair 2cp, 2cp+1 (of each 64-channel round),
     // token octant oc (tokens 8oc..8oc+7; their rows have row % 8 == j).  Swizzled byte
@@ -334,20 +390,20 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
     // w/u products are (the octant-sum barrier at the top of the round publishes them).
     // Norms and beta are double-buffered by chunk parity.
     float2 G0[8];  // round-0 gate of the chunk about to be processed
-    if (cx.nchunks > 0) {
-        load_beta(0);
+    if (nown > 0) {
+        load_beta(uc(0));
         ok = named_bar_and(BAR_IN, NT_IN, wait_or_flag(&bars->qkg[0], 0, 6) && wait_or_flag(&bars->qkg[1], 0, 13));
         if (ok) {
-            norms(chunk_len(0), 0);
-            gate_round(0, chunk_len(0), G0);
-            load_beta(1);
+            norms(chunk_len(uc(0)), 0);
+            gate_round(0, chunk_len(uc(0)), G0);
+            load_beta(uc(1));
         }
     }
 
-    for (int n = 0; n < cx.nchunks && ok; ++n) {
-        const int64_t ctok = cx.tok0 + (int64_t)n * C;
-        const int L = chunk_len(n);
-        const bool has_next = n + 1 < cx.nchunks;
+    for (int n = 0; n < nown && ok; ++n) {
+        const int64_t ctok = cx.tok0 + (int64_t)uc(n) * C;
+        const int L = chunk_len(uc(n));
+        const bool has_next = n + 1 < nown;
         const uint32_t par = (uint32_t)n & 1u, ppar = (uint32_t)(n - 1) & 1u;
         const uint32_t skp = par ? SM_KP1 : SM_KP0;  // this chunk's k' buffer
         const float *rkq_c = cx.rkq_s + par * 128, *b_c = cx.b_s + par * 64;  // norms, beta
@@ -367,7 +423,15 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             // Round 0 first waits until chunk n-2, the previous user of this chunk's k'
             // buffer and gamma slot (both indexed by chunk parity), is fully consumed.
             bool kok = true;
-            if (round == 0 && n >= 2) kok = wait_or_flag(&bars->kp_free[par], (uint32_t)((n >> 1) - 1) & 1u, 8);
+            if constexpr (M == kFused) {
+                if (round == 0 && n >= 2) kok = wait_or_flag(&bars->kp_free[par], (uint32_t)((n >> 1) - 1) & 1u, 8);
+            } else {
+                // the previous hand-off's bulk copies have read [w ; q^ e^G], P, k' and gamma
+                if (round == 0 && n >= 1 && tid == 0) {
+                    bulk_wait_read_all();
+                    kok = sent_ok;
+                }
+            }
 
             // octant sums -> chunk prefix sums and the reference values G15, G31, G47, G63
             ok = named_bar_and(BAR_IN, NT_IN, kok);
@@ -414,7 +478,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             bool wok = true;
             if (round == 1)  // A/P operands of round 0 must be consumed first
                 wok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 1);
-            else if (n > 0)  // q^ e^G of the previous chunk must be consumed
+            else if (M == kFused && n > 0)  // q^ e^G of the previous chunk must be consumed
                 wok = wait_or_flag(&bars->wq_free, ppar, 7);
             // operand rows of this octant; the block (uniform per warp) is a compile-time
             // branch of the loop body, and tokens past the chunk end have zero norms.
@@ -460,7 +524,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             ok = named_bar_and(BAR_IN, NT_IN, wok);
             if (!ok) break;
             // this round's box of q, k, g is consumed: prefetch the next chunk's
-            if (tid == 0 && has_next) load_qkg_box(sm, tm, &bars->qkg[round], h, ctok + C, round);
+            if (tid == 0 && has_next) load_qkg_box(sm, tm, &bars->qkg[round], h, cx.tok0 + (int64_t)uc(n + 1) * C, round);
         }
         if (!ok) break;
         // ---- while the round-1 A/P product runs: the next chunk's round-0 gate (its
@@ -468,13 +532,13 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         bool gok = true;
         if (has_next) {
             gok = wait_or_flag(&bars->qkg[0], par ^ 1u, 6);
-            gate_round(0, chunk_len(n + 1), G0);
+            gate_round(0, chunk_len(uc(n + 1)), G0);
         }
         {
             // the A/P product is complete, and chunk n-1's second state product (the last
             // reader of the single P tile) is done before P is overwritten
             const bool aok = wait_or_flag(&bars->mma_in, (mma_cnt++) & 1u, 1);
-            const bool pok = n < 1 || wait_or_flag(&bars->kp_free[ppar], (uint32_t)((n - 1) >> 1) & 1u, 11);
+            const bool pok = M != kFused || n < 1 || wait_or_flag(&bars->kp_free[ppar], (uint32_t)((n - 1) >> 1) & 1u, 11);
             ok = named_bar_and(BAR_IN, NT_IN, aok && pok && gok);
         }
         tc_fence_after();
@@ -705,8 +769,8 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         bool sok = true;
         if (has_next) {
             sok = wait_or_flag(&bars->qkg[1], par ^ 1u, 13);
-            norms(chunk_len(n + 1), (int)(par ^ 1u));
-            load_beta(n + 2);
+            norms(chunk_len(uc(n + 1)), (int)(par ^ 1u));
+            load_beta(uc(n + 2));
         }
         {
             // (if the issue warp gave up, this bounded wait runs out)
@@ -731,7 +795,27 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
         fence_async_smem();
         tc_fence_before();
         named_bar(BAR_IN, NT_IN);
-        if (tid == 0) mbar_arrive(&bars->full);  // chunk n handed to the state role
+        if constexpr (M == kFused) {
+            if (tid == 0) mbar_arrive(&bars->full);  // chunk n handed to the state role
+        } else if (tid == 0) {
+            // chunk uc(n) into CTA 0's slot uc(n) & 1, once CTA 0 has released it (its
+            // previous content, chunk uc(n) - 2, consumed); the bulk bytes complete the
+            // slot's barrier together with the u^T rows of the sending warps
+            const int c = uc(n);
+            sent_ok = c < 2 || wait_or_flag(&bars->slot_free, (uint32_t)(n - (f >= 2 ? 0 : 1)) & 1u, 16);
+            if (sent_ok) {
+                const uint32_t slot = cx.c_slots + (uint32_t)(c & 1) * SLOT_BYTES;
+                const uint32_t fb = cx.c_full + (uint32_t)(c & 1) * 8u;
+                bulk_s2cluster(slot + SL_WQ, sm + SM_WQ, 32768, fb);
+                bulk_s2cluster(slot + SL_KP, sm + skp, 16384, fb);
+                bulk_s2cluster(slot + SL_P, sm + SM_P, 8192, fb);
+                bulk_s2cluster(slot + SL_GAM, cx.gam_s + par * 128, 512, fb);
+                bulk_commit();
+            }
+        }
+    }
+    if constexpr (M == kProducer) {
+        if (tid == 0) bulk_wait_read_all();  // no copy still reads this CTA's shared memory
     }
 }
 
@@ -741,6 +825,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
 // (the `ops` barrier, one arrival per in-chunk warp) and commits each group to
 // `mma_in`.  The in-chunk warps never stall on issuing.
 // =====================================================================================
+template <Mode M>
 __device__ void mma_role(const Ctx &cx)
 {
     if ((threadIdx.x & 31) != 0) return;
@@ -754,7 +839,10 @@ __device__ void mma_role(const Ctx &cx)
     const uint32_t idw = idesc(128, 64, kF16, kF16, true, false);
     const uint32_t idu = idesc(128, 64, kBF16, kBF16, true, false);
     uint32_t ops_cnt = 0;
-    for (int n = 0; n < cx.nchunks; ++n) {
+    constexpr int S = (M == kProducer) ? kProducers : 1;
+    const int f = (M == kProducer) ? cx.first : 0;
+    const int nown = cx.nchunks > f ? (cx.nchunks - f + S - 1) / S : 0;
+    for (int n = 0; n < nown; ++n) {
         const uint32_t par = (uint32_t)n & 1u, ppar = (uint32_t)(n - 1) & 1u;
         for (int round = 0; round < 2; ++round) {
             if (!wait_or_flag(&bars->ops, (ops_cnt++) & 1u, 12)) return;
@@ -784,6 +872,42 @@ __device__ void mma_role(const Ctx &cx)
             mma_f16_ss(tb + TM_U, desc_sw128(sv + st * 2048, 8192, 1024),
                        desc_sw128(slo + st * 32, 16, 1024), idu, 1);
         mma_commit(&bars->mma_in);  // w and u: T, v and k^ e^G are consumed once it completes
+        if constexpr (M == kProducer) mma_commit(&bars->u_rdy);
+    }
+}
+
+// =====================================================================================
+// Split kernel, CTAs 1..3, warps 8..11 (thread v <-> TMEM lane v): each chunk's u^T
+// row v, read out of TMEM once the w/u products complete, stored into row v of CTA
+// 0's slot for the chunk; then one arrival each on the slot's barrier.
+// =====================================================================================
+__device__ void u_send_role(const Ctx &cx)
+{
+    Bars *bars = cx.bars;
+    const uint32_t tb = cx.tb;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int v = tid - NT_IN;
+    const uint32_t lq = (uint32_t)((warp & 3) * 32) << 16;
+    const int f = cx.first;
+    const int nown = cx.nchunks > f ? (cx.nchunks - f + kProducers - 1) / kProducers : 0;
+    for (int n = 0; n < nown; ++n) {
+        const int c = f + kProducers * n;
+        if (!wait_or_flag(&bars->u_rdy, (uint32_t)n & 1u, 17)) return;
+        tc_fence_after();
+        uint32_t a[32], b[32];
+        tmem_ld32(tb + lq + TM_U, a);
+        tmem_ld32(tb + lq + TM_U + 32, b);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->u_free);  // the next chunk's u product may overwrite TM_U
+        if (c >= 2 && !wait_or_flag(&bars->slot_free, (uint32_t)(n - (f >= 2 ? 0 : 1)) & 1u, 18)) return;
+        const uint32_t row = cx.c_slots + (uint32_t)(c & 1) * SLOT_BYTES + SL_U + (uint32_t)v * SL_UROW;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st_cluster_v4(row + 16u * j, make_uint4(a[4 * j], a[4 * j + 1], a[4 * j + 2], a[4 * j + 3]));
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            st_cluster_v4(row + 128u + 16u * j, make_uint4(b[4 * j], b[4 * j + 1], b[4 * j + 2], b[4 * j + 3]));
+        mbar_arrive_remote(cx.c_full + (uint32_t)(c & 1) * 8u);
     }
 }
 
@@ -794,6 +918,7 @@ __device__ void mma_role(const Ctx &cx)
 //   -> U~ = U / tau' -> TM_S <- (gamma * TM_S) tau / tau' -> MMA2: TM_S += U~^T k',
 //   D3 = U~^T P^T -> out = scale (sigma D1[:,64:128] + tau' D3).
 // =====================================================================================
+template <Mode M>
 __device__ void state_role(const FwdParams &p, const Ctx &cx)
 {
     uint8_t *sm = cx.sm;
@@ -807,6 +932,9 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
     const size_t state_off = (size_t)cx.unit * kHead * kHead;
     uint32_t mma_cnt = 0;
     bool ok = true;
+    // split kernel, CTA 0: the chunks arrive in two slots of this CTA's shared memory
+    SlotBars *sb = reinterpret_cast<SlotBars *>(sm + SL_BARS);
+    uint64_t *bar_mma = (M == kConsumer) ? &sb->mma_st : &bars->mma_st;
 
     // element (k, v) of a state in either layout: S[k][v] (rows of the KV layout are
     // read and written coalesced across threads v) or S[v][k] (thread v owns a row)
@@ -846,6 +974,7 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
         const int64_t rem = cx.len - (int64_t)n * C;
         const int L = (int)(rem < C ? rem : C);
         const uint32_t par = (uint32_t)n & 1u;
+        const uint32_t slot = par * SLOT_BYTES;  // split kernel: this chunk's slot
 
         // ---- S~^T = (tau TM_S) / sigma as fp16 pairs into TM_SS ----
         float sigma;
@@ -876,20 +1005,23 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
 
         // ---- wait for the chunk's operands; MMA1: D1 = S~^T [w ; q^ e^G]^T ----
         tc_fence_before();  // the S~ stores above precede MMA1
-        ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(&bars->full, par, 10));
+        if constexpr (M == kConsumer)
+            ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag_cluster(&sb->full[par], ((uint32_t)n >> 1) & 1u, 10));
+        else
+            ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(&bars->full, par, 10));
         tc_fence_after();
         if (!ok) break;
         if (leader) {
-            const uint32_t swq = smem_u32(sm + SM_WQ);
+            const uint32_t swq = smem_u32(sm + (M == kConsumer ? slot + SL_WQ : SM_WQ));
             const uint32_t id = idesc(128, 128, kF16, kF16, false, false);
 #pragma unroll
             for (int st = 0; st < 8; ++st)
                 mma_f16_ts(tb + TM_D1, tb + TM_SS + st * 8,
                            desc_sw128(swq + (st >> 2) * 16384 + (st & 3) * 32, 16, 1024), id, st > 0);
-            mma_commit(&bars->mma_st);
-            mma_commit(&bars->wq_free);
+            mma_commit(bar_mma);
+            if constexpr (M == kFused) mma_commit(&bars->wq_free);
         }
-        ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(&bars->mma_st, (mma_cnt++) & 1u, 4));
+        ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(bar_mma, (mma_cnt++) & 1u, 4));
         tc_fence_after();
         if (!ok) break;
 
@@ -901,13 +1033,25 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
             for (int t0 = 0; t0 < C; t0 += 32) {
                 uint32_t a[32], b[32];
                 tmem_ld32(tb + lq + TM_D1 + t0, a);
-                tmem_ld32(tb + lq + TM_U + t0, b);
+                if constexpr (M == kConsumer) {  // u^T row v from the slot
+                    const uint4 *ur = reinterpret_cast<const uint4 *>(sm + slot + SL_U + (uint32_t)v * SL_UROW + t0 * 4);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint4 x = ur[j];
+                        b[4 * j] = x.x;
+                        b[4 * j + 1] = x.y;
+                        b[4 * j + 2] = x.z;
+                        b[4 * j + 3] = x.w;
+                    }
+                } else {
+                    tmem_ld32(tb + lq + TM_U + t0, b);
+                }
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) U[t0 + j] = __uint_as_float(b[j]) - sigma * __uint_as_float(a[j]);
             }
             tc_fence_before();
-            mbar_arrive(&bars->u_free);  // u^T of this chunk is out of TMEM
+            if constexpr (M == kFused) mbar_arrive(&bars->u_free);  // u^T of this chunk is out of TMEM
             float mx = 0.f;
 #pragma unroll
             for (int t = 0; t < C; ++t) mx = fmaxf(mx, fabsf(U[t]));
@@ -924,7 +1068,7 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
         // ---- TM_S <- gamma * TM_S * (tau / tau'), so that MMA2 can accumulate U~^T k' ----
         {
             const float f = tau / tau_n;
-            const float *gam = cx.gam_s + par * 128;
+            const float *gam = (M == kConsumer) ? reinterpret_cast<const float *>(sm + slot + SL_GAM) : cx.gam_s + par * 128;
 #pragma unroll
             for (int k0 = 0; k0 < kHead; k0 += 32) {
                 uint32_t a[32];
@@ -953,7 +1097,8 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
 
         // ---- MMA2: TM_S += U~^T k' (N = 128), D3 = U~^T P^T (N = 64) ----
         if (leader) {
-            const uint32_t skp = smem_u32(sm + (par ? SM_KP1 : SM_KP0)), sp = smem_u32(sm + SM_P);
+            const uint32_t skp = smem_u32(sm + (M == kConsumer ? slot + SL_KP : (par ? SM_KP1 : SM_KP0)));
+            const uint32_t sp = smem_u32(sm + (M == kConsumer ? slot + SL_P : SM_P));
             const uint32_t id2 = idesc(128, 128, kF16, kF16, false, true);
             const uint32_t id3 = idesc(128, 64, kF16, kF16, false, false);
 #pragma unroll
@@ -962,12 +1107,22 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
 #pragma unroll
             for (int st = 0; st < 4; ++st)
                 mma_f16_ts(tb + TM_D3, tb + TM_D1 + st * 8, desc_sw128(sp + st * 32, 16, 1024), id3, st > 0);
-            mma_commit(&bars->mma_st);
-            mma_commit(&bars->kp_free[par]);
+            mma_commit(bar_mma);
+            if constexpr (M == kFused) mma_commit(&bars->kp_free[par]);
         }
-        ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(&bars->mma_st, (mma_cnt++) & 1u, 5));
+        ok = named_bar_and(BAR_ST, NT_ST, wait_or_flag(bar_mma, (mma_cnt++) & 1u, 5));
         tc_fence_after();
         if (!ok) break;
+        if constexpr (M == kConsumer) {
+            // the slot is consumed (MMA1, MMA2 complete; u and gamma read before the
+            // barrier above): re-arm it for chunk n + 2 (expected bytes), and tell the CTA
+            // that sends chunk n + 2 that it may
+            if (leader && n + 2 < cx.nchunks) {
+                mbar_arrive_expect_tx(&sb->full[par], kSendBytes);
+                const uint32_t dst = 1u + (uint32_t)((n + 2) % kProducers);
+                mbar_arrive_remote(mapa_shared(smem_u32(&bars->slot_free), dst));
+            }
+        }
 
         // ---- out = scale (sigma D1[:, 64:128] + tau D3): thread v stores column v of each
         //      token; a warp's 32 columns are 64 contiguous bytes of the token's row ----
@@ -1006,30 +1161,31 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
     }
 }
 
-__global__ void __launch_bounds__(NT, 1)
-chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
+// Shared-memory context of a CTA (the same offsets in every CTA of either kernel).
+__device__ __forceinline__ void init_ctx(Ctx &cx, uint8_t *sm)
 {
-    extern __shared__ uint8_t smem_raw[];
-    // 1024-byte alignment by pointer arithmetic on the shared array itself, so that the
-    // compiler keeps every access through sm in the shared space (32-bit addresses,
-    // shared loads/stores) instead of falling back to generic ones
-    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    Ctx cx;
     cx.sm = sm;
     cx.rkq_s = reinterpret_cast<float *>(sm + SM_MISC);
     cx.b_s = cx.rkq_s + 256;    // [2][64]
     cx.gam_s = cx.b_s + 128;    // [2][128]
     cx.osum = cx.gam_s + 256;   // [8][128]
     cx.bars = reinterpret_cast<Bars *>(cx.osum + 1024);
-    uint32_t *tbase_s = reinterpret_cast<uint32_t *>(cx.bars + 1);
     cx.dtb_s = reinterpret_cast<float *>(sm + SM_MISC + 7168);
+    cx.first = 0;
+    cx.c_slots = cx.c_full = 0;
+}
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+// The launch's (sequence, head) unit u into cx: sequence-major, with the sequences of a
+// varlen batch of up to kLptMax in decreasing length.  Every thread of the CTA calls it.
+__device__ void locate_unit(const FwdParams &p, Ctx &cx, int64_t u)
+{
+    uint8_t *sm = cx.sm;
+    const int tid = threadIdx.x;
     cx.H = p.H;
-    int64_t s = blockIdx.x / p.H;
-    cx.h = blockIdx.x % p.H;
+    int64_t s = u / p.H;
+    cx.h = u % p.H;
     if (p.cu && p.N > 1 && p.N <= kLptMax) {
-        // Longest sequences first: CTA group r takes the sequence of rank r in decreasing
+        // Longest sequences first: unit group r takes the sequence of rank r in decreasing
         // length (ties by index; the ranks are a permutation), so that the end of the grid
         // holds short sequences rather than a long one started last.  The A/P region is
         // free until the first chunk.
@@ -1040,7 +1196,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
         for (int c = tid; c < p.N; c += NT) {
             const int64_t lc = lens[c];
             int64_t rank = 0;
-            for (int u = 0; u < p.N; ++u) rank += (lens[u] > lc) || (lens[u] == lc && u < c);
+            for (int v = 0; v < p.N; ++v) rank += (lens[v] > lc) || (lens[v] == lc && v < c);
             if (rank == s) *pick = c;
         }
         __syncthreads();
@@ -1058,23 +1214,52 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
     }
     cx.rstride = p.H * kHead;
     cx.nchunks = (int)((cx.len + C - 1) / C);
+}
+
+// Barriers of a CTA that runs the in-chunk role (fused kernel, or CTAs 1..3 of the split
+// kernel); thread 0.
+__device__ __forceinline__ void init_bars(Bars *b)
+{
+    mbar_init(&b->qkg[0], 1);
+    mbar_init(&b->qkg[1], 1);
+    mbar_init(&b->v, 1);
+    mbar_init(&b->mma_in, 1);
+    mbar_init(&b->mma_st, 1);
+    mbar_init(&b->full, 1);
+    mbar_init(&b->wq_free, 1);
+    mbar_init(&b->kp_free[0], 1);
+    mbar_init(&b->kp_free[1], 1);
+    mbar_init(&b->u_free, NT_ST);
+    mbar_init(&b->ops, NT_IN / 32);
+    mbar_init(&b->u_rdy, 1);
+    mbar_init(&b->slot_free, 1);
+}
+
+// Thread 0: has another CTA of this launch already given up?
+__device__ __forceinline__ void read_abort(const FwdParams &p)
+{
+    s_epoch = p.epoch;
+    const int e = *reinterpret_cast<volatile int *>(&g_chunk_error);
+    s_abort = e != 0 && ((uint32_t)e >> 8) == p.epoch;
+}
+
+__global__ void __launch_bounds__(NT, 1)
+chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
+{
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte alignment by pointer arithmetic on the shared array itself, so that the
+    // compiler keeps every access through sm in the shared space (32-bit addresses,
+    // shared loads/stores) instead of falling back to generic ones
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Ctx cx;
+    init_ctx(cx, sm);
+    uint32_t *tbase_s = reinterpret_cast<uint32_t *>(cx.bars + 1);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    locate_unit(p, cx, blockIdx.x);
 
     if (tid == 0) {
-        s_epoch = p.epoch;
-        const int e = *reinterpret_cast<volatile int *>(&g_chunk_error);
-        s_abort = e != 0 && ((uint32_t)e >> 8) == p.epoch;
-        Bars *b = cx.bars;
-        mbar_init(&b->qkg[0], 1);
-        mbar_init(&b->qkg[1], 1);
-        mbar_init(&b->v, 1);
-        mbar_init(&b->mma_in, 1);
-        mbar_init(&b->mma_st, 1);
-        mbar_init(&b->full, 1);
-        mbar_init(&b->wq_free, 1);
-        mbar_init(&b->kp_free[0], 1);
-        mbar_init(&b->kp_free[1], 1);
-        mbar_init(&b->u_free, NT_ST);
-        mbar_init(&b->ops, NT_IN / 32);
+        read_abort(p);
+        init_bars(cx.bars);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -1097,12 +1282,79 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
         load_tile(sm + SM_V, &tm.v, &cx.bars->v, cx.h, cx.tok0);
     }
 
-    if (warp < NT_IN / 32) in_chunk_role(p, tm, cx);
-    else if (warp < (NT_IN + NT_ST) / 32) state_role(p, cx);
-    else mma_role(cx);
+    if (warp < NT_IN / 32) in_chunk_role<kFused>(p, tm, cx);
+    else if (warp < (NT_IN + NT_ST) / 32) state_role<kFused>(p, cx);
+    else mma_role<kFused>(cx);
 
     tc_fence_before();
     __syncthreads();
+    if (warp == 0) tmem_dealloc(cx.tb, 512);
+}
+
+// Split kernel: a cluster of kSplitCta CTAs per unit (cluster index = unit).  CTA 0 runs
+// the state pass on chunks that CTAs 1..3 prepare (chunk c on CTA 1 + c % 3).
+__global__ void __launch_bounds__(NT, 1)
+chunk_kernel_split(const FwdParams p, const __grid_constant__ TMaps tm)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Ctx cx;
+    init_ctx(cx, sm);
+    uint32_t *tbase_s = reinterpret_cast<uint32_t *>(cx.bars + 1);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const uint32_t rank = cluster_ctarank();
+    locate_unit(p, cx, blockIdx.x / kSplitCta);
+    cx.first = (int)rank - 1;
+    cx.c_slots = mapa_shared(smem_u32(sm), 0);  // the same offsets in every CTA
+    cx.c_full = mapa_shared(smem_u32(sm + SL_BARS), 0);
+    SlotBars *sb = reinterpret_cast<SlotBars *>(sm + SL_BARS);
+
+    if (tid == 0) {
+        read_abort(p);
+        if (rank == 0) {
+            mbar_init(&sb->full[0], 1 + NT_ST);
+            mbar_init(&sb->full[1], 1 + NT_ST);
+            mbar_init(&sb->mma_st, 1);
+        } else {
+            init_bars(cx.bars);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tbase_s, 512);
+        tmem_relinquish();
+    }
+    if (rank != 0 && tid < kHead && cx.nchunks > cx.first) cx.dtb_s[tid] = p.dt_bias[cx.h * kHead + tid];
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    cx.tb = *tbase_s;
+    if (rank == 0 && tid == 0) {  // slots 0 and 1 expect their first chunks' bulk bytes
+        if (cx.nchunks > 0) mbar_arrive_expect_tx(&sb->full[0], kSendBytes);
+        if (cx.nchunks > 1) mbar_arrive_expect_tx(&sb->full[1], kSendBytes);
+    }
+    cluster_sync();  // every CTA's barriers are initialised before any remote access
+
+    if (!s_abort) {
+        if (rank == 0) {
+            if (warp >= NT_IN / 32 && warp < (NT_IN + NT_ST) / 32) state_role<kConsumer>(p, cx);
+        } else {
+            if (tid == 0 && cx.first < cx.nchunks) {  // first own chunk's tiles
+                const int64_t tok = cx.tok0 + (int64_t)cx.first * C;
+                load_qkg_box(sm, tm, &cx.bars->qkg[0], cx.h, tok, 0);
+                load_qkg_box(sm, tm, &cx.bars->qkg[1], cx.h, tok, 1);
+                mbar_arrive_expect_tx(&cx.bars->v, 16384);
+                load_tile(sm + SM_V, &tm.v, &cx.bars->v, cx.h, tok);
+            }
+            if (warp < NT_IN / 32) in_chunk_role<kProducer>(p, tm, cx);
+            else if (warp < (NT_IN + NT_ST) / 32) u_send_role(cx);
+            else mma_role<kProducer>(cx);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // no CTA leaves while a copy or an arrival may still target it
     if (warp == 0) tmem_dealloc(cx.tb, 512);
 }
 
@@ -1130,6 +1382,54 @@ EncodeTiledFn encode_fn()
 }
 
 }  // namespace
+
+// Launch configuration of the split kernel for `units` units (clusters of kSplitCta).
+static void split_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute (&at)[1], int64_t units,
+                         cudaStream_t stream)
+{
+    cfg.gridDim = dim3((unsigned)(units * kSplitCta));
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = SMEM_ALLOC;
+    cfg.stream = stream;
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = kSplitCta;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+}
+
+// The split kernel serves launches whose units all fit the device at once as clusters
+// (so a unit's chunks spread over 4 SMs instead of 1), with at least kSplitMinChunks
+// chunks per unit on average; larger launches already fill the SMs with one CTA per unit.
+constexpr int64_t kSplitMinChunks = 4;
+std::atomic<int> g_schedule{KDA_SCHEDULE_AUTO};
+
+static bool use_split(const FwdParams &p, int64_t units)
+{
+    const int mode = g_schedule.load();
+    if (mode == KDA_SCHEDULE_FUSED || units <= 0) return false;
+    const int64_t tokens = p.B * p.T;
+    if (mode == KDA_SCHEDULE_AUTO && tokens < kSplitMinChunks * C * (p.cu ? p.N : p.B)) return false;
+    static int clusters[64];  // per device: clusters of the split kernel resident at once (+1; 0 = unknown)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    if (clusters[dev] == 0) {
+        static int attr_split[64];
+        int n = 0;
+        if (set_smem_limit_once(chunk_kernel_split, SMEM_ALLOC, attr_split)) {
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute at[1];
+            split_config(cfg, at, 1, 0);
+            if (cudaOccupancyMaxActiveClusters(&n, chunk_kernel_split, &cfg) != cudaSuccess) {
+                n = 0;
+                cudaGetLastError();
+            }
+        }
+        clusters[dev] = n + 1;
+    }
+    return units <= clusters[dev] - 1;
+}
 
 int launch_chunked(const FwdParams &p, cudaStream_t stream)
 {
@@ -1168,8 +1468,22 @@ int launch_chunked(const FwdParams &p, cudaStream_t stream)
                                     stream) != cudaSuccess)
             return KDA_ERR_CUDA;
     }
+    if (use_split(p, ctas)) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute at[1];
+        split_config(cfg, at, ctas, stream);
+        if (cudaLaunchKernelEx(&cfg, chunk_kernel_split, pe, tm) != cudaSuccess) return KDA_ERR_CUDA;
+        return cudaGetLastError() == cudaSuccess ? 1 : KDA_ERR_CUDA;
+    }
     chunk_kernel<<<(unsigned)ctas, NT, SMEM_ALLOC, stream>>>(pe, tm);
     return cudaGetLastError() == cudaSuccess ? 1 : KDA_ERR_CUDA;
+}
+
+int chunked_set_schedule(int mode)
+{
+    if (mode != KDA_SCHEDULE_AUTO && mode != KDA_SCHEDULE_FUSED && mode != KDA_SCHEDULE_SPLIT)
+        return KDA_ERR_ARG;
+    return g_schedule.exchange(mode);
 }
 
 int chunked_inject_error(int code)

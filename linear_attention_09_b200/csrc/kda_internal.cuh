@@ -97,5 +97,6 @@ int launch_chunked(const FwdParams &p, cudaStream_t stream);
 // Error word the chunked kernel sets when a bounded wait gives up (0 = none).
 int chunked_device_error(bool reset);
 int chunked_inject_error(int code);  // the next launch starts failed with `code`
+int chunked_set_schedule(int mode);  // KDA_SCHEDULE_*; the previous mode or KDA_ERR_ARG
 
 }  // namespace kda
