@@ -470,6 +470,7 @@ def run_config_bench(args, world, rank, local):
     for _ in range(args.warmup):
         step()
     launches = kda.kda_last_launch_count()
+    kernel = "chunk_kernel_split" if kda.kda_last_schedule() == "split" else KERNEL
     torch.cuda.synchronize()
     barrier(world)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -495,7 +496,7 @@ def run_config_bench(args, world, rank, local):
                        "schedule": args.schedule},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": None, "peak_source": peak_src,
-                         "alg_bytes_per_launch": bytes_launch, "kernel": KERNEL},
+                         "alg_bytes_per_launch": bytes_launch, "kernel": kernel},
             "clocks": clk.summary(), "gpu_launches": launches * args.steps}), flush=True)
     return 0
 

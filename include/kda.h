@@ -313,6 +313,10 @@ int kda_device_status(int reset);
 #define KDA_SCHEDULE_SPLIT 2
 int kda_set_schedule(int mode);
 
+/* Schedule (KDA_SCHEDULE_FUSED or KDA_SCHEDULE_SPLIT) of the last forward launch this
+ * host thread enqueued (for reports). */
+int kda_last_schedule(void);
+
 /* Testing hook for the failure path (no counterpart on the pages): the next forward
  * launch (kda_fwd, kda_fwd_ex, kda_fwd_host) starts as if one of its CTAs had
  * already given up a bounded wait with `code` (1..255).  Every CTA of that launch

@@ -9,7 +9,7 @@ The functions mirror the C ABI in ``include/kda.h``:
   kda_bwd_workspace_size,
   kda_fwd_host,
   kda_fwd_host_workspace_size, kda_set_checks, kda_strerror, kda_last_launch_count,
-  kda_device_status, kda_inject_error, kda_set_schedule.
+  kda_device_status, kda_inject_error, kda_set_schedule, kda_last_schedule.
 """
 from __future__ import annotations
 
@@ -86,6 +86,8 @@ def lib() -> ctypes.CDLL:
             L.kda_inject_error.restype = I
             L.kda_set_schedule.argtypes = [I]
             L.kda_set_schedule.restype = I
+            L.kda_last_schedule.argtypes = []
+            L.kda_last_schedule.restype = I
             _lib = L
     return _lib
 
@@ -121,6 +123,11 @@ def kda_set_schedule(mode) -> str:
     if rc < 0:
         raise KDAError(rc, "kda_set_schedule")
     return {v: k for k, v in _SCHEDULES.items()}[rc]
+
+
+def kda_last_schedule() -> str:
+    """Schedule ("fused" or "split") of this thread's last forward launch."""
+    return {v: k for k, v in _SCHEDULES.items()}[int(lib().kda_last_schedule())]
 
 
 def kda_inject_error(code: int) -> None:

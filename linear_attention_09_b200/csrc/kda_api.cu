@@ -180,6 +180,8 @@ extern "C" int kda_inject_error(int code) { return kda::chunked_inject_error(cod
 
 extern "C" int kda_set_schedule(int mode) { return kda::chunked_set_schedule(mode); }
 
+extern "C" int kda_last_schedule(void) { return kda::chunked_last_schedule(); }
+
 extern "C" int kda_fwd_ex(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v,
                           const kda_bf16 *g, const kda_bf16 *beta, float scale,
                           const float *A_log, const float *dt_bias, float lower_bound,

@@ -1404,6 +1404,7 @@ static void split_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute (&at)[1], 
 // chunks per unit on average; larger launches already fill the SMs with one CTA per unit.
 constexpr int64_t kSplitMinChunks = 4;
 std::atomic<int> g_schedule{KDA_SCHEDULE_AUTO};
+thread_local int g_last_schedule = KDA_SCHEDULE_FUSED;  // of this thread's last launch
 
 static bool use_split(const FwdParams &p, int64_t units)
 {
@@ -1468,7 +1469,9 @@ int launch_chunked(const FwdParams &p, cudaStream_t stream)
                                     stream) != cudaSuccess)
             return KDA_ERR_CUDA;
     }
+    g_last_schedule = KDA_SCHEDULE_FUSED;
     if (use_split(p, ctas)) {
+        g_last_schedule = KDA_SCHEDULE_SPLIT;
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute at[1];
         split_config(cfg, at, ctas, stream);
@@ -1478,6 +1481,8 @@ int launch_chunked(const FwdParams &p, cudaStream_t stream)
     chunk_kernel<<<(unsigned)ctas, NT, SMEM_ALLOC, stream>>>(pe, tm);
     return cudaGetLastError() == cudaSuccess ? 1 : KDA_ERR_CUDA;
 }
+
+int chunked_last_schedule() { return g_last_schedule; }
 
 int chunked_set_schedule(int mode)
 {

@@ -98,5 +98,6 @@ int launch_chunked(const FwdParams &p, cudaStream_t stream);
 int chunked_device_error(bool reset);
 int chunked_inject_error(int code);  // the next launch starts failed with `code`
 int chunked_set_schedule(int mode);  // KDA_SCHEDULE_*; the previous mode or KDA_ERR_ARG
+int chunked_last_schedule();         // schedule of this thread's last forward launch
 
 }  // namespace kda
