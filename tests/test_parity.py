@@ -458,6 +458,31 @@ def test_pipelined_host_entry_matches_device_entry(case):
     np.testing.assert_array_equal(fin_h.numpy(), fin_d)
 
 
+
+def test_host_entry_point_on_a_nan_workspace_with_rows_past_the_last_sequence():
+    """kda_fwd_host copies each piece into a caller workspace; the last tile of a piece
+    also covers workspace rows that nothing wrote (here all bytes 0xFF, NaN as bf16),
+    including rows after the last sequence (cu_seqlens[N] < rows).  The kernel clears
+    them on chip, so the result is bit for bit the device call's on clean buffers."""
+    lengths, pad = [70, 45, 129], 50
+    inp = small(lengths=lengths, init="f32", seed=47)
+    rows = int(inp.cu_seqlens[-1])
+    out_d, fin_d = run_gpu(inp)
+    def padded(t):
+        extra = torch.zeros((1, pad) + tuple(t.shape[2:]), dtype=t.dtype)
+        return torch.cat([t, extra], dim=1).contiguous().pin_memory()
+    H = inp.H
+    ws = torch.full((kda.kda_fwd_host_workspace_size(1, rows + pad, H, num_seqs=len(lengths),
+                                                     initial_state_dtype=kda.KDA_STATE_F32),),
+                    255, dtype=torch.uint8, device="cuda")
+    out_h, fin_h = kda.kda_fwd_host(padded(inp.q), padded(inp.k), padded(inp.v), padded(inp.g),
+                                    padded(inp.beta), inp.scale, inp.A_log, inp.dt_bias,
+                                    inp.lower_bound, initial_state=inp.initial_state.pin_memory(),
+                                    cu_seqlens=inp.cu_seqlens, workspace=ws)
+    assert kda.kda_device_status(reset=True) == 0
+    np.testing.assert_array_equal(out_h[:, :rows].float().numpy(), out_d)
+    np.testing.assert_array_equal(fin_h.numpy(), fin_d)
+
 @pytest.mark.gpu
 def test_device_offset_check_rejects_bad_cu_seqlens():
     """With checks on, a varlen call whose cu_seqlens is not non-decreasing within
