@@ -134,7 +134,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
 
 // Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from this
 // CTA's shared memory into another CTA's of the cluster; its completion counts the
-// bytes on the destination's mbarrier `cbar` (shared::cluster address).  No multicast.
+// bytes on the destination's mbarrier `cbar` (shared::cluster address); one destination.
 __device__ __forceinline__ void bulk_s2cluster(uint32_t cdst, const void *src, uint32_t bytes, uint32_t cbar)
 {
     asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
