@@ -75,3 +75,31 @@ def test_split_equals_fused_and_meets_the_bars(case):
         assert np.abs(og - orf).max() <= OUT_MAXABS
         assert _rel(og, orf) <= OUT_REL
     assert _rel(fsp.numpy().astype(np.float64), fin_r) <= FIN_REL
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("layout,final_dtype", [("vk", torch.float32), ("kv", torch.bfloat16)])
+def test_split_state_variants_equal_fused(layout, final_dtype):
+    """The state I/O variants (S[v][k] layout, bf16 final state) go through the same
+    state pass on CTA 0 of the split kernel: identical bits to the fused schedule."""
+    w = ki.Workload("split_ex", B=2, T=300, H=3, init_state="f32")
+    inp = ki.make_inputs(w, 13)
+    d = lambda t: t.to("cuda")
+    init = d(inp.initial_state)
+    if layout == "vk":
+        init = init.transpose(-1, -2).contiguous()
+    res = []
+    for sch in ("fused", "split"):
+        prev = kda.kda_set_schedule(sch)
+        try:
+            o, f = kda.kda_fwd_ex(d(inp.q), d(inp.k), d(inp.v), d(inp.g), d(inp.beta), inp.scale,
+                                  d(inp.A_log), d(inp.dt_bias), inp.lower_bound, initial_state=init,
+                                  state_layout=layout, final_state_dtype=final_dtype)
+            torch.cuda.synchronize()
+            assert kda.kda_last_schedule() == sch
+        finally:
+            kda.kda_set_schedule(prev)
+        assert kda.kda_device_status(reset=True) == 0
+        res.append((o.cpu(), f.cpu()))
+    assert torch.equal(res[0][0].view(torch.int16), res[1][0].view(torch.int16))
+    assert torch.equal(res[0][1], res[1][1])
