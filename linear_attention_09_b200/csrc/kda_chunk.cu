@@ -1404,6 +1404,7 @@ static void split_config(cudaLaunchConfig_t &cfg, cudaLaunchAttribute (&at)[1], 
 // chunks per unit on average; larger launches already fill the SMs with one CTA per unit.
 constexpr int64_t kSplitMinChunks = 4;
 std::atomic<int> g_schedule{KDA_SCHEDULE_AUTO};
+int g_split_clusters[64];  // per device: clusters of the split kernel resident at once, + 1 (0 = unknown)
 thread_local int g_last_schedule = KDA_SCHEDULE_FUSED;  // of this thread's last launch
 
 static bool use_split(const FwdParams &p, int64_t units)
@@ -1412,7 +1413,7 @@ static bool use_split(const FwdParams &p, int64_t units)
     if (mode == KDA_SCHEDULE_FUSED || units <= 0) return false;
     const int64_t tokens = p.B * p.T;
     if (mode == KDA_SCHEDULE_AUTO && tokens < kSplitMinChunks * C * (p.cu ? p.N : p.B)) return false;
-    static int clusters[64];  // per device: clusters of the split kernel resident at once (+1; 0 = unknown)
+    int *clusters = g_split_clusters;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
     if (clusters[dev] == 0) {
@@ -1475,8 +1476,13 @@ int launch_chunked(const FwdParams &p, cudaStream_t stream)
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute at[1];
         split_config(cfg, at, ctas, stream);
-        if (cudaLaunchKernelEx(&cfg, chunk_kernel_split, pe, tm) != cudaSuccess) return KDA_ERR_CUDA;
-        return cudaGetLastError() == cudaSuccess ? 1 : KDA_ERR_CUDA;
+        if (cudaLaunchKernelEx(&cfg, chunk_kernel_split, pe, tm) == cudaSuccess) return 1;
+        // the device refused the cluster launch (a configuration error, which does not
+        // stick): the fused kernel computes the same bits; no split launches here again
+        cudaGetLastError();
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) g_split_clusters[dev] = 1;
+        g_last_schedule = KDA_SCHEDULE_FUSED;
     }
     chunk_kernel<<<(unsigned)ctas, NT, SMEM_ALLOC, stream>>>(pe, tm);
     return cudaGetLastError() == cudaSuccess ? 1 : KDA_ERR_CUDA;
