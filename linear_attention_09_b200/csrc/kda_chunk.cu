@@ -436,10 +436,6 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             // octant sums -> chunk prefix sums and the reference values G15, G31, G47, G63
             ok = named_bar_and(BAR_IN, NT_IN, kok);
             if (!ok) break;
-            if (round == 0 && n >= 1 && tid == 0) {  // this chunk's v tile (the previous one is consumed)
-                mbar_arrive_expect_tx(&bars->v, 16384);
-                load_tile(sm + SM_V, &tm.v, &bars->v, h, ctok);
-            }
             float2 os[8];
 #pragma unroll
             for (int o = 0; o < 8; ++o) os[o] = *reinterpret_cast<const float2 *>(cx.osum + o * 128 + c0);
@@ -498,7 +494,6 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
                     st_u64(sm, SM_APA + o32[j], tf32b(kr.x), tf32b(kr.y));
                     st_u64(sm, SM_APA + 8192 + o32[j], tf32b(qr.x), tf32b(qr.y));
                     st_u64(sm, SM_APB + o32[j], tf32b(ks.x), tf32b(ks.y));
-                    const float2 gam = mul2(rho, fa);
                     float2 kp;
                     if (kBlk0) {
                         const float2 s1 = mul2(sig, fb);  // e^{G31 - G_t} <= 1
@@ -508,7 +503,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
                     } else {
                         kp = mul2(sig, fc);
                     }
-                    const float2 kg = mul2(kk, gam), qg = mul2(qv, gam), kpp = mul2(kk, kp);
+                    const float2 kg = mul2(kr, fa), qg = mul2(qr, fa), kpp = mul2(kk, kp);
                     st_u32(sm, SM_KG + rb + o16[j], pack_f16(kg.x, kg.y));
                     st_u32(sm, SM_WQ + 2 * rb + 8192 + o16[j], pack_f16(qg.x, qg.y));
                     st_u32(sm, skp + rb + o16[j], pack_f16(kpp.x, kpp.y));
@@ -523,8 +518,6 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             if (lane == 0) mbar_arrive(&bars->ops);
             ok = named_bar_and(BAR_IN, NT_IN, wok);
             if (!ok) break;
-            // this round's box of q, k, g is consumed: prefetch the next chunk's
-            if (tid == 0 && has_next) load_qkg_box(sm, tm, &bars->qkg[round], h, cx.tok0 + (int64_t)uc(n + 1) * C, round);
         }
         if (!ok) break;
         // ---- while the round-1 A/P product runs: the next chunk's round-0 gate (its
@@ -826,7 +819,7 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
 // `mma_in`.  The in-chunk warps never stall on issuing.
 // =====================================================================================
 template <Mode M>
-__device__ void mma_role(const Ctx &cx)
+__device__ void mma_role(const TMaps &tm, const Ctx &cx)
 {
     if ((threadIdx.x & 31) != 0) return;
     uint8_t *sm = cx.sm;
@@ -854,6 +847,17 @@ __device__ void mma_role(const Ctx &cx)
                 mma_tf32_ss(tb + TM_AP, da, db, idap, (round > 0 || st > 0) ? 1u : 0u);
             }
             mma_commit(&bars->mma_in);
+            // The round's operands are written, so every in-chunk thread is done with this
+            // round's box of q, k and g: the next own chunk's box goes in (off the in-chunk
+            // threads' path, while the product runs).  At round 0 the previous chunk's u
+            // product has completed (the in-chunk threads waited for it before handing the
+            // chunk over), so this chunk's v tile may replace the last one.
+            if (n + 1 < nown)
+                load_qkg_box(sm, tm, &bars->qkg[round], cx.h, cx.tok0 + (int64_t)(f + S * (n + 1)) * C, round);
+            if (round == 0 && n >= 1) {
+                mbar_arrive_expect_tx(&bars->v, 16384);
+                load_tile(sm + SM_V, &tm.v, &bars->v, cx.h, cx.tok0 + (int64_t)(f + S * n) * C);
+            }
         }
         if (!wait_or_flag(&bars->ops, (ops_cnt++) & 1u, 12)) return;
         if (!wait_or_flag(&bars->v, par, 2)) return;
@@ -1284,7 +1288,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
 
     if (warp < NT_IN / 32) in_chunk_role<kFused>(p, tm, cx);
     else if (warp < (NT_IN + NT_ST) / 32) state_role<kFused>(p, cx);
-    else mma_role<kFused>(cx);
+    else mma_role<kFused>(tm, cx);
 
     tc_fence_before();
     __syncthreads();
@@ -1348,7 +1352,7 @@ chunk_kernel_split(const FwdParams p, const __grid_constant__ TMaps tm)
             }
             if (warp < NT_IN / 32) in_chunk_role<kProducer>(p, tm, cx);
             else if (warp < (NT_IN + NT_ST) / 32) u_send_role(cx);
-            else mma_role<kProducer>(cx);
+            else mma_role<kProducer>(tm, cx);
         }
     }
 
