@@ -103,6 +103,8 @@ constexpr int LST = 68;                     // row stride (floats) of the solve 
 // ---- tensor memory columns (512 allocated) ----
 constexpr uint32_t TM_AP = 0;    // A/P product, lanes = rows, 96 cols        (in-chunk role)
 constexpr uint32_t TM_W = 0;     // w^T: lanes = channel, cols = token (64)   (aliases AP)
+constexpr uint32_t TM_G = 96;    // round-1 gate G of the in-chunk threads (32) (state -> in-chunk)
+constexpr int64_t kGateHandoffTokens = 1024;  // mean tokens per unit from which it is used
 constexpr uint32_t TM_S = 128;   // state S / tau, lane v, column k  (128)    (state role)
 constexpr uint32_t TM_D1 = 256;  // [w S~^T | (q^ e^G) S~^T] per lane v (128); cols 0..31
                                  //   then hold U~^T (fp16 pairs)
@@ -192,6 +194,8 @@ struct Bars {
     uint64_t u_free;   // u^T read out of TMEM                 (128 arrivals)
     uint64_t ops;      // operands of the next in-chunk product written (one arrival per
                        // in-chunk warp); the issue warp waits on it
+    uint64_t gate_rdy;  // fused: chunk n's round-1 gate (n >= 2) is in TM_G   (1 arrival)
+    uint64_t gate_free; // fused: TM_G and the round-1 octant sums read   (one arrival per in-chunk warp)
     // split kernel, CTAs 1..3:
     uint64_t u_rdy;     // u^T of the chunk complete in TMEM              (commit)
     uint64_t slot_free; // CTA 0 released the slot this CTA fills next    (1 remote arrival)
@@ -267,7 +271,7 @@ __device__ __forceinline__ void load_tile(uint8_t *dst, const CUtensorMap *tm, u
 // decay-weighted products A and P (tf32), the triangular solve for T, and the
 // products w = T (k^ e^G), u = T v; hands [w ; q^ e^G], k', P, u^T and gamma over.
 // =====================================================================================
-template <Mode M>
+template <Mode M, bool GH = false>
 __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx)
 {
     uint8_t *sm = cx.sm;
@@ -414,9 +418,19 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             const int c0 = 64 * round + 2 * cp;  // first channel of the pair
             const uint32_t rb = (uint32_t)round * 8192u;
             float2 G[8];  // in-chunk cumulative log2-decay of the pair, tokens t0 .. t0+7
+            bool gaok = true;
             if (round == 0) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) G[j] = G0[j];
+            } else if (GH && n >= 2) {
+                // the state warps computed this round's gate during the previous chunk
+                gaok = wait_or_flag(&bars->gate_rdy, par, 23);
+                tc_fence_after();
+                uint32_t gr[16];
+                tmem_ld16(tb + lq + TM_G + 16 * (warp >> 2), gr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 8; ++j) G[j] = make_float2(__uint_as_float(gr[2 * j]), __uint_as_float(gr[2 * j + 1]));
             } else {
                 gate_round(1, L, G);
             }
@@ -434,11 +448,16 @@ __device__ void in_chunk_role(const FwdParams &p, const TMaps &tm, const Ctx &cx
             }
 
             // octant sums -> chunk prefix sums and the reference values G15, G31, G47, G63
-            ok = named_bar_and(BAR_IN, NT_IN, kok);
+            ok = named_bar_and(BAR_IN, NT_IN, kok && gaok);
             if (!ok) break;
             float2 os[8];
 #pragma unroll
             for (int o = 0; o < 8; ++o) os[o] = *reinterpret_cast<const float2 *>(cx.osum + o * 128 + c0);
+            if (GH && round == 1 && n >= 2) {  // TM_G and the round-1 octant sums are read
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->gate_free);
+            }
             float2 pre = make_float2(0.f, 0.f);
 #pragma unroll
             for (int o = 0; o < 8; ++o)
@@ -922,7 +941,7 @@ __device__ void u_send_role(const Ctx &cx)
 //   -> U~ = U / tau' -> TM_S <- (gamma * TM_S) tau / tau' -> MMA2: TM_S += U~^T k',
 //   D3 = U~^T P^T -> out = scale (sigma D1[:,64:128] + tau' D3).
 // =====================================================================================
-template <Mode M>
+template <Mode M, bool GH = false>
 __device__ void state_role(const FwdParams &p, const Ctx &cx)
 {
     uint8_t *sm = cx.sm;
@@ -972,6 +991,53 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
         }
     }
     tmem_wait_st();
+
+    // Fused kernel: the round-1 gate of chunk m >= 2 for the in-chunk threads that share
+    // this thread's TMEM lane (in-chunk warps q and q + 4, lane l: octants q and q + 4 of
+    // the channel pair 64 + 2 l, 65 + 2 l), the same arithmetic as theirs, into TM_G (warp
+    // q reads columns 0..15, warp q + 4 columns 16..31) and the round-1 octant sums,
+    // computed after this role's work on chunk m - 2, in its idle time, once the in-chunk
+    // warps have read chunk m - 1's (gate_free) and chunk m's g box 1 is in.  The gates
+    // of chunks 0 and 1 stay with the in-chunk warps: this role is still loading the
+    // initial state then, and a unit's first chunks would wait for it.
+    auto gate_r1 = [&](int m) -> bool {
+        bool w = m < 3 || wait_or_flag(&bars->gate_free, (uint32_t)(m - 3) & 1u, 24);
+        w = w && wait_or_flag(&bars->qkg[1], (uint32_t)m & 1u, 25);
+        if (!named_bar_and(BAR_ST, NT_ST, w)) return false;
+        tc_fence_after();
+        const int q = warp & 3, l = tid & 31, c0 = 64 + 2 * l;
+        const int64_t rem = cx.len - (int64_t)m * C;
+        const int Lc = (int)(rem < C ? rem : C);
+        const float aexp = ex2(p.A_log[h] * kLog2e), a2 = aexp * kLog2e, lb2 = p.lower_bound * kLog2e;
+        const float2 dtb = *reinterpret_cast<const float2 *>(cx.dtb_s + c0);
+        uint32_t r[2][16];
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl) {
+            const int oc = q + 4 * hl, t0 = 8 * oc;
+            float2 run = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float2 g2 = bf2x2(*reinterpret_cast<const uint32_t *>(
+                    sm + SM_G + 8192u + sw((uint32_t)(t0 + j), (uint32_t)l * 4u)));
+                const float x0 = g2.x + dtb.x, x1 = g2.y + dtb.y;
+                const float e0 = lg2(1.f + ex2(-fabsf(x0) * kLog2e));
+                const float e1 = lg2(1.f + ex2(-fabsf(x1) * kLog2e));
+                const bool valid = t0 + j < Lc;
+                run.x += valid ? fmaxf(lb2, -a2 * fmaxf(x0, 0.f) - aexp * e0) : 0.f;
+                run.y += valid ? fmaxf(lb2, -a2 * fmaxf(x1, 0.f) - aexp * e1) : 0.f;
+                r[hl][2 * j] = __float_as_uint(run.x);
+                r[hl][2 * j + 1] = __float_as_uint(run.y);
+            }
+            *reinterpret_cast<float2 *>(cx.osum + oc * 128 + c0) = run;
+        }
+        tmem_st16(tb + lq + TM_G, r[0]);
+        tmem_st16(tb + lq + TM_G + 16, r[1]);
+        tmem_wait_st();
+        tc_fence_before();
+        named_bar(BAR_ST, NT_ST);
+        if (leader) mbar_arrive(&bars->gate_rdy);
+        return true;
+    };
 
     for (int n = 0; n < cx.nchunks && ok; ++n) {
         const int64_t ctok = cx.tok0 + (int64_t)n * C;
@@ -1146,6 +1212,9 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
                 }
             }
         }
+        if constexpr (GH) {  // the round-1 gate of the chunk after next
+            if (n + 2 < cx.nchunks && !(ok = gate_r1(n + 2))) break;
+        }
     }
 
     // ---- final state = tau TM_S (column v), fp32 or bf16 (round to nearest even) ----
@@ -1235,6 +1304,8 @@ __device__ __forceinline__ void init_bars(Bars *b)
     mbar_init(&b->kp_free[1], 1);
     mbar_init(&b->u_free, NT_ST);
     mbar_init(&b->ops, NT_IN / 32);
+    mbar_init(&b->gate_rdy, 1);
+    mbar_init(&b->gate_free, NT_IN / 32);
     mbar_init(&b->u_rdy, 1);
     mbar_init(&b->slot_free, 1);
 }
@@ -1247,6 +1318,8 @@ __device__ __forceinline__ void read_abort(const FwdParams &p)
     s_abort = e != 0 && ((uint32_t)e >> 8) == p.epoch;
 }
 
+// GH: the state role computes the round-1 gates of chunks 2.. (launches of long units)
+template <bool GH>
 __global__ void __launch_bounds__(NT, 1)
 chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
 {
@@ -1286,8 +1359,8 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
         load_tile(sm + SM_V, &tm.v, &cx.bars->v, cx.h, cx.tok0);
     }
 
-    if (warp < NT_IN / 32) in_chunk_role<kFused>(p, tm, cx);
-    else if (warp < (NT_IN + NT_ST) / 32) state_role<kFused>(p, cx);
+    if (warp < NT_IN / 32) in_chunk_role<kFused, GH>(p, tm, cx);
+    else if (warp < (NT_IN + NT_ST) / 32) state_role<kFused, GH>(p, cx);
     else mma_role<kFused>(tm, cx);
 
     tc_fence_before();
@@ -1461,8 +1534,10 @@ int launch_chunked(const FwdParams &p, cudaStream_t stream)
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return KDA_ERR_CUDA;
     }
-    static int attr_set[64];
-    if (!set_smem_limit_once(chunk_kernel, SMEM_ALLOC, attr_set)) return KDA_ERR_CUDA;
+    static int attr_plain[64], attr_gh[64];
+    if (!set_smem_limit_once(chunk_kernel<false>, SMEM_ALLOC, attr_plain) ||
+        !set_smem_limit_once(chunk_kernel<true>, SMEM_ALLOC, attr_gh))
+        return KDA_ERR_CUDA;
     // the launch's epoch: 24 bits, never 0 (an error word of 0 means no error)
     static std::atomic<uint32_t> epochs{0};
     FwdParams pe = p;
@@ -1488,7 +1563,13 @@ int launch_chunked(const FwdParams &p, cudaStream_t stream)
         if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) g_split_clusters[dev] = 1;
         g_last_schedule = KDA_SCHEDULE_FUSED;
     }
-    chunk_kernel<<<(unsigned)ctas, NT, SMEM_ALLOC, stream>>>(pe, tm);
+    // units averaging kGateHandoffTokens tokens or more: the state role takes the
+    // round-1 gates (measured faster there, and slower for units of a few chunks)
+    const int64_t avg_tokens = p.cu ? (p.B * p.T) / (p.N > 0 ? p.N : 1) : p.T;
+    if (avg_tokens >= kGateHandoffTokens)
+        chunk_kernel<true><<<(unsigned)ctas, NT, SMEM_ALLOC, stream>>>(pe, tm);
+    else
+        chunk_kernel<false><<<(unsigned)ctas, NT, SMEM_ALLOC, stream>>>(pe, tm);
     return cudaGetLastError() == cudaSuccess ? 1 : KDA_ERR_CUDA;
 }
 

@@ -3,7 +3,9 @@ third chunk, one runs the state pass) against the fused one (one CTA per unit).
 
 Both run the same arithmetic in the same order, and the data that crosses between the
 CTAs is copied bit for bit, so out and the final state must be identical; the split
-results are also held to the oracle's bars.  Forced splits cover units with fewer
+results are also held to the oracle's bars.  Cases of long units also compare the fused
+kernel variant whose state warps compute the round-1 gates against the split kernel
+(which does not).  Forced splits cover units with fewer
 chunks than producing CTAs (some CTAs get none) and empty varlen sequences.
 """
 import numpy as np
@@ -54,6 +56,10 @@ CASES = [
     dict(B=1, T=130, H=2, init="bf16", lengths=None),      # three chunks, the last partial
     dict(B=1, T=1, H=2, init="f32", lengths=None),
     dict(B=1, T=0, H=2, init="f32", lengths=[300, 0, 65, 1000, 129]),
+    # units of >= 1024 tokens on average: the fused schedule runs the kernel whose state
+    # warps compute the round-1 gates from chunk 2 on
+    dict(B=1, T=1300, H=3, init="f32", lengths=None),
+    dict(B=1, T=0, H=2, init="bf16", lengths=[1300, 2, 2000]),
 ]
 
 
