@@ -35,6 +35,10 @@
 // column v on the 128 TMEM lanes), so S^T and U^T are tensor-core A operands
 // read straight from TMEM, and thread v owns value column v.
 //
+// Launches of long units (>= 1024 tokens on average) run an instantiation in which the
+// state warps, idle part of each chunk, also compute the round-1 gate of the chunk
+// after next and hand it to the in-chunk warps through TMEM.
+//
 // Split schedule (few units, many idle SMs): a cluster of 4 CTAs per (sequence,
 // head).  CTAs 1..3 each run the in-chunk work for every third chunk and send its
 // results ([w ; q^ e^G], k', P, gamma by a bulk copy, u^T by stores) into one of two
