@@ -66,6 +66,8 @@ def parse():
     ap.add_argument("--seqlen", type=int, default=None)
     # the decode step (one token per sequence, state in HBM) instead of the prefill
     ap.add_argument("--op", default="prefill", choices=["prefill", "decode", "backward"])
+    ap.add_argument("--bwd-schedule", default="chunked", choices=["chunked", "token"],
+                    help="schedule of kda_bwd for --op backward")
     ap.add_argument("--decode-seqs", type=int, default=256)
     # time one of the five parity workloads (kda_inputs recipe) instead of the headline
     ap.add_argument("--config-id", type=int, default=None, choices=[0, 1, 2, 3, 4])
@@ -383,7 +385,6 @@ BWD_BYTES_PER_TOKEN_HEAD = 5 * 256 + 2 + 4 * 512 + 4
 BWD_FLOPS_PER_TOKEN_HEAD = 17 * 128 * 128
 # fp32 FMA peak of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1965 MHz
 FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-BWD_KERNEL_SRC = ["linear_attention_09_b200/csrc/kda_backward.cu"]
 
 
 def run_backward_bench(args, world, rank, local):
@@ -403,6 +404,7 @@ def run_backward_bench(args, world, rank, local):
     dO = dO.to(torch.bfloat16)
     ws = torch.empty(kda.kda_bwd_workspace_size(B, T, H), dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
+    kda.kda_set_bwd_schedule(args.bwd_schedule)
 
     def step():
         kda.kda_bwd(**inp, d_out=dO, workspace=ws, stream=stream)
@@ -434,14 +436,14 @@ def run_backward_bench(args, world, rank, local):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16-in/fp32", "data": "synthetic",
             "config": {"workload": f"bwd_B{B}_T{T}_H{H}_g2", "global_batch": B * world,
-                       "seq_len": T, "heads": H,
+                       "seq_len": T, "heads": H, "schedule": args.bwd_schedule,
                        "l2": f"inputs + gradients {bytes_launch / 1e9:.1f} GB per rank > 126 MB L2"},
             "roofline": {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS,
                          "unit": "TFLOP/s", "frac": achieved / FP32_PEAK_TFLOPS, "traffic": None,
                          "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
                          "alg_flops_per_launch": flops, "alg_bytes_per_launch": bytes_launch,
                          "hbm_gbs_algorithmic": bytes_launch / (ms_local / args.steps / 1e3) / 1e9,
-                         "kernel": "bwd_kernel"},
+                         "kernel": "bwdc_kernel" if args.bwd_schedule == "chunked" else "bwd_kernel"},
             "clocks": clk.summary(), "gpu_launches": launches * args.steps}), flush=True)
     return 0
 

@@ -313,6 +313,19 @@ int kda_device_status(int reset);
 #define KDA_SCHEDULE_SPLIT 2
 int kda_set_schedule(int mode);
 
+/* Schedule of the backward pass (kda_bwd, kda_bwd_noalloc), process-wide; returns the
+ * previous one, or KDA_ERR_ARG:
+ *   KDA_BWD_CHUNKED (default) the forward kernel stores the fp32 state before every
+ *                   64-token chunk in the workspace (one launch), then one CTA per
+ *                   (sequence, head) runs the chunks in reverse in the chunked matrix
+ *                   form (the adjoint of the WY form of the forward);
+ *   KDA_BWD_TOKEN   one CTA per (sequence, head) sweeps the token recurrence forward
+ *                   for its own fp32 checkpoints and reverses it token by token.
+ * Both take the same workspace and meet the same tolerances; their rounding differs. */
+#define KDA_BWD_CHUNKED 0
+#define KDA_BWD_TOKEN 1
+int kda_set_bwd_schedule(int mode);
+
 /* Schedule (KDA_SCHEDULE_FUSED or KDA_SCHEDULE_SPLIT) of the last forward launch this
  * host thread enqueued (for reports). */
 int kda_last_schedule(void);

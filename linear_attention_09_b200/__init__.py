@@ -9,7 +9,8 @@ The functions mirror the C ABI in ``include/kda.h``:
   kda_bwd_workspace_size,
   kda_fwd_host,
   kda_fwd_host_workspace_size, kda_set_checks, kda_strerror, kda_last_launch_count,
-  kda_device_status, kda_inject_error, kda_set_schedule, kda_last_schedule.
+  kda_device_status, kda_inject_error, kda_set_schedule, kda_last_schedule,
+  kda_set_bwd_schedule.
 """
 from __future__ import annotations
 
@@ -88,6 +89,8 @@ def lib() -> ctypes.CDLL:
             L.kda_set_schedule.restype = I
             L.kda_last_schedule.argtypes = []
             L.kda_last_schedule.restype = I
+            L.kda_set_bwd_schedule.argtypes = [I]
+            L.kda_set_bwd_schedule.restype = I
             _lib = L
     return _lib
 
@@ -128,6 +131,20 @@ def kda_set_schedule(mode) -> str:
 def kda_last_schedule() -> str:
     """Schedule ("fused" or "split") of this thread's last forward launch."""
     return {v: k for k, v in _SCHEDULES.items()}[int(lib().kda_last_schedule())]
+
+
+KDA_BWD_CHUNKED, KDA_BWD_TOKEN = 0, 1
+_BWD_SCHEDULES = {"chunked": KDA_BWD_CHUNKED, "token": KDA_BWD_TOKEN}
+
+
+def kda_set_bwd_schedule(mode) -> str:
+    """Backward pass schedule, process-wide: "chunked" (default: the forward kernel's
+    chunk checkpoints, then the chunked matrix form in reverse) or "token" (the token
+    recurrence reversed step by step); returns the previous one."""
+    rc = lib().kda_set_bwd_schedule(_BWD_SCHEDULES[mode] if isinstance(mode, str) else int(mode))
+    if rc < 0:
+        raise KDAError(rc, "kda_set_bwd_schedule")
+    return {v: k for k, v in _BWD_SCHEDULES.items()}[rc]
 
 
 def kda_inject_error(code: int) -> None:

@@ -182,6 +182,8 @@ extern "C" int kda_set_schedule(int mode) { return kda::chunked_set_schedule(mod
 
 extern "C" int kda_last_schedule(void) { return kda::chunked_last_schedule(); }
 
+extern "C" int kda_set_bwd_schedule(int mode) { return kda::bwd_set_schedule(mode); }
+
 extern "C" int kda_fwd_ex(const kda_bf16 *q, const kda_bf16 *k, const kda_bf16 *v,
                           const kda_bf16 *g, const kda_bf16 *beta, float scale,
                           const float *A_log, const float *dt_bias, float lower_bound,

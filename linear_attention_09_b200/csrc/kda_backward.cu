@@ -574,13 +574,24 @@ size_t bwd_layout(int64_t total_tokens, int64_t N, int64_t H, BwdLayout *out)
     const int64_t units = N * H;
     l.grid = (int)(units < kBwdMaxCtas ? units : kBwdMaxCtas);
     l.ckpt_bytes = up((size_t)(total_tokens / CH + N + 1) * H * STATE * 4);
-    l.scratch_bytes = up((size_t)l.grid * NSUB * STATE * 4);
+    // per CTA: the token schedule's sub-chunk states, or the chunked schedule's tiles
+    const size_t per_cta = (size_t)NSUB * STATE * 4 > bwd_chunked_scratch_bytes_per_cta()
+                               ? (size_t)NSUB * STATE * 4
+                               : bwd_chunked_scratch_bytes_per_cta();
+    l.scratch_bytes = up((size_t)l.grid * per_cta);
     l.part_bytes = up((size_t)units * (kHead + 1) * 4);
     if (out) *out = l;
     return l.ckpt_bytes + l.scratch_bytes + l.part_bytes;
 }
 
-int launch_backward(const BwdParams &p, const BwdLayout &l, cudaStream_t stream)
+int launch_param_reduce(const BwdParams &p, cudaStream_t stream)
+{
+    param_reduce_kernel<<<(unsigned)p.H, kHead + 1, 0, stream>>>(p.part, p.N, p.H, p.dA_log,
+                                                                 p.ddt_bias);
+    return cudaGetLastError() == cudaSuccess ? 1 : KDA_ERR_CUDA;
+}
+
+int launch_backward_token(const BwdParams &p, const BwdLayout &l, cudaStream_t stream)
 {
     const int64_t units = p.N * p.H;
     if (units <= 0) return 0;
@@ -589,9 +600,8 @@ int launch_backward(const BwdParams &p, const BwdLayout &l, cudaStream_t stream)
     if (!set_smem_limit_once(bwd_kernel, smem, smem_set)) return KDA_ERR_CUDA;
     bwd_kernel<<<l.grid, BT, smem, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
-    param_reduce_kernel<<<(unsigned)p.H, kHead + 1, 0, stream>>>(p.part, p.N, p.H, p.dA_log,
-                                                                 p.ddt_bias);
-    return cudaGetLastError() == cudaSuccess ? 2 : KDA_ERR_CUDA;
+    const int n = launch_param_reduce(p, stream);
+    return n < 0 ? n : 1 + n;
 }
 
 }  // namespace kda

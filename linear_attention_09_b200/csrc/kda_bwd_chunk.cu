@@ -1,0 +1,787 @@
+// KDA backward pass for sm_100a in the chunked form: the adjoint of the per-chunk
+// matrix form of the forward, over 64-token chunks in reverse.
+//
+// Forward of one chunk of L tokens from state S0 (K x V, S[k][v]), on the activations
+// q^, k^, b, lam, with G the in-chunk inclusive cumulative sum of lam, Gam = e^G and
+// GL = G[L-1] (the chunked form of the recurrence of the FlashKDA pages, 7minutos.es
+// "¿Qué es la atención Kimi Delta...?"):
+//   A_ij = sum_c k^_i k^_j e^(G_i - G_j) (j < i),  P_ij = same with q^_i (j <= i)
+//   M = I + Diag(b) A,  T = M^-1 Diag(b),  Y = v - (k^ Gam) S0,  U = T Y
+//   O = scale [(q^ Gam) S0 + P U],  S_end = Diag(e^GL) S0 + K'^T U,  K' = k^ e^(GL - G).
+// Reverse of the chunk, given dO and dS (= dL/dS_end):
+//   dU = scale P^T dO + K' dS;  dY = T^T dU = dv;  dT = dU Y^T (lower)
+//   dS0 = scale (q^ Gam)^T dO + Diag(e^GL) dS - (k^ Gam)^T dY          (passed to chunk n-1)
+//   d(k^ Gam) = -dY S0^T;  d(q^ Gam) = scale dO S0^T;  dP = scale dO U^T (lower)
+//   dK' = U dS^T;  d(e^GL) contributes rowsum(dS o S0) e^GL to dG[L-1]
+//   dM^-1 = dT Diag(b), db_j = sum_i dT_ij M^-1_ij;  dM = -M^-T dM^-1 M^-T
+//   dA = Diag(b) dM (strict lower), db_i += sum_j dM_ij A_ij
+// then through the decay-weighted products A and P into dq^, dk^ and dG (the factor
+// e^(G_i - G_j) evaluated per channel, so that no factor leaves the fp32 range), and
+// dlam = the reverse cumulative sum of dG over the chunk, followed by the gradients of
+// the L2 norms, the sigmoid and the gate as in the token-level backward.
+//
+// The states before every chunk come from the forward kernel (its checkpoint
+// instantiation, one launch before this one).  Schedule: one CTA of 512 threads per
+// (sequence, head), persistent over the units, chunks in reverse; everything is fp32
+// on the CUDA cores.  The activations (q^, k^, G; channel-major) and the 64 x 64
+// matrices live in shared memory; the 64 x 128 tiles of a chunk (dO, Y, U, dU, dY,
+// their transposes, k^ Gam, q^ Gam, K', the gradient accumulators) and dS live in a
+// per-CTA scratch region of global memory that stays in L2 and L1.  Every product is
+// a register-blocked loop whose second operand is read along its rows by consecutive
+// lanes, so each operand that appears in both orientations is stored in both.
+#include <atomic>
+#include <cstddef>
+
+#include "kda.h"
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int CC = 64;             // tokens per chunk
+constexpr int CT = 512;            // threads per CTA
+constexpr int CW = CT / 32;        // warps
+constexpr int LDT = 65;            // row stride of the channel-major tiles and 64 x 64 matrices
+constexpr int LDE = 129;           // row stride of the token-major epilogue tiles
+constexpr int ST = kHead * kHead;  // floats of one state
+constexpr int TILE = CC * kHead;   // floats of one 64 x 128 tile
+constexpr unsigned FULL = 0xffffffffu;
+constexpr float kL2e = 1.4426950408889634f;
+
+struct CSmem {
+    float QT[kHead][LDT];  // q^   [channel][token]
+    float KT[kHead][LDT];  // k^
+    float GT[kHead][LDT];  // G log2(e): in-chunk inclusive cumulative sum of the log-decay
+    union {
+        struct {
+            float A[CC][LDT];   // A (strict lower part; the rest 0)
+            float PT[CC][LDT];  // P^T: PT[t][i] = P[i][t]; later W = dM^-1 M^-T
+            float Mi[CC][LDT];  // M^-1 (unit lower)
+            float X[CC][LDT];   // dT (lower), then dA (strict lower)
+            float dP[CC][LDT];  // dP (lower)
+        } m;
+        struct {
+            float o0[CC][LDE], o1[CC][LDE];  // [token][channel] staging of the outputs
+        } e;
+    } u;
+    float b[CC], rq[CC], rk[CC], db[CC];
+    float eGL[kHead], G2L[kHead], dGL[kHead], extra[kHead], dtb[kHead];
+    float red[2][CW][CC];
+    float pacc[CW][kHead + 1];  // per-warp partial ddt_bias (0..127) and dA_log (128)
+};
+
+// Per-CTA scratch (floats): the tiles in the order of these offsets.
+enum : int {
+    S_DO = 0, S_DOT = TILE, S_KGT = 2 * TILE, S_QGT = 3 * TILE, S_KPT = 4 * TILE, S_Y = 5 * TILE,
+    S_YT = 6 * TILE, S_U = 7 * TILE, S_UT = 8 * TILE, S_DU = 9 * TILE, S_DY = 10 * TILE,
+    S_DYT = 11 * TILE, S_DKT = 12 * TILE, S_DQT = 13 * TILE, S_DGT = 14 * TILE, S_DS = 15 * TILE,
+    S_FLOATS = 15 * TILE + ST
+};
+
+__device__ __forceinline__ float ex2f(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float bf(const __nv_bfloat16 *p, size_t i) { return __bfloat162float(p[i]); }
+
+__device__ __forceinline__ float wsum(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(FULL, x, o);
+    return x;
+}
+
+// acc[r][j] += sum_{k in [k0, k1)} fa(r, k) fb(k, j): fa is the same for every lane of
+// the warp (a broadcast), fb(k, j) reads column lane + 32 j of row k.
+template <int R, int J, class FA, class FB>
+__device__ __forceinline__ void mm(float (&acc)[R][J], int k0, int k1, FA fa, FB fb)
+{
+#pragma unroll 2
+    for (int k = k0; k < k1; ++k) {
+        float a[R], b[J];
+#pragma unroll
+        for (int r = 0; r < R; ++r) a[r] = fa(r, k);
+#pragma unroll
+        for (int j = 0; j < J; ++j) b[j] = fb(k, j);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int j = 0; j < J; ++j) acc[r][j] = fmaf(a[r], b[j], acc[r][j]);
+    }
+}
+
+__global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
+{
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    CSmem &sm = *reinterpret_cast<CSmem *>(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float *scr = p.scratch + (size_t)blockIdx.x * S_FLOATS;
+    float *DO = scr + S_DO, *DOT = scr + S_DOT, *KGT = scr + S_KGT, *QGT = scr + S_QGT;
+    float *KPT = scr + S_KPT, *Y = scr + S_Y, *YT = scr + S_YT, *U = scr + S_U, *UT = scr + S_UT;
+    float *DU = scr + S_DU, *DY = scr + S_DY, *DYT = scr + S_DYT, *DKT = scr + S_DKT;
+    float *DQT = scr + S_DQT, *DGT = scr + S_DGT, *DS = scr + S_DS;
+    const int r0 = 4 * warp;  // rows of this warp in the 64-row products
+    const int c0 = 8 * warp;  // rows (channels) of this warp in the 128-row products
+    const int64_t units = p.N * p.H;
+    const size_t rs = (size_t)p.H * kHead;  // row stride of the [tokens, H, 128] tensors
+
+    for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+        const int64_t sq = u / p.H, h = u % p.H;
+        const int64_t bos = p.cu ? p.cu[sq] : sq * p.T;
+        int64_t len = p.cu ? p.cu[sq + 1] - bos : p.T;
+        if (len < 0) len = 0;
+        const int64_t nch = (len + CC - 1) / CC;
+        const float ea = expf(p.A_log[h]);
+        const float *ckb = p.ckpt + (size_t)((bos / CC + sq) * p.H + h) * ST;
+        const size_t ckstride = (size_t)p.H * ST;
+        const size_t st_off = (size_t)u * ST;
+        const size_t hb = (size_t)h * kHead;
+
+        __syncthreads();  // the previous unit's readers of dtb / pacc / DS are done
+        if (tid < kHead) sm.dtb[tid] = p.dt_bias[h * kHead + tid];
+        for (int i = tid; i < CW * (kHead + 1); i += CT) (&sm.pacc[0][0])[i] = 0.f;
+        for (int i = tid; i < ST; i += CT) DS[i] = p.dfinal ? p.dfinal[st_off + i] : 0.f;
+        __syncthreads();
+
+        for (int64_t n = nch - 1; n >= 0; --n) {
+            const int64_t tok = bos + n * CC;
+            const int L = (int)(len - n * CC < CC ? len - n * CC : CC);
+            const float *S0 = ckb + n * ckstride;
+
+            // ---- 1. activations of the chunk's tokens (zero past L), dO ----
+#pragma unroll 1
+            for (int i = 0; i < CC / CW; ++i) {
+                const int t = warp + CW * i;
+                const bool in = t < L;
+                const size_t row = (size_t)(tok + t) * rs + hb;
+                float qv[4], kv[4], gv[4], s2q = 0.f, s2k = 0.f;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int c = lane + 32 * m;
+                    qv[m] = in ? bf(p.q, row + c) : 0.f;
+                    kv[m] = in ? bf(p.k, row + c) : 0.f;
+                    gv[m] = in ? bf(p.g, row + c) : 0.f;
+                    s2q = fmaf(qv[m], qv[m], s2q);
+                    s2k = fmaf(kv[m], kv[m], s2k);
+                }
+                const float rq = rsqrtf(wsum(s2q) + 1e-6f), rk = rsqrtf(wsum(s2k) + 1e-6f);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int c = lane + 32 * m;
+                    float lam2 = 0.f;
+                    if (in) {
+                        const float x = gv[m] + sm.dtb[c];
+                        const float sp = fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));  // softplus
+                        lam2 = fmaxf(p.lower_bound, -ea * sp) * kL2e;
+                    }
+                    sm.QT[c][t] = qv[m] * rq;
+                    sm.KT[c][t] = kv[m] * rk;
+                    sm.GT[c][t] = lam2;
+                    const float d = in ? bf(p.dout, row + c) : 0.f;
+                    DO[t * kHead + c] = d;
+                    DOT[c * CC + t] = d;
+                }
+                if (lane == 0) {
+                    sm.b[t] = in ? 1.f / (1.f + expf(-bf(p.beta, (size_t)(tok + t) * p.H + h))) : 0.f;
+                    sm.rq[t] = rq;
+                    sm.rk[t] = rk;
+                }
+            }
+            for (int i = tid; i < CC * LDT; i += CT) {
+                (&sm.u.m.A[0][0])[i] = 0.f;
+                (&sm.u.m.PT[0][0])[i] = 0.f;
+            }
+            __syncthreads();
+
+            // ---- 2. G: inclusive cumulative sum over the chunk (log2 units) ----
+            if (tid < kHead) {
+                float run = 0.f;
+                for (int t = 0; t < CC; ++t) {
+                    run += sm.GT[tid][t];
+                    sm.GT[tid][t] = run;
+                }
+                sm.G2L[tid] = sm.GT[tid][L - 1];
+                sm.eGL[tid] = ex2f(sm.G2L[tid]);
+            }
+            __syncthreads();
+
+            // ---- 3. (k^ Gam)^T, (q^ Gam)^T, K'^T ----
+            for (int e = tid; e < TILE; e += CT) {
+                const int c = e >> 6, t = e & (CC - 1);
+                const float g2 = sm.GT[c][t], gam = ex2f(g2), kh = sm.KT[c][t];
+                KGT[e] = kh * gam;
+                QGT[e] = sm.QT[c][t] * gam;
+                KPT[e] = kh * ex2f(sm.G2L[c] - g2);
+            }
+
+            // ---- 4. A and P in 4 x 4 blocks (a warp per block, lanes over channels) ----
+            for (int blk = warp; blk < 136; blk += CW) {
+                int bi = 0, bj = blk;
+                while (bj > bi) {
+                    bj -= bi + 1;
+                    ++bi;
+                }
+                const int i0 = 4 * bi, j0 = 4 * bj;
+                float v[32];
+#pragma unroll
+                for (int x = 0; x < 32; ++x) v[x] = 0.f;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int c = lane + 32 * m;
+                    float gi[4], ki[4], qi[4], gj[4], kj[4];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        gi[x] = sm.GT[c][i0 + x];
+                        ki[x] = sm.KT[c][i0 + x];
+                        qi[x] = sm.QT[c][i0 + x];
+                        gj[x] = sm.GT[c][j0 + x];
+                        kj[x] = sm.KT[c][j0 + x];
+                    }
+#pragma unroll
+                    for (int ii = 0; ii < 4; ++ii)
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const float ke = kj[jj] * ex2f(fminf(gi[ii] - gj[jj], 0.f));
+                            v[ii * 4 + jj] = fmaf(ki[ii], ke, v[ii * 4 + jj]);
+                            v[16 + ii * 4 + jj] = fmaf(qi[ii], ke, v[16 + ii * 4 + jj]);
+                        }
+                }
+                // reduce-scatter over the lanes: lane l ends with the total of value l
+#pragma unroll
+                for (int hh = 16; hh >= 1; hh >>= 1) {
+                    const bool up = lane & hh;
+#pragma unroll
+                    for (int x = 0; x < hh; ++x) {
+                        const float send = up ? v[x] : v[x + hh];
+                        const float keep = up ? v[x + hh] : v[x];
+                        v[x] = keep + __shfl_xor_sync(FULL, send, hh);
+                    }
+                }
+                const int i = i0 + ((lane >> 2) & 3), j = j0 + (lane & 3);
+                if (lane < 16) {
+                    if (j < i) sm.u.m.A[i][j] = v[0];
+                } else if (j <= i) {
+                    sm.u.m.PT[j][i] = v[0];
+                }
+            }
+            __syncthreads();
+
+            // ---- 5. M^-1 = (I + Diag(b) A)^-1 by forward substitution: column 4 warp +
+            //      lane / 8, rows j = s + 8 m held by lane s = lane % 8 ----
+            {
+                const int col = 4 * warp + (lane >> 3), s = lane & 7;
+                float xr[8];
+#pragma unroll
+                for (int m = 0; m < 8; ++m) xr[m] = 0.f;
+#pragma unroll
+                for (int i = 0; i < CC; ++i) {
+                    float part = 0.f;
+#pragma unroll
+                    for (int m = 0; m < (i + 7) / 8; ++m) part = fmaf(sm.u.m.A[i][s + 8 * m], xr[m], part);
+                    part += __shfl_xor_sync(FULL, part, 1);
+                    part += __shfl_xor_sync(FULL, part, 2);
+                    part += __shfl_xor_sync(FULL, part, 4);
+                    const float xi = (i == col) ? 1.f : -sm.b[i] * part;
+                    if (s == (i & 7)) xr[i >> 3] = xi;
+                }
+#pragma unroll
+                for (int m = 0; m < 8; ++m) sm.u.m.Mi[s + 8 * m][col] = xr[m];
+            }
+            __syncthreads();
+
+            // ---- 6. Y = v - (k^ Gam) S0 ----
+            {
+                float acc[4][4] = {};
+                mm(acc, 0, kHead, [&](int r, int k) { return KGT[k * CC + r0 + r]; },
+                   [&](int k, int j) { return S0[(size_t)k * kHead + lane + 32 * j]; });
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int t = r0 + r, vc = lane + 32 * j;
+                        const float vin = t < L ? bf(p.v, (size_t)(tok + t) * rs + hb + vc) : 0.f;
+                        const float y = vin - acc[r][j];
+                        Y[t * kHead + vc] = y;
+                        YT[vc * CC + t] = y;
+                    }
+            }
+            __syncthreads();
+
+            // ---- 7. U = M^-1 Diag(b) Y ----
+            {
+                float acc[4][4] = {};
+                mm(acc, 0, r0 + 4, [&](int r, int j) { return sm.u.m.Mi[r0 + r][j] * sm.b[j]; },
+                   [&](int j, int jj) { return Y[j * kHead + lane + 32 * jj]; });
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int t = r0 + r, vc = lane + 32 * j;
+                        U[t * kHead + vc] = acc[r][j];
+                        UT[vc * CC + t] = acc[r][j];
+                    }
+            }
+            __syncthreads();
+
+            // ---- 8. dU = scale P^T dO + K' dS ----
+            {
+                float acc[4][4] = {};
+                mm(acc, r0, CC, [&](int r, int i) { return sm.u.m.PT[r0 + r][i]; },
+                   [&](int i, int j) { return DO[i * kHead + lane + 32 * j]; });
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) acc[r][j] *= p.scale;
+                mm(acc, 0, kHead, [&](int r, int k) { return KPT[k * CC + r0 + r]; },
+                   [&](int k, int j) { return DS[k * kHead + lane + 32 * j]; });
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) DU[(r0 + r) * kHead + lane + 32 * j] = acc[r][j];
+            }
+            __syncthreads();
+
+            // ---- 9. dY = Diag(b) M^-T dU (= dv) ----
+            {
+                float acc[4][4] = {};
+                mm(acc, r0, CC, [&](int r, int i) { return sm.u.m.Mi[i][r0 + r]; },
+                   [&](int i, int j) { return DU[i * kHead + lane + 32 * j]; });
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int t = r0 + r, vc = lane + 32 * j;
+                        const float dy = sm.b[t] * acc[r][j];
+                        DY[t * kHead + vc] = dy;
+                        DYT[vc * CC + t] = dy;
+                        if (t < L) p.dv[(size_t)(tok + t) * rs + hb + vc] = dy;
+                    }
+            }
+            __syncthreads();
+
+            // ---- 10. dT = dU Y^T, dP = scale dO U^T (lower parts); rowsum(dS o S0) e^GL ----
+            {
+                float aT[4][2] = {}, aP[4][2] = {};
+#pragma unroll 2
+                for (int vc = 0; vc < kHead; ++vc) {
+                    float du[4], dox[4], yt[2], ut[2];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        du[r] = DU[(r0 + r) * kHead + vc];
+                        dox[r] = DO[(r0 + r) * kHead + vc];
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        yt[jj] = YT[vc * CC + lane + 32 * jj];
+                        ut[jj] = UT[vc * CC + lane + 32 * jj];
+                    }
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            aT[r][jj] = fmaf(du[r], yt[jj], aT[r][jj]);
+                            aP[r][jj] = fmaf(dox[r], ut[jj], aP[r][jj]);
+                        }
+                }
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int i = r0 + r, j = lane + 32 * jj;
+                        sm.u.m.X[i][j] = j <= i ? aT[r][jj] : 0.f;
+                        sm.u.m.dP[i][j] = j <= i ? p.scale * aP[r][jj] : 0.f;
+                    }
+#pragma unroll 1
+                for (int rr = 0; rr < 8; ++rr) {
+                    const int k = c0 + rr;
+                    float s = 0.f;
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const int vc = lane + 32 * m;
+                        s = fmaf(DS[k * kHead + vc], S0[(size_t)k * kHead + vc], s);
+                    }
+                    s = wsum(s);
+                    if (lane == 0) sm.dGL[k] = sm.eGL[k] * s;
+                }
+            }
+
+            // ---- 11. dK' = U dS^T, d(k^ Gam) = -dY S0^T, d(q^ Gam) = scale dO S0^T, as
+            //      [channel][token] (rows c0.., columns lane + 32 jj) into dk^, dq^, dG ----
+            {
+                float acc[8][2] = {};
+                mm(acc, 0, kHead, [&](int r, int vc) { return DS[(c0 + r) * kHead + vc]; },
+                   [&](int vc, int jj) { return UT[vc * CC + lane + 32 * jj]; });
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const int c = c0 + r;
+                    float cs = 0.f;
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int t = lane + 32 * jj;
+                        const float f = ex2f(sm.G2L[c] - sm.GT[c][t]);
+                        const float kp = sm.KT[c][t] * f, d = acc[r][jj];
+                        DKT[c * CC + t] = d * f;
+                        DGT[c * CC + t] = -d * kp;
+                        cs = fmaf(d, kp, cs);
+                    }
+                    cs = wsum(cs);
+                    if (lane == 0) sm.extra[c] = cs;
+                }
+            }
+            {
+                float ak[8][2] = {}, aq[8][2] = {};
+#pragma unroll 2
+                for (int vc = 0; vc < kHead; ++vc) {
+                    float s0[8], dyt[2], dot[2];
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) s0[r] = S0[(size_t)(c0 + r) * kHead + vc];
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        dyt[jj] = DYT[vc * CC + lane + 32 * jj];
+                        dot[jj] = DOT[vc * CC + lane + 32 * jj];
+                    }
+#pragma unroll
+                    for (int r = 0; r < 8; ++r)
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            ak[r][jj] = fmaf(s0[r], dyt[jj], ak[r][jj]);
+                            aq[r][jj] = fmaf(s0[r], dot[jj], aq[r][jj]);
+                        }
+                }
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int c = c0 + r, t = lane + 32 * jj, e = c * CC + t;
+                        const float gam = ex2f(sm.GT[c][t]);
+                        const float dkg = -ak[r][jj], dqg = p.scale * aq[r][jj];
+                        DKT[e] += dkg * gam;
+                        DQT[e] = dqg * gam;
+                        DGT[e] += (dkg * sm.KT[c][t] + dqg * sm.QT[c][t]) * gam;
+                    }
+            }
+            __syncthreads();
+
+            // ---- 12. dS <- Diag(e^GL) dS + scale (q^ Gam)^T dO - (k^ Gam)^T dY ----
+            {
+                float acc[8][4] = {};
+#pragma unroll 2
+                for (int t = 0; t < CC; ++t) {
+                    float aq[8], ak[8], bo[4], by[4];
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        aq[r] = p.scale * QGT[(c0 + r) * CC + t];
+                        ak[r] = KGT[(c0 + r) * CC + t];
+                    }
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        bo[j] = DO[t * kHead + lane + 32 * j];
+                        by[j] = DY[t * kHead + lane + 32 * j];
+                    }
+#pragma unroll
+                    for (int r = 0; r < 8; ++r)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            acc[r][j] = fmaf(-ak[r], by[j], fmaf(aq[r], bo[j], acc[r][j]));
+                }
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int e = (c0 + r) * kHead + lane + 32 * j;
+                        DS[e] = fmaf(sm.eGL[c0 + r], DS[e], acc[r][j]);
+                    }
+            }
+
+            // ---- 13. the solve's adjoint: db_j = sum_i dT_ij M^-1_ij; W = dM^-1 M^-T
+            //      (into PT); dM = -M^-T W; dA = Diag(b) dM (strict lower, into X) ----
+            if (tid < CC) {
+                float s = 0.f;
+                for (int i = tid; i < CC; ++i) s = fmaf(sm.u.m.X[i][tid], sm.u.m.Mi[i][tid], s);
+                sm.db[tid] = s;
+            }
+            {
+                float acc[4][2] = {};
+                mm(acc, 0, r0 + 4, [&](int r, int k) { return sm.u.m.X[r0 + r][k] * sm.b[k]; },
+                   [&](int k, int jj) { return sm.u.m.Mi[lane + 32 * jj][k]; });
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) sm.u.m.PT[r0 + r][lane + 32 * jj] = acc[r][jj];
+            }
+            __syncthreads();
+            {
+                float acc[4][2] = {};
+                mm(acc, r0, CC, [&](int r, int k) { return sm.u.m.Mi[k][r0 + r]; },
+                   [&](int k, int jj) { return sm.u.m.PT[k][lane + 32 * jj]; });
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int i = r0 + r;
+                    float d2 = 0.f;
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int j = lane + 32 * jj;
+                        const float dm = -acc[r][jj];
+                        const bool lo = j < i;
+                        d2 += lo ? dm * sm.u.m.A[i][j] : 0.f;
+                        sm.u.m.X[i][j] = lo ? sm.b[i] * dm : 0.f;
+                    }
+                    d2 = wsum(d2);
+                    if (lane == 0) sm.db[i] += d2;
+                }
+            }
+            __syncthreads();
+
+            // ---- 14. adjoints of the decay-weighted products, per (channel, token) ----
+            {
+                // row side: token t = i; sums over j <= i
+                float gi[8][2], ta[8][2], tp[8][2];
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        gi[r][jj] = sm.GT[c0 + r][lane + 32 * jj];
+                        ta[r][jj] = 0.f;
+                        tp[r][jj] = 0.f;
+                    }
+#pragma unroll 1
+                for (int j = 0; j < CC; ++j) {
+                    const int jj0 = j < 32 ? 0 : 1;  // tokens i = lane + 32 jj >= j only
+                    float dA_[2], dP_[2];
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        dA_[jj] = sm.u.m.X[lane + 32 * jj][j];
+                        dP_[jj] = sm.u.m.dP[lane + 32 * jj][j];
+                    }
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const float kj = sm.KT[c0 + r][j], gj = sm.GT[c0 + r][j];
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            if (jj < jj0) continue;
+                            const float ke = kj * ex2f(fminf(gi[r][jj] - gj, 0.f));
+                            ta[r][jj] = fmaf(dA_[jj], ke, ta[r][jj]);
+                            tp[r][jj] = fmaf(dP_[jj], ke, tp[r][jj]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int c = c0 + r, t = lane + 32 * jj, e = c * CC + t;
+                        DKT[e] += ta[r][jj];
+                        DQT[e] += tp[r][jj];
+                        DGT[e] += sm.KT[c][t] * ta[r][jj] + sm.QT[c][t] * tp[r][jj];
+                    }
+            }
+            {
+                // column side: token t = j; sums over i >= j
+                float gj[8][2], ta[8][2];
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        gj[r][jj] = sm.GT[c0 + r][lane + 32 * jj];
+                        ta[r][jj] = 0.f;
+                    }
+#pragma unroll 1
+                for (int i = 0; i < CC; ++i) {
+                    const int jj1 = i < 32 ? 1 : 2;  // tokens j = lane + 32 jj <= i only
+                    float dA_[2], dP_[2];
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        dA_[jj] = sm.u.m.X[i][lane + 32 * jj];
+                        dP_[jj] = sm.u.m.dP[i][lane + 32 * jj];
+                    }
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const float ki = sm.KT[c0 + r][i], qi = sm.QT[c0 + r][i], g = sm.GT[c0 + r][i];
+#pragma unroll
+                        for (int jj = 0; jj < 2; ++jj) {
+                            if (jj >= jj1) continue;
+                            const float e = ex2f(fminf(g - gj[r][jj], 0.f));
+                            ta[r][jj] = fmaf(fmaf(dA_[jj], ki, dP_[jj] * qi), e, ta[r][jj]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int c = c0 + r, t = lane + 32 * jj, e = c * CC + t;
+                        DKT[e] += ta[r][jj];
+                        DGT[e] -= sm.KT[c][t] * ta[r][jj];
+                    }
+            }
+            __syncthreads();
+
+            // ---- 15. epilogue: dG[L-1] terms, dlam, norms, sigmoid and gate ----
+            if (tid < kHead) DGT[tid * CC + L - 1] += sm.extra[tid] + sm.dGL[tid];
+            __syncthreads();
+            {
+                float pq[2] = {0.f, 0.f}, pk[2] = {0.f, 0.f};
+#pragma unroll
+                for (int r = 0; r < 8; ++r) {
+                    const int c = c0 + r;
+                    // reverse cumulative sum over the chunk's tokens: lane holds t = lane, lane + 32
+                    float s0 = DGT[c * CC + lane], s1 = DGT[c * CC + lane + 32];
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const float y0 = __shfl_down_sync(FULL, s0, o), y1 = __shfl_down_sync(FULL, s1, o);
+                        if (lane + o < 32) {
+                            s0 += y0;
+                            s1 += y1;
+                        }
+                    }
+                    s0 += __shfl_sync(FULL, s1, 0);
+                    sm.u.e.o0[lane][c] = s0;
+                    sm.u.e.o0[lane + 32][c] = s1;
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int t = lane + 32 * jj;
+                        pq[jj] = fmaf(sm.QT[c][t], DQT[c * CC + t], pq[jj]);
+                        pk[jj] = fmaf(sm.KT[c][t], DKT[c * CC + t], pk[jj]);
+                    }
+                }
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    sm.red[0][warp][lane + 32 * jj] = pq[jj];
+                    sm.red[1][warp][lane + 32 * jj] = pk[jj];
+                }
+            }
+            __syncthreads();
+            if (tid < 2 * CC) {
+                const int a = tid >> 6, t = tid & (CC - 1);
+                float s = 0.f;
+#pragma unroll
+                for (int w = 0; w < CW; ++w) s += sm.red[a][w][t];
+                sm.red[a][0][t] = s;
+            }
+            __syncthreads();
+#pragma unroll 1
+            for (int a = 0; a < 2; ++a) {  // a = 0: dq, a = 1: dk
+                const float *DXT = a ? DKT : DQT;
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+#pragma unroll
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int c = c0 + r, t = lane + 32 * jj;
+                        const float xh = a ? sm.KT[c][t] : sm.QT[c][t];
+                        const float rn = a ? sm.rk[t] : sm.rq[t];
+                        sm.u.e.o1[t][c] = rn * (DXT[c * CC + t] - xh * sm.red[a][0][t]);
+                    }
+                __syncthreads();
+                float *dst = a ? p.dk : p.dq;
+#pragma unroll 1
+                for (int i = 0; i < CC / CW; ++i) {
+                    const int t = warp + CW * i;
+                    if (t < L) {
+                        const size_t row = (size_t)(tok + t) * rs + hb;
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) dst[row + lane + 32 * m] = sm.u.e.o1[t][lane + 32 * m];
+                    }
+                }
+                __syncthreads();
+            }
+            {
+                float da = 0.f;
+#pragma unroll 1
+                for (int i = 0; i < CC / CW; ++i) {
+                    const int t = warp + CW * i;
+                    if (t >= L) continue;
+                    const size_t row = (size_t)(tok + t) * rs + hb;
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const int c = lane + 32 * m;
+                        const float x = bf(p.g, row + c) + sm.dtb[c];
+                        const float z = -ea * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))));
+                        const bool open = z >= p.lower_bound;  // the clamp is not holding
+                        const float dl = sm.u.e.o0[t][c];
+                        const float dx = open ? -dl * ea / (1.f + expf(-x)) : 0.f;
+                        p.dg[row + c] = dx;
+                        sm.pacc[warp][c] += dx;
+                        da += open ? dl * z : 0.f;
+                    }
+                }
+                da = wsum(da);
+                if (lane == 0) sm.pacc[warp][kHead] += da;
+                if (tid < L) {
+                    const float bt = sm.b[tid];
+                    p.dbeta[(size_t)(tok + tid) * p.H + h] = sm.db[tid] * bt * (1.f - bt);
+                }
+            }
+            __syncthreads();
+        }
+
+        // ---- dL/dS_0 and the unit's parameter partials ----
+        if (p.dinit)
+            for (int i = tid; i < ST; i += CT) p.dinit[st_off + i] = DS[i];
+        __syncthreads();
+        if (tid <= kHead) {
+            float acc = 0.f;
+#pragma unroll
+            for (int w = 0; w < CW; ++w) acc += sm.pacc[w][tid];
+            p.part[(size_t)u * (kHead + 1) + tid] = acc;
+        }
+    }
+}
+
+std::atomic<int> g_bwd_mode{KDA_BWD_CHUNKED};
+
+}  // namespace
+
+size_t bwd_chunked_scratch_bytes_per_cta() { return (size_t)S_FLOATS * sizeof(float); }
+
+int bwd_set_schedule(int mode)
+{
+    if (mode != KDA_BWD_CHUNKED && mode != KDA_BWD_TOKEN) return KDA_ERR_ARG;
+    return g_bwd_mode.exchange(mode);
+}
+
+int launch_backward(const BwdParams &p, const BwdLayout &l, cudaStream_t stream)
+{
+    if (g_bwd_mode.load() == KDA_BWD_TOKEN) return launch_backward_token(p, l, stream);
+    const int64_t units = p.N * p.H;
+    if (units <= 0) return 0;
+    int launches = 0;
+    if (p.B * p.T > 0) {  // the states before every chunk (no chunks: nothing to store)
+        FwdParams f{};
+        f.q = p.q;
+        f.k = p.k;
+        f.v = p.v;
+        f.g = p.g;
+        f.beta = p.beta;
+        f.A_log = p.A_log;
+        f.dt_bias = p.dt_bias;
+        f.init = p.init;
+        f.init_dtype = p.init_dtype;
+        f.final_state = nullptr;
+        f.final_dtype = KDA_STATE_F32;
+        f.state_layout = KDA_LAYOUT_KV;
+        f.cu = p.cu;
+        f.out = nullptr;
+        f.scale = p.scale;
+        f.lower_bound = p.lower_bound;
+        f.B = p.B;
+        f.T = p.T;
+        f.H = p.H;
+        f.N = p.N;
+        f.ckpt = p.ckpt;
+        const int n = launch_chunked(f, stream);
+        if (n < 0) return n;
+        launches += n;
+    }
+    static int smem_set[64];
+    const int smem = (int)sizeof(CSmem);
+    if (!set_smem_limit_once(bwdc_kernel, smem, smem_set)) return KDA_ERR_CUDA;
+    bwdc_kernel<<<l.grid, CT, smem, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return KDA_ERR_CUDA;
+    const int n = launch_param_reduce(p, stream);
+    return n < 0 ? n : launches + 1 + n;
+}
+
+}  // namespace kda

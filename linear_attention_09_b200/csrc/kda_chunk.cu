@@ -945,7 +945,7 @@ __device__ void u_send_role(const Ctx &cx)
 //   -> U~ = U / tau' -> TM_S <- (gamma * TM_S) tau / tau' -> MMA2: TM_S += U~^T k',
 //   D3 = U~^T P^T -> out = scale (sigma D1[:,64:128] + tau' D3).
 // =====================================================================================
-template <Mode M, bool GH = false>
+template <Mode M, bool GH = false, bool CK = false>
 __device__ void state_role(const FwdParams &p, const Ctx &cx)
 {
     uint8_t *sm = cx.sm;
@@ -1054,6 +1054,11 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
         float sigma;
         {
             float mx = 0.f;
+            // checkpoint instantiation: the state before this chunk, fp32 S[k][v], to
+            // slot (tok0 / 64 + sequence + n) * H + h of p.ckpt
+            float *ck = nullptr;
+            if constexpr (CK)
+                ck = p.ckpt + ((size_t)(cx.tok0 / C + cx.unit / H + n) * H + h) * (kHead * kHead) + v;
 #pragma unroll
             for (int k0 = 0; k0 < kHead; k0 += 32) {
                 uint32_t a[32];
@@ -1061,6 +1066,10 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 32; ++j) mx = fmaxf(mx, fabsf(__uint_as_float(a[j])));
+                if constexpr (CK) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) ck[(k0 + j) * kHead] = tau * __uint_as_float(a[j]);
+                }
             }
             sigma = pow2_ceil(mx * tau);
             const float f = tau / sigma;
@@ -1199,8 +1208,9 @@ __device__ void state_role(const FwdParams &p, const Ctx &cx)
         }
 
         // ---- out = scale (sigma D1[:, 64:128] + tau D3): thread v stores column v of each
-        //      token; a warp's 32 columns are 64 contiguous bytes of the token's row ----
-        {
+        //      token; a warp's 32 columns are 64 contiguous bytes of the token's row
+        //      (not in the checkpoint instantiation, which writes no output) ----
+        if constexpr (!CK) {
             __nv_bfloat16 *op = p.out + (ctok * H + h) * kHead + v;
             const float fs = p.scale * sigma, ft = p.scale * tau;
 #pragma unroll 1
@@ -1323,7 +1333,7 @@ __device__ __forceinline__ void read_abort(const FwdParams &p)
 }
 
 // GH: the state role computes the round-1 gates of chunks 2.. (launches of long units)
-template <bool GH>
+template <bool GH, bool CK = false>
 __global__ void __launch_bounds__(NT, 1)
 chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
 {
@@ -1364,7 +1374,7 @@ chunk_kernel(const FwdParams p, const __grid_constant__ TMaps tm)
     }
 
     if (warp < NT_IN / 32) in_chunk_role<kFused, GH>(p, tm, cx);
-    else if (warp < (NT_IN + NT_ST) / 32) state_role<kFused, GH>(p, cx);
+    else if (warp < (NT_IN + NT_ST) / 32) state_role<kFused, GH, CK>(p, cx);
     else mma_role<kFused>(tm, cx);
 
     tc_fence_before();
@@ -1538,9 +1548,10 @@ int launch_chunked(const FwdParams &p, cudaStream_t stream)
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return KDA_ERR_CUDA;
     }
-    static int attr_plain[64], attr_gh[64];
+    static int attr_plain[64], attr_gh[64], attr_ck[64];
     if (!set_smem_limit_once(chunk_kernel<false>, SMEM_ALLOC, attr_plain) ||
-        !set_smem_limit_once(chunk_kernel<true>, SMEM_ALLOC, attr_gh))
+        !set_smem_limit_once(chunk_kernel<true>, SMEM_ALLOC, attr_gh) ||
+        (p.ckpt && !set_smem_limit_once(chunk_kernel<true, true>, SMEM_ALLOC, attr_ck)))
         return KDA_ERR_CUDA;
     // the launch's epoch: 24 bits, never 0 (an error word of 0 means no error)
     static std::atomic<uint32_t> epochs{0};
@@ -1554,6 +1565,10 @@ int launch_chunked(const FwdParams &p, cudaStream_t stream)
             return KDA_ERR_CUDA;
     }
     g_last_schedule = KDA_SCHEDULE_FUSED;
+    if (p.ckpt) {  // the backward pass's checkpoints: fused schedule, no output
+        chunk_kernel<true, true><<<(unsigned)ctas, NT, SMEM_ALLOC, stream>>>(pe, tm);
+        return cudaGetLastError() == cudaSuccess ? 1 : KDA_ERR_CUDA;
+    }
     if (use_split(p, ctas)) {
         g_last_schedule = KDA_SCHEDULE_SPLIT;
         cudaLaunchConfig_t cfg = {};

@@ -22,6 +22,10 @@ struct FwdParams {
     float scale, lower_bound;
     int64_t B, T, H, N;      // N = number of sequences
     uint32_t epoch;          // set by the launcher: tags the launch's error word
+    // Backward pass only: when set, the launch stores the fp32 state S[k][v] before
+    // every 64-token chunk of unit (sequence s, head h) starting at token bos, chunk n,
+    // at slot (bos / 64 + s + n) * H + h (64 KB each), and writes no output.
+    float *ckpt;
 };
 
 // One decode step: one token per (sequence, head), state updated in HBM.
@@ -64,7 +68,13 @@ struct BwdLayout {
 
 // Workspace bytes of a backward call (and the split into regions).
 size_t bwd_layout(int64_t total_tokens, int64_t N, int64_t H, BwdLayout *out);
+// The backward pass in the schedule set by bwd_set_schedule (KDA_BWD_*): the number of
+// kernels enqueued or a negative KDA_ERR_* code.
 int launch_backward(const BwdParams &p, const BwdLayout &l, cudaStream_t stream);
+int launch_backward_token(const BwdParams &p, const BwdLayout &l, cudaStream_t stream);
+int launch_param_reduce(const BwdParams &p, cudaStream_t stream);  // dA_log, ddt_bias
+int bwd_set_schedule(int mode);  // the previous mode or KDA_ERR_ARG
+size_t bwd_chunked_scratch_bytes_per_cta();
 
 // Raises `kernel`'s dynamic shared-memory limit to `bytes` once per device (the
 // attribute belongs to the device's context); `done` is the caller's per-device flags.

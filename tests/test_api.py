@@ -231,6 +231,19 @@ def test_bwd_workspace_size():
     assert kda.kda_bwd_workspace_size(1, 1000, 2, num_seqs=3) >= (1000 // 64 + 3) * 2 * 65536
 
 
+def test_bwd_schedule_switch(L):
+    """Backward schedule: "chunked" by default, "token" on request; unknown modes are
+    rejected without changing the setting."""
+    prev = kda.kda_set_bwd_schedule("chunked")
+    try:
+        assert prev == "chunked"
+        assert L.kda_set_bwd_schedule(5) == -15
+        assert kda.kda_set_bwd_schedule("token") == "chunked"
+        assert kda.kda_set_bwd_schedule(kda.KDA_BWD_CHUNKED) == "token"
+    finally:
+        kda.kda_set_bwd_schedule(prev)
+
+
 def test_bwd_valid_arguments_without_device(L):
     import torch
     if not torch.cuda.is_available():
