@@ -26,9 +26,12 @@
 // on the CUDA cores.  The activations (q^, k^, G; channel-major) and the 64 x 64
 // matrices live in shared memory; the 64 x 128 tiles of a chunk (dO, Y, U, dU, dY,
 // their transposes, k^ Gam, q^ Gam, K', the gradient accumulators) and dS live in a
-// per-CTA scratch region of global memory that stays in L2 and L1.  Every product is
-// a register-blocked loop whose second operand is read along its rows by consecutive
-// lanes, so each operand that appears in both orientations is stored in both.
+// per-CTA scratch region of global memory that stays in L2.  The products stream
+// their operands from there through a two-slab shared-memory ring filled by cp.async
+// (the copy of slab s + 1 in flight while slab s is used), so that L2 latency is not
+// paid per load.  Every product is a register-blocked loop whose second operand is
+// read along its rows by consecutive lanes, so each operand that appears in both
+// orientations is stored in both.
 #include <atomic>
 #include <cstddef>
 
@@ -48,7 +51,11 @@ constexpr int TILE = CC * kHead;   // floats of one 64 x 128 tile
 constexpr unsigned FULL = 0xffffffffu;
 constexpr float kL2e = 1.4426950408889634f;
 
+constexpr int STG = 4096;  // floats of one slot of the operand ring
+constexpr int NSLOT = 2;   // slots: slab s + 1 in flight while slab s is used
+
 struct CSmem {
+    float stg[NSLOT][STG];  // operand ring (first: 16-byte aligned for cp.async)
     float QT[kHead][LDT];  // q^   [channel][token]
     float KT[kHead][LDT];  // k^
     float GT[kHead][LDT];  // G log2(e): in-chunk inclusive cumulative sum of the log-decay
@@ -62,12 +69,11 @@ struct CSmem {
         } m;
         struct {
             float o0[CC][LDE], o1[CC][LDE];  // [token][channel] staging of the outputs
+            float red[2][CW][CC];            // per-warp partial sums of the norm gradients
         } e;
     } u;
     float b[CC], rq[CC], rk[CC], db[CC];
     float eGL[kHead], G2L[kHead], dGL[kHead], extra[kHead], dtb[kHead];
-    float red[2][CW][CC];
-    float pacc[CW][kHead + 1];  // per-warp partial ddt_bias (0..127) and dA_log (128)
 };
 
 // Per-CTA scratch (floats): the tiles in the order of these offsets.
@@ -75,7 +81,8 @@ enum : int {
     S_DO = 0, S_DOT = TILE, S_KGT = 2 * TILE, S_QGT = 3 * TILE, S_KPT = 4 * TILE, S_Y = 5 * TILE,
     S_YT = 6 * TILE, S_U = 7 * TILE, S_UT = 8 * TILE, S_DU = 9 * TILE, S_DY = 10 * TILE,
     S_DYT = 11 * TILE, S_DKT = 12 * TILE, S_DQT = 13 * TILE, S_DGT = 14 * TILE, S_DS = 15 * TILE,
-    S_FLOATS = 15 * TILE + ST
+    S_PACC = 15 * TILE + ST,  // per-warp partial ddt_bias (0..127) and dA_log (128)
+    S_FLOATS = S_PACC + CW * (kHead + 1)
 };
 
 __device__ __forceinline__ float ex2f(float x)
@@ -94,12 +101,103 @@ __device__ __forceinline__ float wsum(float x)
     return x;
 }
 
+__device__ __forceinline__ void cp16(float *dst, const float *src)
+{
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// This thread's share of copying n contiguous floats (n % 4 == 0, 16-byte aligned).
+__device__ __forceinline__ void stage_rows(float *dst, const float *src, int n)
+{
+    for (int i = threadIdx.x; i < n / 4; i += CT) cp16(dst + 4 * i, src + 4 * i);
+}
+
+// This thread's share of copying columns [c, c + w) of `rows` rows of a row-major matrix
+// with leading dimension ld into a dense [rows][w] block (w % 4 == 0).
+__device__ __forceinline__ void stage_cols(float *dst, const float *src, int rows, int ld, int c, int w)
+{
+    const int per = w / 4;
+    for (int i = threadIdx.x; i < rows * per; i += CT) {
+        const int r = i / per, q = i - r * per;
+        cp16(dst + r * w + 4 * q, src + (size_t)r * ld + c + 4 * q);
+    }
+}
+
+// Slabs 0..nslab-1 of a product: issue(s, buf) starts the copies of slab s into ring
+// slot s % 2, body(buf, s) uses it once it has landed (every thread's copies); the
+// copy of slab s + 1 is in flight during body(., s).  Called by all threads; ends
+// with a barrier, after which the ring is free.  (Measured: slabs of 16 rows in two
+// slots beat slabs of 8 in four slots with two in flight; the cost per slab does not
+// shrink with its size.)
+template <class Issue, class Body>
+__device__ __forceinline__ void staged(float (*stg)[STG], int nslab, Issue issue, Body body)
+{
+    issue(0, stg[0]);
+    cp_commit();
+    for (int s = 0; s < nslab; ++s) {
+        if (s + 1 < nslab) issue(s + 1, stg[(s + 1) & 1]);
+        cp_commit();
+        cp_wait1();
+        __syncthreads();
+        body(static_cast<const float *>(stg[s & 1]), s);
+        __syncthreads();
+    }
+}
+
+__device__ __forceinline__ float comp(const float4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+
+// acc[r][j] += sum_k A[k][r0 + r] B[k][lane + 32 j] over a slab: A is [ks][64] (rows
+// r0..r0 + 3 of row k in one 16-byte load), B is [ks][32 J].
+template <int J>
+__device__ __forceinline__ void mm_k4(float (&acc)[4][J], const float *A, int r0, const float *B, int ks)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll 4
+    for (int k = 0; k < ks; ++k) {
+        const float4 a = *reinterpret_cast<const float4 *>(A + k * CC + r0);
+        float b[J];
+#pragma unroll
+        for (int j = 0; j < J; ++j) b[j] = B[k * 32 * J + lane + 32 * j];
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int j = 0; j < J; ++j) acc[r][j] = fmaf(comp(a, r), b[j], acc[r][j]);
+    }
+}
+
+// acc[r][j] += sum_k A[row0 + r][k] B[k][lane + 32 j] over a slab: A is [rows][ks]
+// (four k of a row in one 16-byte load), B is [ks][32 J]; ks % 4 == 0.
+template <int R, int J>
+__device__ __forceinline__ void mm_r4(float (&acc)[R][J], const float *A, int row0, const float *B, int ks)
+{
+    const int lane = threadIdx.x & 31;
+#pragma unroll 1
+    for (int k = 0; k < ks; k += 4) {
+        float4 a[R];
+#pragma unroll
+        for (int r = 0; r < R; ++r) a[r] = *reinterpret_cast<const float4 *>(A + (row0 + r) * ks + k);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            float b[J];
+#pragma unroll
+            for (int j = 0; j < J; ++j) b[j] = B[(k + kk) * 32 * J + lane + 32 * j];
+#pragma unroll
+            for (int r = 0; r < R; ++r)
+#pragma unroll
+                for (int j = 0; j < J; ++j) acc[r][j] = fmaf(comp(a[r], kk), b[j], acc[r][j]);
+        }
+    }
+}
+
 // acc[r][j] += sum_{k in [k0, k1)} fa(r, k) fb(k, j): fa is the same for every lane of
 // the warp (a broadcast), fb(k, j) reads column lane + 32 j of row k.
 template <int R, int J, class FA, class FB>
 __device__ __forceinline__ void mm(float (&acc)[R][J], int k0, int k1, FA fa, FB fb)
 {
-#pragma unroll 2
+#pragma unroll 4
     for (int k = k0; k < k1; ++k) {
         float a[R], b[J];
 #pragma unroll
@@ -122,7 +220,7 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
     float *DO = scr + S_DO, *DOT = scr + S_DOT, *KGT = scr + S_KGT, *QGT = scr + S_QGT;
     float *KPT = scr + S_KPT, *Y = scr + S_Y, *YT = scr + S_YT, *U = scr + S_U, *UT = scr + S_UT;
     float *DU = scr + S_DU, *DY = scr + S_DY, *DYT = scr + S_DYT, *DKT = scr + S_DKT;
-    float *DQT = scr + S_DQT, *DGT = scr + S_DGT, *DS = scr + S_DS;
+    float *DQT = scr + S_DQT, *DGT = scr + S_DGT, *DS = scr + S_DS, *PACC = scr + S_PACC;
     const int r0 = 4 * warp;  // rows of this warp in the 64-row products
     const int c0 = 8 * warp;  // rows (channels) of this warp in the 128-row products
     const int64_t units = p.N * p.H;
@@ -140,9 +238,9 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
         const size_t st_off = (size_t)u * ST;
         const size_t hb = (size_t)h * kHead;
 
-        __syncthreads();  // the previous unit's readers of dtb / pacc / DS are done
+        __syncthreads();  // the previous unit's readers of dtb, the partials and DS are done
         if (tid < kHead) sm.dtb[tid] = p.dt_bias[h * kHead + tid];
-        for (int i = tid; i < CW * (kHead + 1); i += CT) (&sm.pacc[0][0])[i] = 0.f;
+        for (int i = tid; i < CW * (kHead + 1); i += CT) PACC[i] = 0.f;
         for (int i = tid; i < ST; i += CT) DS[i] = p.dfinal ? p.dfinal[st_off + i] : 0.f;
         __syncthreads();
 
@@ -152,7 +250,7 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             const float *S0 = ckb + n * ckstride;
 
             // ---- 1. activations of the chunk's tokens (zero past L), dO ----
-#pragma unroll 1
+#pragma unroll 2
             for (int i = 0; i < CC / CW; ++i) {
                 const int t = warp + CW * i;
                 const bool in = t < L;
@@ -193,6 +291,25 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             for (int i = tid; i < CC * LDT; i += CT) {
                 (&sm.u.m.A[0][0])[i] = 0.f;
                 (&sm.u.m.PT[0][0])[i] = 0.f;
+            }
+            if (n > 0) {
+                // the next chunk's state and input rows towards L2 while this one computes:
+                // 512 lines of the state, 2 lines per row of q, k, g, v, dO, 1 per beta
+                const float *Sn = S0 - ckstride;
+                const int64_t tn = tok - CC;
+                for (int x = tid; x < 512 + 5 * 2 * CC + CC; x += CT) {
+                    const void *a;
+                    if (x < 512) {
+                        a = Sn + 32 * x;
+                    } else if (x < 512 + 10 * CC) {
+                        const int y = x - 512, w = y / (2 * CC), t = (y >> 1) % CC;
+                        const __nv_bfloat16 *base = w == 0 ? p.q : w == 1 ? p.k : w == 2 ? p.g : w == 3 ? p.v : p.dout;
+                        a = base + (size_t)(tn + t) * rs + hb + 64 * (y & 1);
+                    } else {
+                        a = p.beta + (size_t)(tn + (x - 512 - 10 * CC)) * p.H + h;
+                    }
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
+                }
             }
             __syncthreads();
 
@@ -240,13 +357,22 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                         gj[x] = sm.GT[c][j0 + x];
                         kj[x] = sm.KT[c][j0 + x];
                     }
+                    // e^(G_i - G_j) = e^(G_i - G_j0) e^(G_j0 - G_j): the first factor <= 1
+                    // (i >= j0), the second <= e^15 (j - j0 <= 3, lam >= -5)
+                    float ka[4], qa[4], kb[4];
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const float a = ex2f(gi[x] - gj[0]);
+                        ka[x] = ki[x] * a;
+                        qa[x] = qi[x] * a;
+                        kb[x] = x == 0 ? kj[0] : kj[x] * ex2f(gj[0] - gj[x]);
+                    }
 #pragma unroll
                     for (int ii = 0; ii < 4; ++ii)
 #pragma unroll
                         for (int jj = 0; jj < 4; ++jj) {
-                            const float ke = kj[jj] * ex2f(fminf(gi[ii] - gj[jj], 0.f));
-                            v[ii * 4 + jj] = fmaf(ki[ii], ke, v[ii * 4 + jj]);
-                            v[16 + ii * 4 + jj] = fmaf(qi[ii], ke, v[16 + ii * 4 + jj]);
+                            v[ii * 4 + jj] = fmaf(ka[ii], kb[jj], v[ii * 4 + jj]);
+                            v[16 + ii * 4 + jj] = fmaf(qa[ii], kb[jj], v[16 + ii * 4 + jj]);
                         }
                 }
                 // reduce-scatter over the lanes: lane l ends with the total of value l
@@ -295,8 +421,12 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             // ---- 6. Y = v - (k^ Gam) S0 ----
             {
                 float acc[4][4] = {};
-                mm(acc, 0, kHead, [&](int r, int k) { return KGT[k * CC + r0 + r]; },
-                   [&](int k, int j) { return S0[(size_t)k * kHead + lane + 32 * j]; });
+                staged(sm.stg, kHead / 16,
+                       [&](int s, float *buf) {
+                           stage_rows(buf, KGT + s * 16 * CC, 16 * CC);                         // [16][64]
+                           stage_rows(buf + 16 * CC, S0 + (size_t)s * 16 * kHead, 16 * kHead);  // [16][128]
+                       },
+                       [&](const float *buf, int) { mm_k4(acc, buf, r0, buf + 16 * CC, 16); });
 #pragma unroll
                 for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -313,8 +443,12 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             // ---- 7. U = M^-1 Diag(b) Y ----
             {
                 float acc[4][4] = {};
-                mm(acc, 0, r0 + 4, [&](int r, int j) { return sm.u.m.Mi[r0 + r][j] * sm.b[j]; },
-                   [&](int j, int jj) { return Y[j * kHead + lane + 32 * jj]; });
+                staged(sm.stg, CC / 16, [&](int s, float *buf) { stage_rows(buf, Y + s * 16 * kHead, 16 * kHead); },
+                       [&](const float *buf, int s) {
+                           const int k0 = 16 * s, k1 = min(k0 + 16, r0 + 4);
+                           mm(acc, 0, k1 - k0, [&](int r, int k) { return sm.u.m.Mi[r0 + r][k0 + k] * sm.b[k0 + k]; },
+                              [&](int k, int jj) { return buf[k * kHead + lane + 32 * jj]; });
+                       });
 #pragma unroll
                 for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -329,14 +463,22 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             // ---- 8. dU = scale P^T dO + K' dS ----
             {
                 float acc[4][4] = {};
-                mm(acc, r0, CC, [&](int r, int i) { return sm.u.m.PT[r0 + r][i]; },
-                   [&](int i, int j) { return DO[i * kHead + lane + 32 * j]; });
+                staged(sm.stg, CC / 16, [&](int s, float *buf) { stage_rows(buf, DO + s * 16 * kHead, 16 * kHead); },
+                       [&](const float *buf, int s) {
+                           const int k0 = 16 * s, lo = max(r0 - k0, 0);
+                           mm(acc, lo, 16, [&](int r, int k) { return sm.u.m.PT[r0 + r][k0 + k]; },
+                              [&](int k, int j) { return buf[k * kHead + lane + 32 * j]; });
+                       });
 #pragma unroll
                 for (int r = 0; r < 4; ++r)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) acc[r][j] *= p.scale;
-                mm(acc, 0, kHead, [&](int r, int k) { return KPT[k * CC + r0 + r]; },
-                   [&](int k, int j) { return DS[k * kHead + lane + 32 * j]; });
+                staged(sm.stg, kHead / 16,
+                       [&](int s, float *buf) {
+                           stage_rows(buf, KPT + s * 16 * CC, 16 * CC);                 // [16][64]
+                           stage_rows(buf + 16 * CC, DS + s * 16 * kHead, 16 * kHead);  // [16][128]
+                       },
+                       [&](const float *buf, int) { mm_k4(acc, buf, r0, buf + 16 * CC, 16); });
 #pragma unroll
                 for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -347,8 +489,12 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             // ---- 9. dY = Diag(b) M^-T dU (= dv) ----
             {
                 float acc[4][4] = {};
-                mm(acc, r0, CC, [&](int r, int i) { return sm.u.m.Mi[i][r0 + r]; },
-                   [&](int i, int j) { return DU[i * kHead + lane + 32 * j]; });
+                staged(sm.stg, CC / 16, [&](int s, float *buf) { stage_rows(buf, DU + s * 16 * kHead, 16 * kHead); },
+                       [&](const float *buf, int s) {
+                           const int k0 = 16 * s, lo = max(r0 - k0, 0);
+                           mm(acc, lo, 16, [&](int r, int k) { return sm.u.m.Mi[k0 + k][r0 + r]; },
+                              [&](int k, int j) { return buf[k * kHead + lane + 32 * j]; });
+                       });
 #pragma unroll
                 for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -365,27 +511,17 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             // ---- 10. dT = dU Y^T, dP = scale dO U^T (lower parts); rowsum(dS o S0) e^GL ----
             {
                 float aT[4][2] = {}, aP[4][2] = {};
-#pragma unroll 2
-                for (int vc = 0; vc < kHead; ++vc) {
-                    float du[4], dox[4], yt[2], ut[2];
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        du[r] = DU[(r0 + r) * kHead + vc];
-                        dox[r] = DO[(r0 + r) * kHead + vc];
-                    }
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        yt[jj] = YT[vc * CC + lane + 32 * jj];
-                        ut[jj] = UT[vc * CC + lane + 32 * jj];
-                    }
-#pragma unroll
-                    for (int r = 0; r < 4; ++r)
-#pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) {
-                            aT[r][jj] = fmaf(du[r], yt[jj], aT[r][jj]);
-                            aP[r][jj] = fmaf(dox[r], ut[jj], aP[r][jj]);
-                        }
-                }
+                staged(sm.stg, kHead / 16,
+                       [&](int s, float *buf) {
+                           stage_cols(buf, DU, CC, kHead, 16 * s, 16);  // [64][16]
+                           stage_cols(buf + 1024, DO, CC, kHead, 16 * s, 16);
+                           stage_rows(buf + 2048, YT + s * 16 * CC, 16 * CC);  // [16][64]
+                           stage_rows(buf + 3072, UT + s * 16 * CC, 16 * CC);
+                       },
+                       [&](const float *buf, int) {
+                           mm_r4(aT, buf, r0, buf + 2048, 16);
+                           mm_r4(aP, buf + 1024, r0, buf + 3072, 16);
+                       });
 #pragma unroll
                 for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -394,7 +530,7 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                         sm.u.m.X[i][j] = j <= i ? aT[r][jj] : 0.f;
                         sm.u.m.dP[i][j] = j <= i ? p.scale * aP[r][jj] : 0.f;
                     }
-#pragma unroll 1
+#pragma unroll 4
                 for (int rr = 0; rr < 8; ++rr) {
                     const int k = c0 + rr;
                     float s = 0.f;
@@ -412,8 +548,12 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             //      [channel][token] (rows c0.., columns lane + 32 jj) into dk^, dq^, dG ----
             {
                 float acc[8][2] = {};
-                mm(acc, 0, kHead, [&](int r, int vc) { return DS[(c0 + r) * kHead + vc]; },
-                   [&](int vc, int jj) { return UT[vc * CC + lane + 32 * jj]; });
+                staged(sm.stg, kHead / 16,
+                       [&](int s, float *buf) {
+                           stage_cols(buf, DS, kHead, kHead, 16 * s, 16);  // [128][16]
+                           stage_rows(buf + 2048, UT + s * 16 * CC, 16 * CC);  // [16][64]
+                       },
+                       [&](const float *buf, int) { mm_r4(acc, buf, c0, buf + 2048, 16); });
 #pragma unroll
                 for (int r = 0; r < 8; ++r) {
                     const int c = c0 + r;
@@ -433,24 +573,16 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             }
             {
                 float ak[8][2] = {}, aq[8][2] = {};
-#pragma unroll 2
-                for (int vc = 0; vc < kHead; ++vc) {
-                    float s0[8], dyt[2], dot[2];
-#pragma unroll
-                    for (int r = 0; r < 8; ++r) s0[r] = S0[(size_t)(c0 + r) * kHead + vc];
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        dyt[jj] = DYT[vc * CC + lane + 32 * jj];
-                        dot[jj] = DOT[vc * CC + lane + 32 * jj];
-                    }
-#pragma unroll
-                    for (int r = 0; r < 8; ++r)
-#pragma unroll
-                        for (int jj = 0; jj < 2; ++jj) {
-                            ak[r][jj] = fmaf(s0[r], dyt[jj], ak[r][jj]);
-                            aq[r][jj] = fmaf(s0[r], dot[jj], aq[r][jj]);
-                        }
-                }
+                staged(sm.stg, kHead / 16,
+                       [&](int s, float *buf) {
+                           stage_cols(buf, S0, kHead, kHead, 16 * s, 16);  // [128][16]
+                           stage_rows(buf + 2048, DYT + s * 16 * CC, 16 * CC);  // [16][64]
+                           stage_rows(buf + 3072, DOT + s * 16 * CC, 16 * CC);
+                       },
+                       [&](const float *buf, int) {
+                           mm_r4(ak, buf, c0, buf + 2048, 16);
+                           mm_r4(aq, buf, c0, buf + 3072, 16);
+                       });
 #pragma unroll
                 for (int r = 0; r < 8; ++r)
 #pragma unroll
@@ -468,31 +600,24 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             // ---- 12. dS <- Diag(e^GL) dS + scale (q^ Gam)^T dO - (k^ Gam)^T dY ----
             {
                 float acc[8][4] = {};
-#pragma unroll 2
-                for (int t = 0; t < CC; ++t) {
-                    float aq[8], ak[8], bo[4], by[4];
-#pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        aq[r] = p.scale * QGT[(c0 + r) * CC + t];
-                        ak[r] = KGT[(c0 + r) * CC + t];
-                    }
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        bo[j] = DO[t * kHead + lane + 32 * j];
-                        by[j] = DY[t * kHead + lane + 32 * j];
-                    }
-#pragma unroll
-                    for (int r = 0; r < 8; ++r)
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            acc[r][j] = fmaf(-ak[r], by[j], fmaf(aq[r], bo[j], acc[r][j]));
-                }
+                float acc2[8][4] = {};  // (k^ Gam)^T dY, subtracted below
+                staged(sm.stg, CC / 8,
+                       [&](int s, float *buf) {
+                           stage_cols(buf, QGT, kHead, CC, 8 * s, 8);  // [128][8]
+                           stage_cols(buf + 1024, KGT, kHead, CC, 8 * s, 8);
+                           stage_rows(buf + 2048, DO + s * 8 * kHead, 8 * kHead);  // [8][128]
+                           stage_rows(buf + 3072, DY + s * 8 * kHead, 8 * kHead);
+                       },
+                       [&](const float *buf, int) {
+                           mm_r4(acc, buf, c0, buf + 2048, 8);
+                           mm_r4(acc2, buf + 1024, c0, buf + 3072, 8);
+                       });
 #pragma unroll
                 for (int r = 0; r < 8; ++r)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int e = (c0 + r) * kHead + lane + 32 * j;
-                        DS[e] = fmaf(sm.eGL[c0 + r], DS[e], acc[r][j]);
+                        DS[e] = fmaf(sm.eGL[c0 + r], DS[e], fmaf(p.scale, acc[r][j], -acc2[r][j]));
                     }
             }
 
@@ -535,87 +660,129 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             }
             __syncthreads();
 
-            // ---- 14. adjoints of the decay-weighted products, per (channel, token) ----
+            // ---- 14. adjoints of the decay-weighted products, per (channel, token), with the
+            //      factor e^(G_i - G_j) split at a reference token of a 16-token block so
+            //      that the exponentials are per (channel, token) instead of per pair.
+            //      Row side (sums over j <= i), reference e = the last token of j's block:
+            //        e^(G_i - G_j) = e^(G_i - G_e) e^(G_e - G_j), the second factor in
+            //        [e^-75, 1], the first <= e^75 (it underflows only where the product is
+            //        below e^-87).  KS[c][j] = k^_j e^(G_e - G_j) sits in the operand ring.
             {
-                // row side: token t = i; sums over j <= i
-                float gi[8][2], ta[8][2], tp[8][2];
-#pragma unroll
-                for (int r = 0; r < 8; ++r)
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        gi[r][jj] = sm.GT[c0 + r][lane + 32 * jj];
-                        ta[r][jj] = 0.f;
-                        tp[r][jj] = 0.f;
-                    }
+                float *KS = &sm.stg[0][0];
+                for (int e = tid; e < TILE; e += CT) {
+                    const int c = e >> 6, j = e & (CC - 1);
+                    KS[e] = sm.KT[c][j] * ex2f(sm.GT[c][j | 15] - sm.GT[c][j]);
+                }
+                __syncthreads();
 #pragma unroll 1
-                for (int j = 0; j < CC; ++j) {
-                    const int jj0 = j < 32 ? 0 : 1;  // tokens i = lane + 32 jj >= j only
-                    float dA_[2], dP_[2];
+                for (int rg = 0; rg < 2; ++rg) {
+                    const int cr = c0 + 4 * rg;
+                    float ta[4][2] = {}, tp[4][2] = {};
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        dA_[jj] = sm.u.m.X[lane + 32 * jj][j];
-                        dP_[jj] = sm.u.m.dP[lane + 32 * jj][j];
+                    for (int J = 0; J < 4; ++J) {
+                        // tokens i = lane + 32 jj: blocks J >= 2 hold only j > i for jj = 0
+                        float pa[4][2] = {}, pp[4][2] = {};
+#pragma unroll 4
+                        for (int j = 16 * J; j < 16 * J + 16; ++j) {
+                            float dA_[2], dP_[2];
+#pragma unroll
+                            for (int jj = 0; jj < 2; ++jj) {
+                                dA_[jj] = (J < 2 || jj == 1) ? sm.u.m.X[lane + 32 * jj][j] : 0.f;
+                                dP_[jj] = (J < 2 || jj == 1) ? sm.u.m.dP[lane + 32 * jj][j] : 0.f;
+                            }
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) {
+                                const float ks = KS[(cr + r) * CC + j];
+#pragma unroll
+                                for (int jj = 0; jj < 2; ++jj) {
+                                    if (J >= 2 && jj == 0) continue;
+                                    pa[r][jj] = fmaf(dA_[jj], ks, pa[r][jj]);
+                                    pp[r][jj] = fmaf(dP_[jj], ks, pp[r][jj]);
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+#pragma unroll
+                            for (int jj = 0; jj < 2; ++jj) {
+                                if (J >= 2 && jj == 0) continue;
+                                const int c = cr + r, i = lane + 32 * jj;
+                                // blocks past i contribute 0; the clamp keeps their factor finite
+                                const float rho = ex2f(fminf(sm.GT[c][i] - sm.GT[c][16 * J + 15], 120.f));
+                                ta[r][jj] = fmaf(rho, pa[r][jj], ta[r][jj]);
+                                tp[r][jj] = fmaf(rho, pp[r][jj], tp[r][jj]);
+                            }
                     }
 #pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        const float kj = sm.KT[c0 + r][j], gj = sm.GT[c0 + r][j];
+                    for (int r = 0; r < 4; ++r)
 #pragma unroll
                         for (int jj = 0; jj < 2; ++jj) {
-                            if (jj < jj0) continue;
-                            const float ke = kj * ex2f(fminf(gi[r][jj] - gj, 0.f));
-                            ta[r][jj] = fmaf(dA_[jj], ke, ta[r][jj]);
-                            tp[r][jj] = fmaf(dP_[jj], ke, tp[r][jj]);
+                            const int c = cr + r, t = lane + 32 * jj, e = c * CC + t;
+                            DKT[e] += ta[r][jj];
+                            DQT[e] += tp[r][jj];
+                            DGT[e] += sm.KT[c][t] * ta[r][jj] + sm.QT[c][t] * tp[r][jj];
                         }
-                    }
                 }
-#pragma unroll
-                for (int r = 0; r < 8; ++r)
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        const int c = c0 + r, t = lane + 32 * jj, e = c * CC + t;
-                        DKT[e] += ta[r][jj];
-                        DQT[e] += tp[r][jj];
-                        DGT[e] += sm.KT[c][t] * ta[r][jj] + sm.QT[c][t] * tp[r][jj];
-                    }
             }
+            __syncthreads();
             {
-                // column side: token t = j; sums over i >= j
-                float gj[8][2], ta[8][2];
-#pragma unroll
-                for (int r = 0; r < 8; ++r)
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        gj[r][jj] = sm.GT[c0 + r][lane + 32 * jj];
-                        ta[r][jj] = 0.f;
-                    }
+                //      Column side (sums over i >= j), reference s = the first token of i's
+                //      block: e^(G_i - G_j) = e^(G_i - G_s) e^(G_s - G_j), the first factor
+                //      in [e^-75, 1], the second <= e^75 (it underflows only where the
+                //      product is below e^-87).  R[c][i] = e^(G_i - G_s) in the ring.
+                float *R = &sm.stg[0][0];
+                for (int e = tid; e < TILE; e += CT) {
+                    const int c = e >> 6, i = e & (CC - 1);
+                    R[e] = ex2f(sm.GT[c][i] - sm.GT[c][i & ~15]);
+                }
+                __syncthreads();
 #pragma unroll 1
-                for (int i = 0; i < CC; ++i) {
-                    const int jj1 = i < 32 ? 1 : 2;  // tokens j = lane + 32 jj <= i only
-                    float dA_[2], dP_[2];
+                for (int rg = 0; rg < 2; ++rg) {
+                    const int cr = c0 + 4 * rg;
+                    float ta[4][2] = {};
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        dA_[jj] = sm.u.m.X[i][lane + 32 * jj];
-                        dP_[jj] = sm.u.m.dP[i][lane + 32 * jj];
+                    for (int I = 0; I < 4; ++I) {
+                        // tokens j = lane + 32 jj: blocks I < 2 hold only i < j for jj = 1
+                        float pa[4][2] = {};
+#pragma unroll 4
+                        for (int i = 16 * I; i < 16 * I + 16; ++i) {
+                            float dA_[2], dP_[2];
+#pragma unroll
+                            for (int jj = 0; jj < 2; ++jj) {
+                                dA_[jj] = (I >= 2 || jj == 0) ? sm.u.m.X[i][lane + 32 * jj] : 0.f;
+                                dP_[jj] = (I >= 2 || jj == 0) ? sm.u.m.dP[i][lane + 32 * jj] : 0.f;
+                            }
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) {
+                                const int c = cr + r;
+                                const float kq = sm.KT[c][i], qq = sm.QT[c][i], rr = R[c * CC + i];
+#pragma unroll
+                                for (int jj = 0; jj < 2; ++jj) {
+                                    if (I < 2 && jj == 1) continue;
+                                    pa[r][jj] = fmaf(fmaf(dA_[jj], kq, dP_[jj] * qq), rr, pa[r][jj]);
+                                }
+                            }
+                        }
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+#pragma unroll
+                            for (int jj = 0; jj < 2; ++jj) {
+                                if (I < 2 && jj == 1) continue;
+                                const int c = cr + r, j = lane + 32 * jj;
+                                // blocks before j contribute 0; the clamp keeps their factor finite
+                                const float sig = ex2f(fminf(sm.GT[c][16 * I] - sm.GT[c][j], 120.f));
+                                ta[r][jj] = fmaf(sig, pa[r][jj], ta[r][jj]);
+                            }
                     }
 #pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        const float ki = sm.KT[c0 + r][i], qi = sm.QT[c0 + r][i], g = sm.GT[c0 + r][i];
+                    for (int r = 0; r < 4; ++r)
 #pragma unroll
                         for (int jj = 0; jj < 2; ++jj) {
-                            if (jj >= jj1) continue;
-                            const float e = ex2f(fminf(g - gj[r][jj], 0.f));
-                            ta[r][jj] = fmaf(fmaf(dA_[jj], ki, dP_[jj] * qi), e, ta[r][jj]);
+                            const int c = cr + r, t = lane + 32 * jj, e = c * CC + t;
+                            DKT[e] += ta[r][jj];
+                            DGT[e] -= sm.KT[c][t] * ta[r][jj];
                         }
-                    }
                 }
-#pragma unroll
-                for (int r = 0; r < 8; ++r)
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        const int c = c0 + r, t = lane + 32 * jj, e = c * CC + t;
-                        DKT[e] += ta[r][jj];
-                        DGT[e] -= sm.KT[c][t] * ta[r][jj];
-                    }
             }
             __syncthreads();
 
@@ -649,8 +816,8 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                 }
 #pragma unroll
                 for (int jj = 0; jj < 2; ++jj) {
-                    sm.red[0][warp][lane + 32 * jj] = pq[jj];
-                    sm.red[1][warp][lane + 32 * jj] = pk[jj];
+                    sm.u.e.red[0][warp][lane + 32 * jj] = pq[jj];
+                    sm.u.e.red[1][warp][lane + 32 * jj] = pk[jj];
                 }
             }
             __syncthreads();
@@ -658,8 +825,8 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                 const int a = tid >> 6, t = tid & (CC - 1);
                 float s = 0.f;
 #pragma unroll
-                for (int w = 0; w < CW; ++w) s += sm.red[a][w][t];
-                sm.red[a][0][t] = s;
+                for (int w = 0; w < CW; ++w) s += sm.u.e.red[a][w][t];
+                sm.u.e.red[a][0][t] = s;
             }
             __syncthreads();
 #pragma unroll 1
@@ -672,7 +839,7 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                         const int c = c0 + r, t = lane + 32 * jj;
                         const float xh = a ? sm.KT[c][t] : sm.QT[c][t];
                         const float rn = a ? sm.rk[t] : sm.rq[t];
-                        sm.u.e.o1[t][c] = rn * (DXT[c * CC + t] - xh * sm.red[a][0][t]);
+                        sm.u.e.o1[t][c] = rn * (DXT[c * CC + t] - xh * sm.u.e.red[a][0][t]);
                     }
                 __syncthreads();
                 float *dst = a ? p.dk : p.dq;
@@ -688,8 +855,8 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                 __syncthreads();
             }
             {
-                float da = 0.f;
-#pragma unroll 1
+                float da = 0.f, dxs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
                 for (int i = 0; i < CC / CW; ++i) {
                     const int t = warp + CW * i;
                     if (t >= L) continue;
@@ -703,12 +870,14 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                         const float dl = sm.u.e.o0[t][c];
                         const float dx = open ? -dl * ea / (1.f + expf(-x)) : 0.f;
                         p.dg[row + c] = dx;
-                        sm.pacc[warp][c] += dx;
+                        dxs[m] += dx;
                         da += open ? dl * z : 0.f;
                     }
                 }
+#pragma unroll
+                for (int m = 0; m < 4; ++m) PACC[warp * (kHead + 1) + lane + 32 * m] += dxs[m];
                 da = wsum(da);
-                if (lane == 0) sm.pacc[warp][kHead] += da;
+                if (lane == 0) PACC[warp * (kHead + 1) + kHead] += da;
                 if (tid < L) {
                     const float bt = sm.b[tid];
                     p.dbeta[(size_t)(tok + tid) * p.H + h] = sm.db[tid] * bt * (1.f - bt);
@@ -724,7 +893,7 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
         if (tid <= kHead) {
             float acc = 0.f;
 #pragma unroll
-            for (int w = 0; w < CW; ++w) acc += sm.pacc[w][tid];
+            for (int w = 0; w < CW; ++w) acc += PACC[w * (kHead + 1) + tid];
             p.part[(size_t)u * (kHead + 1) + tid] = acc;
         }
     }
