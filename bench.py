@@ -64,6 +64,7 @@ def parse():
     # profiling aids: a smaller batch / sequence of the same workload (default: the full one)
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--seqlen", type=int, default=None)
+    ap.add_argument("--heads", type=int, default=None)
     # the decode step (one token per sequence, state in HBM) instead of the prefill
     ap.add_argument("--op", default="prefill", choices=["prefill", "decode", "backward"])
     ap.add_argument("--bwd-schedule", default="chunked", choices=["chunked", "token"],
@@ -78,7 +79,9 @@ def parse():
         WORKLOAD["B"] = a.batch
     if a.seqlen:
         WORKLOAD["T"] = a.seqlen
-    if a.batch or a.seqlen:
+    if a.heads:
+        WORKLOAD["H"] = a.heads
+    if a.batch or a.seqlen or a.heads:
         WORKLOAD["name"] = f"long_B{WORKLOAD['B']}_T{WORKLOAD['T']}_H{WORKLOAD['H']}_g2"
     return a
 

@@ -24,9 +24,9 @@
 // instantiation, one launch before this one).  Schedule: one CTA of 512 threads per
 // (sequence, head), persistent over the units, chunks in reverse; everything is fp32
 // on the CUDA cores.  The activations (q^, k^, G; channel-major) and the 64 x 64
-// matrices live in shared memory; the 64 x 128 tiles of a chunk (dO, Y, U, dU, dY,
-// their transposes, k^ Gam, q^ Gam, K', the gradient accumulators) and dS live in a
-// per-CTA scratch region of global memory that stays in L2.  The products stream
+// matrices live in shared memory; the 64 x 128 tiles of a chunk (dO, Y, dU, dY, the
+// transposes of dO, Y, U and dY, k^ Gam, q^ Gam, K', the gradient accumulators) and dS
+// live in a per-CTA scratch region of global memory (L2-resident as far as it fits).  The products stream
 // their operands from there through a two-slab shared-memory ring filled by cp.async
 // (the copy of slab s + 1 in flight while slab s is used), so that L2 latency is not
 // paid per load.  Every product is a register-blocked loop whose second operand is
@@ -76,12 +76,15 @@ struct CSmem {
     float eGL[kHead], G2L[kHead], dGL[kHead], extra[kHead], dtb[kHead];
 };
 
-// Per-CTA scratch (floats): the tiles in the order of these offsets.
+// Per-CTA scratch (floats): the tiles in the order of these offsets.  The gradient
+// accumulators reuse the tiles of operands that are dead by the time they are first
+// written (phase 11): dk^ that of Y (last read in phase 7), dq^ that of K' (8), dG that
+// of dU (10).  A smaller footprint keeps more of the scratch in L2.
 enum : int {
     S_DO = 0, S_DOT = TILE, S_KGT = 2 * TILE, S_QGT = 3 * TILE, S_KPT = 4 * TILE, S_Y = 5 * TILE,
-    S_YT = 6 * TILE, S_U = 7 * TILE, S_UT = 8 * TILE, S_DU = 9 * TILE, S_DY = 10 * TILE,
-    S_DYT = 11 * TILE, S_DKT = 12 * TILE, S_DQT = 13 * TILE, S_DGT = 14 * TILE, S_DS = 15 * TILE,
-    S_PACC = 15 * TILE + ST,  // per-warp partial ddt_bias (0..127) and dA_log (128)
+    S_YT = 6 * TILE, S_UT = 7 * TILE, S_DU = 8 * TILE, S_DY = 9 * TILE, S_DYT = 10 * TILE,
+    S_DS = 11 * TILE, S_DKT = S_Y, S_DQT = S_KPT, S_DGT = S_DU,
+    S_PACC = 11 * TILE + ST,  // per-warp partial ddt_bias (0..127) and dA_log (128)
     S_FLOATS = S_PACC + CW * (kHead + 1)
 };
 
@@ -218,7 +221,7 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     float *scr = p.scratch + (size_t)blockIdx.x * S_FLOATS;
     float *DO = scr + S_DO, *DOT = scr + S_DOT, *KGT = scr + S_KGT, *QGT = scr + S_QGT;
-    float *KPT = scr + S_KPT, *Y = scr + S_Y, *YT = scr + S_YT, *U = scr + S_U, *UT = scr + S_UT;
+    float *KPT = scr + S_KPT, *Y = scr + S_Y, *YT = scr + S_YT, *UT = scr + S_UT;
     float *DU = scr + S_DU, *DY = scr + S_DY, *DYT = scr + S_DYT, *DKT = scr + S_DKT;
     float *DQT = scr + S_DQT, *DGT = scr + S_DGT, *DS = scr + S_DS, *PACC = scr + S_PACC;
     const int r0 = 4 * warp;  // rows of this warp in the 64-row products
@@ -454,7 +457,6 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int t = r0 + r, vc = lane + 32 * j;
-                        U[t * kHead + vc] = acc[r][j];
                         UT[vc * CC + t] = acc[r][j];
                     }
             }
