@@ -296,7 +296,9 @@ int kda_last_launch_count(void);
 
 /* Diagnostic: the error word the kernels set when one of their bounded waits
  * gave up (0 = none; the kernel then skipped the rest of its work and returned
- * without trapping).  Synchronous (reads device memory); reset != 0 clears it. */
+ * without trapping).  This covers the checkpoint launch of a chunked kda_bwd too, whose
+ * gradients are then not valid.  Synchronous (reads device memory); reset != 0
+ * clears it. */
 int kda_device_status(int reset);
 
 /* Schedule of the forward kernel, process-wide (returns the previous one, or
@@ -331,7 +333,8 @@ int kda_set_bwd_schedule(int mode);
 int kda_last_schedule(void);
 
 /* Testing hook for the failure path (no counterpart on the pages): the next forward
- * launch (kda_fwd, kda_fwd_ex, kda_fwd_host) starts as if one of its CTAs had
+ * launch (kda_fwd, kda_fwd_ex, kda_fwd_host, or the checkpoint launch of a chunked
+ * kda_bwd) starts as if one of its CTAs had
  * already given up a bounded wait with `code` (1..255).  Every CTA of that launch
  * then returns at its start without writing out or the final state, exactly as
  * the CTAs that start after a real failure do, and kda_device_status reports

@@ -97,6 +97,21 @@ __device__ __forceinline__ float ex2f(float x)
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 *p, size_t i) { return __bfloat162float(p[i]); }
 
+// L2 policy for inputs read once per chunk: evicted before the scratch tiles.
+__device__ __forceinline__ uint64_t evict_first_policy()
+{
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+__device__ __forceinline__ float bf_once(const __nv_bfloat16 *p, size_t i, uint64_t pol)
+{
+    unsigned short x;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.b16 %0, [%1], %2;" : "=h"(x) : "l"(p + i), "l"(pol));
+    return __bfloat162float(__ushort_as_bfloat16(x));
+}
+
 __device__ __forceinline__ float wsum(float x)
 {
 #pragma unroll
@@ -228,6 +243,7 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
     const int c0 = 8 * warp;  // rows (channels) of this warp in the 128-row products
     const int64_t units = p.N * p.H;
     const size_t rs = (size_t)p.H * kHead;  // row stride of the [tokens, H, 128] tensors
+    const uint64_t once = evict_first_policy();
 
     for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
         const int64_t sq = u / p.H, h = u % p.H;
@@ -262,8 +278,8 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     const int c = lane + 32 * m;
-                    qv[m] = in ? bf(p.q, row + c) : 0.f;
-                    kv[m] = in ? bf(p.k, row + c) : 0.f;
+                    qv[m] = in ? bf_once(p.q, row + c, once) : 0.f;
+                    kv[m] = in ? bf_once(p.k, row + c, once) : 0.f;
                     gv[m] = in ? bf(p.g, row + c) : 0.f;
                     s2q = fmaf(qv[m], qv[m], s2q);
                     s2k = fmaf(kv[m], kv[m], s2k);
@@ -281,12 +297,12 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                     sm.QT[c][t] = qv[m] * rq;
                     sm.KT[c][t] = kv[m] * rk;
                     sm.GT[c][t] = lam2;
-                    const float d = in ? bf(p.dout, row + c) : 0.f;
+                    const float d = in ? bf_once(p.dout, row + c, once) : 0.f;
                     DO[t * kHead + c] = d;
                     DOT[c * CC + t] = d;
                 }
                 if (lane == 0) {
-                    sm.b[t] = in ? 1.f / (1.f + expf(-bf(p.beta, (size_t)(tok + t) * p.H + h))) : 0.f;
+                    sm.b[t] = in ? 1.f / (1.f + expf(-bf_once(p.beta, (size_t)(tok + t) * p.H + h, once))) : 0.f;
                     sm.rq[t] = rq;
                     sm.rk[t] = rk;
                 }
@@ -296,23 +312,11 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                 (&sm.u.m.PT[0][0])[i] = 0.f;
             }
             if (n > 0) {
-                // the next chunk's state and input rows towards L2 while this one computes:
-                // 512 lines of the state, 2 lines per row of q, k, g, v, dO, 1 per beta
-                const float *Sn = S0 - ckstride;
-                const int64_t tn = tok - CC;
-                for (int x = tid; x < 512 + 5 * 2 * CC + CC; x += CT) {
-                    const void *a;
-                    if (x < 512) {
-                        a = Sn + 32 * x;
-                    } else if (x < 512 + 10 * CC) {
-                        const int y = x - 512, w = y / (2 * CC), t = (y >> 1) % CC;
-                        const __nv_bfloat16 *base = w == 0 ? p.q : w == 1 ? p.k : w == 2 ? p.g : w == 3 ? p.v : p.dout;
-                        a = base + (size_t)(tn + t) * rs + hb + 64 * (y & 1);
-                    } else {
-                        a = p.beta + (size_t)(tn + (x - 512 - 10 * CC)) * p.H + h;
-                    }
-                    asm volatile("prefetch.global.L2 [%0];" ::"l"(a));
-                }
+                // the next chunk's state towards L2 while this one computes (512 lines); the
+                // input rows are read once, with the evict-first policy, and not prefetched
+                // (prefetching them displaced scratch tiles: measured slower)
+                const float *Sn = S0 - ckstride;  // 16384 floats: line tid of 512
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(Sn + 32 * tid));
             }
             __syncthreads();
 
@@ -435,7 +439,7 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int t = r0 + r, vc = lane + 32 * j;
-                        const float vin = t < L ? bf(p.v, (size_t)(tok + t) * rs + hb + vc) : 0.f;
+                        const float vin = t < L ? bf_once(p.v, (size_t)(tok + t) * rs + hb + vc, once) : 0.f;
                         const float y = vin - acc[r][j];
                         Y[t * kHead + vc] = y;
                         YT[vc * CC + t] = y;
@@ -866,7 +870,7 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
                         const int c = lane + 32 * m;
-                        const float x = bf(p.g, row + c) + sm.dtb[c];
+                        const float x = bf_once(p.g, row + c, once) + sm.dtb[c];
                         const float z = -ea * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))));
                         const bool open = z >= p.lower_bound;  // the clamp is not holding
                         const float dl = sm.u.e.o0[t][c];
