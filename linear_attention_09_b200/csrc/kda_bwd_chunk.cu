@@ -95,6 +95,23 @@ __device__ __forceinline__ float ex2f(float x)
     return y;
 }
 
+__device__ __forceinline__ float lg2f(float x)
+{
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// softplus(x) = max(x, 0) + ln(1 + e^-|x|) in the base-2 hardware functions (relative
+// error ~1e-6, far inside the gradients' bars; where e^-|x| < 2^-24 the second term,
+// then below 6e-8, rounds away against max(x, 0) > 16)
+__device__ __forceinline__ float softplus_f(float x)
+{
+    return fmaxf(x, 0.f) + 0.6931471805599453f * lg2f(1.f + ex2f(-fabsf(x) * kL2e));
+}
+
+__device__ __forceinline__ float sigmoid_f(float x) { return 1.f / (1.f + ex2f(-x * kL2e)); }
+
 __device__ __forceinline__ float bf(const __nv_bfloat16 *p, size_t i) { return __bfloat162float(p[i]); }
 
 // L2 policy for inputs read once per chunk: evicted before the scratch tiles.
@@ -291,7 +308,7 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                     float lam2 = 0.f;
                     if (in) {
                         const float x = gv[m] + sm.dtb[c];
-                        const float sp = fmaxf(x, 0.f) + log1pf(expf(-fabsf(x)));  // softplus
+                        const float sp = softplus_f(x);
                         lam2 = fmaxf(p.lower_bound, -ea * sp) * kL2e;
                     }
                     sm.QT[c][t] = qv[m] * rq;
@@ -302,7 +319,7 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                     DOT[c * CC + t] = d;
                 }
                 if (lane == 0) {
-                    sm.b[t] = in ? 1.f / (1.f + expf(-bf_once(p.beta, (size_t)(tok + t) * p.H + h, once))) : 0.f;
+                    sm.b[t] = in ? sigmoid_f(bf_once(p.beta, (size_t)(tok + t) * p.H + h, once)) : 0.f;
                     sm.rq[t] = rq;
                     sm.rk[t] = rk;
                 }
@@ -871,10 +888,10 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                     for (int m = 0; m < 4; ++m) {
                         const int c = lane + 32 * m;
                         const float x = bf_once(p.g, row + c, once) + sm.dtb[c];
-                        const float z = -ea * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))));
+                        const float z = -ea * softplus_f(x);
                         const bool open = z >= p.lower_bound;  // the clamp is not holding
                         const float dl = sm.u.e.o0[t][c];
-                        const float dx = open ? -dl * ea / (1.f + expf(-x)) : 0.f;
+                        const float dx = open ? -dl * ea * sigmoid_f(x) : 0.f;
                         p.dg[row + c] = dx;
                         dxs[m] += dx;
                         da += open ? dl * z : 0.f;

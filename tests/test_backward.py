@@ -170,6 +170,21 @@ def test_more_units_than_resident_ctas():
         check(run_gpu(inp, dO, dSf, schedule=sch), ref, inp)
 
 
+def test_decay_at_the_lower_bound():
+    """Every token of half the channels at lam = lower_bound = -5 (g far above the clamp),
+    the other half with weak decay: the per-block factors of the chunked schedule reach
+    their widest range there (e^(+-75) across a 16-token block) and must stay finite."""
+    inp, dO, dSf = case(T=300, B=1, H=2, init="f32", seed=12)
+    g = inp.g.float()
+    g[..., 0::2] = 20.0 + 0.1 * g[..., 0::2]   # softplus ~ 20: z << -5, the clamp holds
+    g[..., 1::2] = -6.0 + 0.1 * g[..., 1::2]   # softplus ~ 2.5e-3: weak decay
+    inp.g = g.to(torch.bfloat16)
+    inp.lower_bound = -5.0
+    ref = oracle.backward_inputs(inp, dO, dSf, want_dlam=True)
+    for sch in SCHEDULES:
+        check(run_gpu(inp, dO, dSf, schedule=sch), ref, inp)
+
+
 @pytest.mark.parametrize("sch", SCHEDULES)
 def test_zero_length(sch):
     """T = 0: every output is the pass-through of dL/dS_final (or zeros)."""
