@@ -76,14 +76,15 @@ struct CSmem {
     float eGL[kHead], G2L[kHead], dGL[kHead], extra[kHead], dtb[kHead];
 };
 
-// Per-CTA scratch (floats): the tiles in the order of these offsets.  The gradient
+// Per-CTA scratch (floats): the tiles in the order of these offsets.  Two gradient
 // accumulators reuse the tiles of operands that are dead by the time they are first
-// written (phase 11): dk^ that of Y (last read in phase 7), dq^ that of K' (8), dG that
-// of dU (10).  A smaller footprint keeps more of the scratch in L2.
+// written (phase 11): dq^ that of K' (last read in phase 8), dG that of dU (10).  Y
+// itself never leaves the SM (phase 7 reads it from the operand ring).  A smaller
+// footprint keeps more of the scratch in L2.
 enum : int {
-    S_DO = 0, S_DOT = TILE, S_KGT = 2 * TILE, S_QGT = 3 * TILE, S_KPT = 4 * TILE, S_Y = 5 * TILE,
+    S_DO = 0, S_DOT = TILE, S_KGT = 2 * TILE, S_QGT = 3 * TILE, S_KPT = 4 * TILE, S_DKT = 5 * TILE,
     S_YT = 6 * TILE, S_UT = 7 * TILE, S_DU = 8 * TILE, S_DY = 9 * TILE, S_DYT = 10 * TILE,
-    S_DS = 11 * TILE, S_DKT = S_Y, S_DQT = S_KPT, S_DGT = S_DU,
+    S_DS = 11 * TILE, S_DQT = S_KPT, S_DGT = S_DU,
     S_PACC = 11 * TILE + ST,  // per-warp partial ddt_bias (0..127) and dA_log (128)
     S_FLOATS = S_PACC + CW * (kHead + 1)
 };
@@ -253,7 +254,8 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     float *scr = p.scratch + (size_t)blockIdx.x * S_FLOATS;
     float *DO = scr + S_DO, *DOT = scr + S_DOT, *KGT = scr + S_KGT, *QGT = scr + S_QGT;
-    float *KPT = scr + S_KPT, *Y = scr + S_Y, *YT = scr + S_YT, *UT = scr + S_UT;
+    float *KPT = scr + S_KPT, *YT = scr + S_YT, *UT = scr + S_UT;
+    float *ring = &sm.stg[0][0];  // the operand ring as one [64][128] tile between products
     float *DU = scr + S_DU, *DY = scr + S_DY, *DYT = scr + S_DYT, *DKT = scr + S_DKT;
     float *DQT = scr + S_DQT, *DGT = scr + S_DGT, *DS = scr + S_DS, *PACC = scr + S_PACC;
     const int r0 = 4 * warp;  // rows of this warp in the 64-row products
@@ -291,13 +293,19 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                 const int t = warp + CW * i;
                 const bool in = t < L;
                 const size_t row = (size_t)(tok + t) * rs + hb;
-                float qv[4], kv[4], gv[4], s2q = 0.f, s2k = 0.f;
+                // every load of the token first, so that they share one round trip
+                float qv[4], kv[4], gv[4], dv[4], s2q = 0.f, s2k = 0.f;
 #pragma unroll
                 for (int m = 0; m < 4; ++m) {
                     const int c = lane + 32 * m;
                     qv[m] = in ? bf_once(p.q, row + c, once) : 0.f;
                     kv[m] = in ? bf_once(p.k, row + c, once) : 0.f;
                     gv[m] = in ? bf(p.g, row + c) : 0.f;
+                    dv[m] = in ? bf_once(p.dout, row + c, once) : 0.f;
+                }
+                const float braw = (in && lane == 0) ? bf_once(p.beta, (size_t)(tok + t) * p.H + h, once) : 0.f;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
                     s2q = fmaf(qv[m], qv[m], s2q);
                     s2k = fmaf(kv[m], kv[m], s2k);
                 }
@@ -314,12 +322,11 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                     sm.QT[c][t] = qv[m] * rq;
                     sm.KT[c][t] = kv[m] * rk;
                     sm.GT[c][t] = lam2;
-                    const float d = in ? bf_once(p.dout, row + c, once) : 0.f;
-                    DO[t * kHead + c] = d;
-                    DOT[c * CC + t] = d;
+                    DO[t * kHead + c] = dv[m];
+                    DOT[c * CC + t] = dv[m];
                 }
                 if (lane == 0) {
-                    sm.b[t] = in ? sigmoid_f(bf_once(p.beta, (size_t)(tok + t) * p.H + h, once)) : 0.f;
+                    sm.b[t] = in ? sigmoid_f(braw) : 0.f;
                     sm.rq[t] = rq;
                     sm.rk[t] = rk;
                 }
@@ -458,7 +465,7 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
                         const int t = r0 + r, vc = lane + 32 * j;
                         const float vin = t < L ? bf_once(p.v, (size_t)(tok + t) * rs + hb + vc, once) : 0.f;
                         const float y = vin - acc[r][j];
-                        Y[t * kHead + vc] = y;
+                        ring[t * kHead + vc] = y;  // Y stays in the (now free) ring for phase 7
                         YT[vc * CC + t] = y;
                     }
             }
@@ -467,12 +474,8 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             // ---- 7. U = M^-1 Diag(b) Y ----
             {
                 float acc[4][4] = {};
-                staged(sm.stg, CC / 16, [&](int s, float *buf) { stage_rows(buf, Y + s * 16 * kHead, 16 * kHead); },
-                       [&](const float *buf, int s) {
-                           const int k0 = 16 * s, k1 = min(k0 + 16, r0 + 4);
-                           mm(acc, 0, k1 - k0, [&](int r, int k) { return sm.u.m.Mi[r0 + r][k0 + k] * sm.b[k0 + k]; },
-                              [&](int k, int jj) { return buf[k * kHead + lane + 32 * jj]; });
-                       });
+                mm(acc, 0, r0 + 4, [&](int r, int j) { return sm.u.m.Mi[r0 + r][j] * sm.b[j]; },
+                   [&](int j, int jj) { return ring[j * kHead + lane + 32 * jj]; });
 #pragma unroll
                 for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -505,19 +508,18 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
 #pragma unroll
                 for (int r = 0; r < 4; ++r)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) DU[(r0 + r) * kHead + lane + 32 * j] = acc[r][j];
+                    for (int j = 0; j < 4; ++j) {
+                        DU[(r0 + r) * kHead + lane + 32 * j] = acc[r][j];  // for phase 10
+                        ring[(r0 + r) * kHead + lane + 32 * j] = acc[r][j];  // for phase 9
+                    }
             }
             __syncthreads();
 
             // ---- 9. dY = Diag(b) M^-T dU (= dv) ----
             {
                 float acc[4][4] = {};
-                staged(sm.stg, CC / 16, [&](int s, float *buf) { stage_rows(buf, DU + s * 16 * kHead, 16 * kHead); },
-                       [&](const float *buf, int s) {
-                           const int k0 = 16 * s, lo = max(r0 - k0, 0);
-                           mm(acc, lo, 16, [&](int r, int k) { return sm.u.m.Mi[k0 + k][r0 + r]; },
-                              [&](int k, int j) { return buf[k * kHead + lane + 32 * j]; });
-                       });
+                mm(acc, r0, CC, [&](int r, int i) { return sm.u.m.Mi[i][r0 + r]; },
+                   [&](int i, int j) { return ring[i * kHead + lane + 32 * j]; });
 #pragma unroll
                 for (int r = 0; r < 4; ++r)
 #pragma unroll
