@@ -16,21 +16,23 @@
 //   dM^-1 = dT Diag(b), db_j = sum_i dT_ij M^-1_ij;  dM = -M^-T dM^-1 M^-T
 //   dA = Diag(b) dM (strict lower), db_i += sum_j dM_ij A_ij
 // then through the decay-weighted products A and P into dq^, dk^ and dG (the factor
-// e^(G_i - G_j) evaluated per channel, so that no factor leaves the fp32 range), and
-// dlam = the reverse cumulative sum of dG over the chunk, followed by the gradients of
-// the L2 norms, the sigmoid and the gate as in the token-level backward.
+// e^(G_i - G_j) split at reference tokens of 16-token blocks, so that every factor stays
+// in the fp32 range), and dlam = the reverse cumulative sum of dG over the chunk,
+// followed by the gradients of the L2 norms, the sigmoid and the gate as in the
+// token-level backward.
 //
 // The states before every chunk come from the forward kernel (its checkpoint
 // instantiation, one launch before this one).  Schedule: one CTA of 512 threads per
 // (sequence, head), persistent over the units, chunks in reverse; everything is fp32
 // on the CUDA cores.  The activations (q^, k^, G; channel-major) and the 64 x 64
-// matrices live in shared memory; the 64 x 128 tiles of a chunk (dO, Y, dU, dY, the
+// matrices live in shared memory; the 64 x 128 tiles of a chunk (dO, dU, dY, the
 // transposes of dO, Y, U and dY, k^ Gam, q^ Gam, K', the gradient accumulators) and dS
-// live in a per-CTA scratch region of global memory (L2-resident as far as it fits).  The products stream
-// their operands from there through a two-slab shared-memory ring filled by cp.async
-// (the copy of slab s + 1 in flight while slab s is used), so that L2 latency is not
-// paid per load.  Every product is a register-blocked loop whose second operand is
-// read along its rows by consecutive lanes, so each operand that appears in both
+// live in a per-CTA scratch region of global memory (L2-resident as far as it fits).
+// The products stream their operands from there through a two-slab shared-memory ring
+// filled by cp.async (the copy of slab s + 1 in flight while slab s is used), so that
+// L2 latency is not paid per load; Y and dU stay in the ring for the product right
+// after theirs.  Every product is a register-blocked loop whose second operand is read
+// along its rows by consecutive lanes, so each operand that appears in both
 // orientations is stored in both.
 #include <atomic>
 #include <cstddef>
