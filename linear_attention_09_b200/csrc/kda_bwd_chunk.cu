@@ -358,72 +358,52 @@ __global__ void __launch_bounds__(CT, 1) bwdc_kernel(const BwdParams p)
             }
             __syncthreads();
 
-            // ---- 3. (k^ Gam)^T, (q^ Gam)^T, K'^T ----
-            for (int e = tid; e < TILE; e += CT) {
-                const int c = e >> 6, t = e & (CC - 1);
-                const float g2 = sm.GT[c][t], gam = ex2f(g2), kh = sm.KT[c][t];
-                KGT[e] = kh * gam;
-                QGT[e] = sm.QT[c][t] * gam;
-                KPT[e] = kh * ex2f(sm.G2L[c] - g2);
+            // ---- 3. (k^ Gam)^T, (q^ Gam)^T, K'^T; KS[c][j] = k^_j e^(G_e - G_j), e the last
+            //      token of j's 16-token block (in the ring, for phase 4) ----
+            {
+                float *KS = ring;
+                for (int e = tid; e < TILE; e += CT) {
+                    const int c = e >> 6, t = e & (CC - 1);
+                    const float g2 = sm.GT[c][t], gam = ex2f(g2), kh = sm.KT[c][t];
+                    KGT[e] = kh * gam;
+                    QGT[e] = sm.QT[c][t] * gam;
+                    KPT[e] = kh * ex2f(sm.G2L[c] - g2);
+                    KS[e] = kh * ex2f(sm.GT[c][t | 15] - g2);
+                }
             }
+            __syncthreads();
 
-            // ---- 4. A and P in 4 x 4 blocks (a warp per block, lanes over channels) ----
-            for (int blk = warp; blk < 136; blk += CW) {
-                int bi = 0, bj = blk;
-                while (bj > bi) {
-                    bj -= bi + 1;
-                    ++bi;
-                }
-                const int i0 = 4 * bi, j0 = 4 * bj;
-                float v[32];
+            // ---- 4. A and P: A_ij = sum_c (k^_i e^(G_i - G_e)) KS[c][j] with e the last token of
+            //      j's block J (the first factor <= 1 past the block, <= e^75 inside it; KS in
+            //      [e^-75, 1]).  Warp (J, rows i0..i0 + 31, half jq of the block): lane = row i,
+            //      8 columns j each; 12 warps cover every (row, block J <= row's block) ----
+            if (warp < 12) {
+                const int jq = warp & 1, slot = warp >> 1;
+                const int J = slot < 2 ? 0 : slot < 4 ? 1 : slot == 4 ? 2 : 3;
+                const int i0 = slot == 0 ? 0 : slot == 1 ? 32 : slot == 2 ? 16 : slot == 3 ? 48 : slot == 4 ? 32 : 48;
+                const int i = i0 + lane, jb = 16 * J + 8 * jq, eJ = 16 * J + 15;
+                if (i < CC) {  // lanes past row 63 idle; no shuffles below
+                    const float *KS = ring;
+                    float a[8], pp[8];
 #pragma unroll
-                for (int x = 0; x < 32; ++x) v[x] = 0.f;
+                    for (int x = 0; x < 8; ++x) a[x] = pp[x] = 0.f;
+#pragma unroll 4
+                    for (int c = 0; c < kHead; ++c) {
+                        const float rho = ex2f(sm.GT[c][i] - sm.GT[c][eJ]);
+                        const float kr = sm.KT[c][i] * rho, qr = sm.QT[c][i] * rho;
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    const int c = lane + 32 * m;
-                    float gi[4], ki[4], qi[4], gj[4], kj[4];
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        gi[x] = sm.GT[c][i0 + x];
-                        ki[x] = sm.KT[c][i0 + x];
-                        qi[x] = sm.QT[c][i0 + x];
-                        gj[x] = sm.GT[c][j0 + x];
-                        kj[x] = sm.KT[c][j0 + x];
-                    }
-                    // e^(G_i - G_j) = e^(G_i - G_j0) e^(G_j0 - G_j): the first factor <= 1
-                    // (i >= j0), the second <= e^15 (j - j0 <= 3, lam >= -5)
-                    float ka[4], qa[4], kb[4];
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        const float a = ex2f(gi[x] - gj[0]);
-                        ka[x] = ki[x] * a;
-                        qa[x] = qi[x] * a;
-                        kb[x] = x == 0 ? kj[0] : kj[x] * ex2f(gj[0] - gj[x]);
-                    }
-#pragma unroll
-                    for (int ii = 0; ii < 4; ++ii)
-#pragma unroll
-                        for (int jj = 0; jj < 4; ++jj) {
-                            v[ii * 4 + jj] = fmaf(ka[ii], kb[jj], v[ii * 4 + jj]);
-                            v[16 + ii * 4 + jj] = fmaf(qa[ii], kb[jj], v[16 + ii * 4 + jj]);
+                        for (int x = 0; x < 8; ++x) {
+                            const float ks = KS[c * CC + jb + x];
+                            a[x] = fmaf(kr, ks, a[x]);
+                            pp[x] = fmaf(qr, ks, pp[x]);
                         }
-                }
-                // reduce-scatter over the lanes: lane l ends with the total of value l
-#pragma unroll
-                for (int hh = 16; hh >= 1; hh >>= 1) {
-                    const bool up = lane & hh;
-#pragma unroll
-                    for (int x = 0; x < hh; ++x) {
-                        const float send = up ? v[x] : v[x + hh];
-                        const float keep = up ? v[x + hh] : v[x];
-                        v[x] = keep + __shfl_xor_sync(FULL, send, hh);
                     }
-                }
-                const int i = i0 + ((lane >> 2) & 3), j = j0 + (lane & 3);
-                if (lane < 16) {
-                    if (j < i) sm.u.m.A[i][j] = v[0];
-                } else if (j <= i) {
-                    sm.u.m.PT[j][i] = v[0];
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) {
+                        const int j = jb + x;
+                        if (j < i) sm.u.m.A[i][j] = a[x];
+                        if (j <= i) sm.u.m.PT[j][i] = pp[x];
+                    }
                 }
             }
             __syncthreads();
