@@ -93,3 +93,51 @@ def test_three_tf32_products_recover_the_adjoints():
     got = cb.backward_inputs(inp, dO, dSf, prec=dict(BWD_PLAN, APb="tf32x3"))
     for n in BARS:
         assert _rel(got[n], ref[n]) <= 1e-3, (n, _rel(got[n], ref[n]))
+
+
+def _split_factors_f32(G, ref_of_j_block, clamp=120.0):
+    """e^(G_i - G_j) for j <= i as the product of two float32 factors split at the
+    reference token r = ref(block of j or i), in base 2 with the exponent clamped as the
+    chunked backward kernel does; returns the [C, C] products in float64."""
+    L2E = np.float32(1.4426950408889634)
+    G2 = (G.astype(np.float32) * L2E).astype(np.float32)
+    C = G.shape[0]
+    out = np.zeros((C, C))
+    with np.errstate(over="ignore", invalid="ignore", under="ignore"):
+        for i in range(C):
+            for j in range(i + 1):
+                r = ref_of_j_block(i, j)
+                a = np.exp2(np.minimum(np.float32(G2[i] - G2[r]), np.float32(clamp)), dtype=np.float32)
+                b = np.exp2(np.minimum(np.float32(G2[r] - G2[j]), np.float32(clamp)), dtype=np.float32)
+                out[i, j] = float(np.float32(a * b))
+    return out
+
+
+@pytest.mark.parametrize("side", ["row", "column"])
+def test_block_reference_split_stays_in_fp32_range(side):
+    """The chunked backward kernel splits e^(G_i - G_j) at a reference token of a 16-token
+    block (row side and A/P: the last token of j's block; column side: the first token of
+    i's block).  At the steepest decay the operator allows (lam = lower_bound = -5 on
+    every token) both factors must stay finite and their product must match e^(G_i - G_j)
+    to float32 accuracy wherever it is above float32's normal range; below it, the
+    product may flush to zero.  A wrong reference (e.g. a chunk-wide one) overflows."""
+    C = 64
+    lam = np.full(C, -5.0)
+    G = np.cumsum(lam)
+    exact = np.exp(G[:, None] - G[None, :])
+    if side == "row":
+        ref = lambda i, j: (j // 16) * 16 + 15
+    else:
+        ref = lambda i, j: (i // 16) * 16
+    got = _split_factors_f32(G, ref)
+    lower = np.tril(np.ones((C, C), bool))
+    assert np.all(np.isfinite(got[lower]))
+    big = lower & (exact > 1e-30)
+    rel = np.abs(got[big] - exact[big]) / exact[big]
+    # the exponent G*log2(e) is rounded to float32 (|G| <= 320): ~2e-5 relative at most
+    assert rel.max() < 1e-4, rel.max()
+    small = lower & (exact <= 1e-30)
+    assert np.all(got[small] <= 1e-29)
+    # a chunk-wide reference (token 0) is what the blocks avoid: its factors overflow
+    chunk_ref = _split_factors_f32(G, lambda i, j: 0, clamp=1e9)
+    assert not np.all(np.isfinite(chunk_ref[lower]))
