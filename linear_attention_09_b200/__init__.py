@@ -382,7 +382,10 @@ def kda_bwd(q, k, v, g, beta, scale, A_log, dt_bias, lower_bound, d_out, initial
     Returns a dict of fp32 tensors: dq, dk, dg [B,T,H,128], dv [B,T,H,128], dbeta
     [B,T,H], dA_log [H], ddt_bias [H,128] and dS0 [N,H,128,128] (None unless
     ``want_d_initial_state``).  ``workspace`` is a CUDA uint8 tensor of at least
-    ``kda_bwd_workspace_size`` bytes (allocated here if None).
+    ``kda_bwd_workspace_size`` bytes (allocated here if None).  The schedule is the
+    process-wide one of ``kda_set_bwd_schedule`` ("chunked" by default: three kernel
+    launches, the forward kernel's chunk checkpoints, the chunked reverse and a
+    parameter reduction).
     """
     if d_out is None:
         raise ValueError("d_out is required")
